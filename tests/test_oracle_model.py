@@ -1,0 +1,356 @@
+"""Pins of the oracle forward pass: closed forms, brute force on tiny inputs,
+structured special cases and invariants the pages state."""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import model as om
+from oracle import serialize_row, EncodeOptions
+from workloads import weight_specs, rows_config0
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------------ LayerNorm / GELU
+
+
+def test_layer_norm_textbook_values():
+    # population z-scores of [1, 2, 3, 4]: std = sqrt(1.25)
+    y = om.layer_norm(np.array([1.0, 2.0, 3.0, 4.0]), np.ones(4), eps=0.0)
+    s = math.sqrt(1.25)
+    np.testing.assert_allclose(y, [-1.5 / s, -0.5 / s, 0.5 / s, 1.5 / s], rtol=0, atol=1e-15)
+
+
+def test_layer_norm_moments_and_affine():
+    rng = np.random.default_rng(0)
+    x = rng.normal(3.0, 5.0, size=(7, 384))
+    y = om.layer_norm(x, np.ones(384), eps=1e-5)
+    np.testing.assert_allclose(y.mean(-1), 0, atol=1e-12)
+    var = x.var(-1)
+    np.testing.assert_allclose(y.var(-1), var / (var + 1e-5), rtol=1e-12)
+    g, b = rng.normal(size=384), rng.normal(size=384)
+    np.testing.assert_allclose(om.layer_norm(x, g, b), y * g + b, rtol=1e-12, atol=1e-12)
+
+
+def test_gelu_is_exact_erf_form():
+    # GELU(x) = x * Phi(x); Phi(1) = 0.8413447460685429 (standard normal CDF)
+    np.testing.assert_allclose(om.gelu(np.array([1.0, -1.0, 0.0])),
+                               [0.8413447460685429, -0.15865525393145707, 0.0], atol=1e-15)
+    # the tanh approximation differs by ~1.5e-4 at x = 1, far beyond this bound
+    assert abs(om.gelu(np.array([3.0]))[0] - 3.0 * 0.9986501019683699) < 1e-14
+
+
+# ------------------------------------------------------------------ RoPE
+
+
+def test_rope_position_zero_identity_and_norm():
+    rng = np.random.default_rng(1)
+    x = rng.normal(size=(50, 3, 64))
+    y = om.rope(x, 10000.0)
+    np.testing.assert_allclose(y[0], x[0], atol=1e-15)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-12)
+
+
+def test_rope_pairing_closed_form():
+    # frequency 0 is theta^0 = 1 rad per position; dim 0 pairs with dim 32
+    L = 9
+    x = np.zeros((L, 1, 64))
+    x[:, 0, 0] = 1.0
+    y = om.rope(x, 160000.0)
+    p = np.arange(L)
+    np.testing.assert_allclose(y[:, 0, 0], np.cos(p), atol=1e-14)
+    np.testing.assert_allclose(y[:, 0, 32], np.sin(p), atol=1e-14)
+    assert np.abs(np.delete(y[:, 0, :], [0, 32], axis=1)).max() == 0
+    x = np.zeros((L, 1, 64))
+    x[:, 0, 32] = 1.0
+    y = om.rope(x, 160000.0)
+    np.testing.assert_allclose(y[:, 0, 0], -np.sin(p), atol=1e-14)
+    np.testing.assert_allclose(y[:, 0, 32], np.cos(p), atol=1e-14)
+    # slowest pair (31, 63) turns at theta^(-62/64) rad per position
+    x = np.zeros((L, 1, 64))
+    x[:, 0, 31] = 1.0
+    y = om.rope(x, 10000.0)
+    w = 10000.0 ** (-62 / 64)
+    np.testing.assert_allclose(y[:, 0, 63], np.sin(p * w), atol=1e-14)
+
+
+def test_rope_relative_position():
+    rng = np.random.default_rng(2)
+    q, k = rng.normal(size=64), rng.normal(size=64)
+    L = 40
+    Q = om.rope(np.tile(q, (L, 1, 1)), 10000.0)[:, 0]
+    K = om.rope(np.tile(k, (L, 1, 1)), 10000.0)[:, 0]
+    d1 = Q[10] @ K[3]
+    d2 = Q[30] @ K[23]
+    assert abs(d1 - d2) < 1e-10 and abs(d1 - Q[11] @ K[3]) > 1e-6
+
+
+# ------------------------------------------------------------------ attention
+
+
+def _attention_brute(q, k, v, window):
+    L, H, dh = q.shape
+    out = np.zeros_like(q)
+    for h in range(H):
+        for i in range(L):
+            keys = [j for j in range(L) if window is None or abs(i - j) <= window]
+            s = [sum(q[i, h, c] * k[j, h, c] for c in range(dh)) / math.sqrt(dh) for j in keys]
+            m = max(s)
+            w = [math.exp(t - m) for t in s]
+            z = sum(w)
+            for jj, j in enumerate(keys):
+                out[i, h, :] += (w[jj] / z) * v[j, h, :]
+    return out
+
+
+@pytest.mark.parametrize("window", [None, 0, 2, 5])
+def test_attention_brute_force(window):
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.normal(size=(11, 2, 4)) for _ in range(3))
+    np.testing.assert_allclose(om.attention(q, k, v, window), _attention_brute(q, k, v, window), atol=1e-13)
+
+
+def test_attention_window_covering_row_is_global():
+    rng = np.random.default_rng(4)
+    q, k, v = (rng.normal(size=(65, 6, 64)) for _ in range(3))
+    np.testing.assert_allclose(om.attention(q, k, v, 64), om.attention(q, k, v, None), atol=1e-14)
+    q, k, v = (rng.normal(size=(66, 1, 8)) for _ in range(3))
+    assert np.abs(om.attention(q, k, v, 64) - om.attention(q, k, v, None)).max() > 1e-6
+
+
+def test_attention_uniform_window_average():
+    # zero queries -> equal weights over the 2w+1 (clipped) visible keys
+    L, w = 300, 64
+    rng = np.random.default_rng(5)
+    v = rng.normal(size=(L, 1, 4))
+    z = np.zeros((L, 1, 4))
+    out = om.attention(z, z, v, w)
+    for i in (0, 10, 150, 299):
+        lo, hi = max(0, i - w), min(L, i + w + 1)
+        np.testing.assert_allclose(out[i, 0], v[lo:hi, 0].mean(0), atol=1e-13)
+        assert hi - lo == min(L, i + w + 1) - max(0, i - w)
+    assert min(L, 150 + w + 1) - max(0, 150 - w) == 129
+
+
+# ------------------------------------------------------------------ blocks (tiny dims)
+
+
+def _tiny_weights(d=8, H=2, f=4, hf=6, layers=2):
+    """A structured dict of weights with tiny dims (all zero unless set)."""
+    W = {}
+    for l in range(layers):
+        p = f"enc.{l}."
+        W[p + "attn_norm.g"] = np.ones(d)
+        W[p + "Wqkv"] = np.zeros((3 * d, d))
+        W[p + "Wo"] = np.zeros((d, d))
+        W[p + "mlp_norm.g"] = np.ones(d)
+        W[p + "Wi"] = np.zeros((2 * f, d))
+        W[p + "Wo2"] = np.zeros((d, f))
+    for i in range(2):
+        p = f"head.{i}."
+        for n, s in (("norm1.g", d), ("norm2.g", d)):
+            W[p + n] = np.ones(s)
+        for n, s in (("norm1.b", (d,)), ("norm2.b", (d,)), ("in_proj.W", (3 * d, d)), ("in_proj.b", (3 * d,)),
+                     ("out_proj.W", (d, d)), ("out_proj.b", (d,)), ("linear1.W", (hf, d)), ("linear1.b", (hf,)),
+                     ("linear2.W", (d, hf)), ("linear2.b", (d,))):
+            W[p + n] = np.zeros(s)
+    return W
+
+
+def test_encoder_layer_value_path_and_wo_orientation():
+    # q = k = 0 (uniform attention), v = x, Wo a non-symmetric permutation
+    d, L = 8, 10
+    W = _tiny_weights(d=d)
+    W["enc.1.Wqkv"][2 * d:, :] = np.eye(d)
+    perm = np.roll(np.arange(d), 3)          # out[a] = in[perm[a]]
+    W["enc.1.Wo"][np.arange(d), perm] = 1.0
+    mo = om.ModelOptions(n_heads=2, window=2)
+    rng = np.random.default_rng(6)
+    x = rng.normal(size=(L, d))
+    y = om.encoder_layer(x, W, 1, mo)       # layer 1 is local
+    xn = om.layer_norm(x, np.ones(d))
+    for i in range(L):
+        lo, hi = max(0, i - 2), min(L, i + 3)
+        avg = xn[lo:hi].mean(0)
+        np.testing.assert_allclose(y[i], x[i] + avg[perm], atol=1e-12)
+
+
+def test_encoder_layer0_skips_attention_norm_and_is_global():
+    d, L = 8, 10
+    W = _tiny_weights(d=d)
+    W["enc.0.Wqkv"][2 * d:, :] = np.eye(d)
+    W["enc.0.Wo"][:] = np.eye(d)
+    mo = om.ModelOptions(n_heads=2, window=2)
+    x = np.random.default_rng(7).normal(size=(L, d)) * 3 + 1
+    y = om.encoder_layer(x, W, 0, mo)
+    np.testing.assert_allclose(y, x + x.mean(0), atol=1e-12)  # raw x, all keys
+
+
+def test_encoder_geglu_split_and_orientation():
+    d, f, L = 8, 8, 5                          # Wi square: a transposed read would differ
+    W = _tiny_weights(d=d, f=f)
+    W["enc.1.Wi"][0, 1] = 1.0                  # u_0 = xn_1 (GELU branch, first half)
+    W["enc.1.Wi"][f + 0, 2] = 1.0              # g_0 = xn_2 (gate, second half)
+    W["enc.1.Wo2"][5, 0] = 1.0                 # out_5 = y_0
+    mo = om.ModelOptions(n_heads=2)
+    x = np.random.default_rng(8).normal(size=(L, d))
+    y = om.encoder_layer(x, W, 1, mo)
+    xn = om.layer_norm(x, np.ones(d))
+    expect = x.copy()
+    expect[:, 5] += om.gelu(xn[:, 1]) * xn[:, 2]
+    np.testing.assert_allclose(y, expect, atol=1e-12)
+
+
+def test_encoder_rope_theta_by_layer():
+    # q = k = x projections; a local layer uses theta 10000, a global one 160000
+    d, L = 64, 6
+    W = _tiny_weights(d=d, H=1, f=4)
+    for l in (0, 1):
+        W[f"enc.{l}.Wqkv"][:d] = np.eye(d)
+        W[f"enc.{l}.Wqkv"][d:2 * d] = np.eye(d)
+        W[f"enc.{l}.Wqkv"][2 * d:] = np.eye(d)
+        W[f"enc.{l}.Wo"][:] = np.eye(d)
+    mo = om.ModelOptions(n_heads=1, window=100)
+    x = np.random.default_rng(9).normal(size=(L, d))
+    for l, theta in ((0, 160000.0), (1, 10000.0)):
+        h = x if l == 0 else om.layer_norm(x, np.ones(d))
+        q = om.rope(h[:, None, :], theta)
+        ref = x + om.attention(q, q, h[:, None, :])[:, 0]
+        np.testing.assert_allclose(om.encoder_layer(x, W, l, mo), ref, atol=1e-12)
+
+
+def test_head_layer_biases_and_relu():
+    # in_proj.W = 0: v = b_v for every key, so attention returns b_v exactly
+    d, hf, L = 8, 6, 7
+    W = _tiny_weights(d=d, hf=hf)
+    rng = np.random.default_rng(10)
+    bv = rng.normal(size=d)
+    W["head.0.in_proj.b"][2 * d:] = bv
+    Wo = rng.normal(size=(d, d))
+    W["head.0.out_proj.W"][:] = Wo
+    W["head.0.out_proj.b"][:] = rng.normal(size=d)
+    b1 = np.array([1.0, -2.0, 0.5, -0.1, 3.0, -4.0])
+    W["head.0.linear1.b"][:] = b1
+    W2 = rng.normal(size=(d, hf))
+    W["head.0.linear2.W"][:] = W2
+    W["head.0.linear2.b"][:] = rng.normal(size=d)
+    h = rng.normal(size=(L, d))
+    for act, a in (("relu", np.maximum(b1, 0)), ("gelu", om.gelu(b1))):
+        mo = om.ModelOptions(n_heads=2, head_act=act)
+        y = om.head_layer(h, W, 0, mo)
+        expect = h + Wo @ bv + W["head.0.out_proj.b"] + W2 @ a + W["head.0.linear2.b"]
+        np.testing.assert_allclose(y, expect, atol=1e-12)
+
+
+def test_head_layer_attention_is_global_and_norm1_feeds_it():
+    d, L = 8, 70
+    W = _tiny_weights(d=d)
+    W["head.0.in_proj.W"][2 * d:] = np.eye(d)      # v = LN1(h), q = k = 0
+    W["head.0.out_proj.W"][:] = np.eye(d)
+    g1 = np.linspace(0.5, 2.0, d)
+    W["head.0.norm1.g"][:] = g1
+    W["head.0.norm1.b"][:] = 0.25
+    mo = om.ModelOptions(n_heads=2)
+    h = np.random.default_rng(11).normal(size=(L, d))
+    y = om.head_layer(h, W, 0, mo)
+    a = om.layer_norm(h, g1, 0.25)
+    np.testing.assert_allclose(y, h + a.mean(0), atol=1e-12)
+
+
+def test_scorer_structured():
+    d = 8
+    rng = np.random.default_rng(12)
+    W = {"scorer.norm.g": np.full(d, 2.0), "scorer.norm.b": np.full(d, 0.5),
+         "scorer.linear1.W": np.eye(d), "scorer.linear1.b": np.zeros(d),
+         "scorer.linear2.W": np.eye(d)[3:4], "scorer.linear2.b": np.array([0.7]),
+         "scorer_lin.W": np.eye(d)[6:7], "scorer_lin.b": np.array([-0.2])}
+    hm = rng.normal(size=(4, d))
+    n = om.layer_norm(hm, np.full(d, 2.0), np.full(d, 0.5))
+    np.testing.assert_allclose(om.scorer(hm, W, om.ModelOptions()), om.gelu(n[:, 3]) + 0.7, atol=1e-12)
+    np.testing.assert_allclose(om.scorer(hm, W, om.ModelOptions(scorer="linear")), n[:, 6] - 0.2, atol=1e-12)
+
+
+# ------------------------------------------------------------------ shapes / counts
+
+
+def _golden_counts():
+    out = {}
+    for line in open(os.path.join(GOLD, "param_counts.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        k, v, unit, dec = line.split()
+        out[k] = (float(v), unit, int(dec))
+    return out
+
+
+def test_param_counts_match_pages():
+    n = {name: int(np.prod(shape)) for name, shape, _ in weight_specs()}
+    emb = n["embed.E"]
+    enc = sum(v for k, v in n.items() if k.startswith("enc.") or k == "embed.norm.g")
+    head = sum(v for k, v in n.items() if k.startswith("head.") or k.startswith("scorer."))
+    g = _golden_counts()
+    assert round(emb / 1e6, 0) == g["embedding"][0]
+    assert round(enc / 1e6, 0) == g["non_embedding"][0]
+    assert round((emb + enc) / 1e6, 0) == g["backbone"][0]
+    assert round(head / 1e6, 1) == g["head"][0]
+    total = emb + enc + head
+    # the undocumented, unused act_head is not built, so the total sits just below 144.3M
+    assert g["total"][0] - 0.2 <= total / 1e6 <= g["total"][0]
+    assert abs(total * 4 / 2 ** 20 - g["weights_fp32"][0]) < 1.0
+    # the head's weights are independent of the option count ("The decision head")
+    assert n["scorer.linear2.W"] == 384 and n["head.type_table"] == 3 * 384
+
+
+# ------------------------------------------------------------------ full model invariants
+
+
+def test_window_covering_row_equals_global_model(weights_file):
+    (r,) = rows_config0()
+    e = serialize_row(r, EncodeOptions())
+    a = om.OracleModel(weights_file).logits(e)
+    b = om.OracleModel(weights_file, om.ModelOptions(window=10 ** 6)).logits(e)
+    np.testing.assert_allclose(a, b, atol=1e-13)
+    assert len(e.ids) <= 65
+
+
+def test_marker_only_last_layer_equals_full(weights_file):
+    """"julia1 -- Rust runtime", "Why it is faster": the last head layer needs
+    queries, out-projection and feed-forward only at the markers."""
+    m = om.OracleModel(weights_file)
+    (r,) = rows_config0()
+    e = serialize_row(r, EncodeOptions())
+    W, mo = m.W, m.mo
+    h = m.encode(e.ids) + W["head.type_table"][e.qtype]
+    h = om.head_layer(h, W, 0, mo)
+    full = om.head_layer(h, W, 1, mo)[e.mask_pos]
+    # marker-only evaluation written independently: keys/values over all positions
+    p = "head.1."
+    a = om.layer_norm(h, W[p + "norm1.g"], W[p + "norm1.b"])
+    Wi, bi = W[p + "in_proj.W"], W[p + "in_proj.b"]
+    k = a @ Wi[384:768].T + bi[384:768]
+    v = a @ Wi[768:].T + bi[768:]
+    hm = h[e.mask_pos]
+    q = a[e.mask_pos] @ Wi[:384].T + bi[:384]
+    o = np.zeros_like(q)
+    for hh in range(6):
+        sl = slice(64 * hh, 64 * hh + 64)
+        s = q[:, sl] @ k[:, sl].T / 8.0
+        s = np.exp(s - s.max(1, keepdims=True))
+        o[:, sl] = (s / s.sum(1, keepdims=True)) @ v[:, sl]
+    hm = hm + o @ W[p + "out_proj.W"].T + W[p + "out_proj.b"]
+    f = om.layer_norm(hm, W[p + "norm2.g"], W[p + "norm2.b"])
+    hm = hm + np.maximum(f @ W[p + "linear1.W"].T + W[p + "linear1.b"], 0) @ W[p + "linear2.W"].T + W[p + "linear2.b"]
+    np.testing.assert_allclose(full, hm, atol=1e-11)
+
+
+def test_type_row_changes_only_through_type(weights_file):
+    m = om.OracleModel(weights_file)
+    (r,) = rows_config0()
+    e = serialize_row(r, EncodeOptions())
+    enc = m.encode(e.ids)
+    e1 = type(e)(ids=e.ids, mask_pos=e.mask_pos, qtype=1, trunc=0, head_len=e.head_len)
+    za, zb = m.logits(e), m.logits(e1)
+    assert za.shape == (3,) and np.abs(za - zb).max() > 1e-6
+    np.testing.assert_allclose(enc.mean(-1), 0, atol=1e-12)  # final norm output
