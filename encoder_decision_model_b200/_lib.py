@@ -1,0 +1,269 @@
+"""ctypes binding of libjulia_decide.so (argument marshalling only).
+
+Every function here forwards to the C entry point of the same name declared in
+include/julia_decide.h; no step of the forward pass runs in Python.  Device
+buffers are passed as integers or objects with a ``data_ptr()`` method (torch
+tensors); streams as integers or objects with a ``cuda_stream`` attribute.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from pathlib import Path
+
+import numpy as np
+
+LIB_PATH = Path(__file__).resolve().parent / "libjulia_decide.so"
+
+JD_OK, JD_ERR_INVALID_ARG, JD_ERR_OPTION_COUNT, JD_ERR_OVERFLOW, JD_ERR_TOKEN_RANGE = 0, 1, 2, 3, 4
+JD_ERR_CAPACITY, JD_ERR_CUDA, JD_ERR_DEVICE_STATUS, JD_ERR_IO = 5, 6, 7, 8
+JD_PREC_BF16, JD_PREC_FP32 = 0, 1
+JD_SCORER_MLP, JD_SCORER_LINEAR = 0, 1
+JD_ACT_RELU, JD_ACT_GELU = 0, 1
+
+i32p = C.POINTER(C.c_int32)
+f32p = C.POINTER(C.c_float)
+
+
+class jd_row(C.Structure):
+    _fields_ = [("state", i32p), ("n_state", C.c_int32), ("question", i32p), ("n_question", C.c_int32),
+                ("options", C.POINTER(i32p)), ("n_option_ids", i32p), ("k", C.c_int32), ("type", C.c_int32)]
+
+
+class jd_encode_opts(C.Structure):
+    _fields_ = [("max_length", C.c_int32), ("head_budget", C.c_int32), ("strict", C.c_int32),
+                ("bos", C.c_int32), ("eos", C.c_int32), ("mask", C.c_int32), ("vocab", C.c_int32)]
+
+
+class jd_batch(C.Structure):
+    _fields_ = [("n_rows", C.c_int32), ("n_tokens", C.c_int32), ("n_markers", C.c_int32),
+                ("max_row_len", C.c_int32), ("tokens", C.c_void_p), ("cu_seqlens", C.c_void_p),
+                ("mask_pos", C.c_void_p), ("opt_off", C.c_void_p), ("row_type", C.c_void_p),
+                ("head_len", C.c_void_p), ("trunc", C.c_void_p)]
+
+
+class jd_outputs(C.Structure):
+    _fields_ = [("logits", C.c_void_p), ("probs", C.c_void_p), ("choice", C.c_void_p), ("score", C.c_void_p),
+                ("noul", C.c_void_p), ("max_p", C.c_void_p)]
+
+
+class jd_taps(C.Structure):
+    _fields_ = [("encoder_out", C.c_void_p), ("marker_state", C.c_void_p)]
+
+
+class jd_model_config(C.Structure):
+    _fields_ = [("max_tokens", C.c_int32), ("max_rows", C.c_int32), ("max_markers", C.c_int32),
+                ("precision", C.c_int32), ("scorer", C.c_int32), ("head_act", C.c_int32)]
+
+
+class jd_host_outputs(C.Structure):
+    _fields_ = [("logits", f32p), ("probs", f32p), ("choice", i32p), ("score", f32p), ("noul", f32p),
+                ("max_p", f32p), ("n_rows", C.c_int32), ("n_markers", C.c_int32)]
+
+
+class JDError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """Load the CUDA library; raises if it has not been built (no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = Path(os.environ.get("JD_LIB", LIB_PATH))
+    if not path.exists():
+        raise FileNotFoundError(f"{path} is missing: build it with python -m encoder_decision_model_b200.build")
+    L = C.CDLL(str(path))
+    L.jd_last_error.restype = C.c_char_p
+    L.jd_version.restype = C.c_char_p
+    L.jd_serialize.argtypes = [C.POINTER(jd_row), C.c_int32, C.POINTER(jd_encode_opts),
+                               C.POINTER(C.POINTER(jd_batch)), C.POINTER(C.c_int32)]
+    L.jd_batch_free.argtypes = [C.POINTER(jd_batch)]
+    L.jd_batch_free.restype = None
+    L.jd_model_create.argtypes = [C.POINTER(jd_model_config), C.c_char_p, C.c_int, C.POINTER(C.c_void_p)]
+    L.jd_model_destroy.argtypes = [C.c_void_p]
+    L.jd_model_destroy.restype = None
+    L.jd_model_device_bytes.argtypes = [C.c_void_p]
+    L.jd_model_device_bytes.restype = C.c_size_t
+    L.jd_decide.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.POINTER(jd_outputs), C.POINTER(jd_taps), C.c_void_p]
+    L.jd_forward.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.c_void_p, C.c_void_p]
+    L.jd_decide_host.argtypes = [C.c_void_p, C.POINTER(jd_row), C.c_int32, C.POINTER(jd_encode_opts),
+                                 C.POINTER(jd_host_outputs), C.c_void_p]
+    L.jd_decide_packed_host.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.POINTER(jd_host_outputs), C.c_void_p]
+    L.jd_check_status.argtypes = [C.c_void_p]
+    L.jd_set_graph_mode.argtypes = [C.c_void_p, C.c_int]
+    for name in ("jd_serialize", "jd_model_create", "jd_decide", "jd_forward", "jd_decide_host",
+                 "jd_decide_packed_host", "jd_check_status", "jd_set_graph_mode"):
+        getattr(L, name).restype = C.c_int
+    _lib = L
+    return L
+
+
+def _check(code):
+    if code != JD_OK:
+        raise JDError(code, lib().jd_last_error().decode())
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    raise TypeError(f"cannot take a pointer of {type(x)}")
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def jd_version():
+    return lib().jd_version().decode()
+
+
+def encode_opts(max_length=8192, head_budget=256, strict=True, bos=2, eos=1, mask=4, vocab=256000):
+    return jd_encode_opts(max_length, head_budget, int(bool(strict)), bos, eos, mask, vocab)
+
+
+class _RowKeep:
+    """Holds the ctypes row array and the numpy buffers it points into."""
+
+    def __init__(self, rows):
+        self.keep = []
+        self.arr = (jd_row * max(1, len(rows)))()
+        for i, r in enumerate(rows):
+            st = np.ascontiguousarray(r.state, dtype=np.int32)
+            q = np.ascontiguousarray(r.question, dtype=np.int32)
+            opts = [np.ascontiguousarray(o, dtype=np.int32) for o in r.options]
+            optp = (i32p * max(1, len(opts)))(*[o.ctypes.data_as(i32p) for o in opts])
+            lens = np.asarray([len(o) for o in opts] or [0], dtype=np.int32)
+            self.keep += [st, q, opts, optp, lens]
+            self.arr[i] = jd_row(st.ctypes.data_as(i32p), len(st), q.ctypes.data_as(i32p), len(q), optp,
+                                 lens.ctypes.data_as(i32p), len(opts), int(r.qtype))
+
+
+class HostBatch:
+    """A packed batch copied out of jd_serialize into numpy arrays."""
+
+    def __init__(self, d):
+        self.__dict__.update(d)
+
+    def as_struct(self):
+        """jd_batch over these host arrays (kept alive by self)."""
+        return jd_batch(self.n_rows, self.n_tokens, self.n_markers, self.max_row_len, self.tokens.ctypes.data,
+                        self.cu_seqlens.ctypes.data, self.mask_pos.ctypes.data, self.opt_off.ctypes.data,
+                        self.row_type.ctypes.data, self.head_len.ctypes.data, self.trunc.ctypes.data)
+
+
+def jd_serialize(rows, opts: jd_encode_opts):
+    """Serialize rows (objects with state/question/options/qtype) -> HostBatch.
+
+    Raises JDError with the C status code; the failing row index is in
+    ``err.bad_row``.
+    """
+    L = lib()
+    keep = _RowKeep(rows)
+    out = C.POINTER(jd_batch)()
+    bad = C.c_int32(-1)
+    code = L.jd_serialize(keep.arr, len(rows), C.byref(opts), C.byref(out), C.byref(bad))
+    if code != JD_OK:
+        e = JDError(code, L.jd_last_error().decode())
+        e.bad_row = bad.value
+        raise e
+    b = out.contents
+
+    def arr(ptr, n, dt):
+        if n == 0:
+            return np.zeros(0, dt)
+        ct = C.c_int32 if dt == np.int32 else C.c_uint8
+        return np.ctypeslib.as_array(C.cast(ptr, C.POINTER(ct)), shape=(n,)).copy()
+
+    d = dict(n_rows=b.n_rows, n_tokens=b.n_tokens, n_markers=b.n_markers, max_row_len=b.max_row_len,
+             tokens=arr(b.tokens, b.n_tokens, np.int32), cu_seqlens=arr(b.cu_seqlens, b.n_rows + 1, np.int32),
+             mask_pos=arr(b.mask_pos, b.n_markers, np.int32), opt_off=arr(b.opt_off, b.n_rows + 1, np.int32),
+             row_type=arr(b.row_type, b.n_rows, np.int32), head_len=arr(b.head_len, b.n_rows, np.int32),
+             trunc=arr(b.trunc, b.n_rows, np.uint8))
+    L.jd_batch_free(out)
+    return HostBatch(d)
+
+
+class Model:
+    """Owner of a jd_model handle (weights + workspace on one device)."""
+
+    def __init__(self, weights_path, max_tokens, max_rows, max_markers, precision=JD_PREC_BF16,
+                 scorer=JD_SCORER_MLP, head_act=JD_ACT_RELU, device=0):
+        L = lib()
+        cfg = jd_model_config(int(max_tokens), int(max_rows), int(max_markers), precision, scorer, head_act)
+        h = C.c_void_p()
+        _check(L.jd_model_create(C.byref(cfg), str(weights_path).encode(), int(device), C.byref(h)))
+        self.h = h
+        self.cfg = cfg
+
+    def close(self):
+        if getattr(self, "h", None):
+            lib().jd_model_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def device_bytes(self):
+        return lib().jd_model_device_bytes(self.h)
+
+    @staticmethod
+    def device_batch(n_rows, n_tokens, n_markers, max_row_len, tokens, cu_seqlens, mask_pos, opt_off, row_type):
+        return jd_batch(n_rows, n_tokens, n_markers, max_row_len, _ptr(tokens), _ptr(cu_seqlens), _ptr(mask_pos),
+                        _ptr(opt_off), _ptr(row_type), None, None)
+
+    def jd_decide(self, batch: jd_batch, logits, probs, choice, score, noul, max_p, taps=None, stream=None):
+        out = jd_outputs(_ptr(logits), _ptr(probs), _ptr(choice), _ptr(score), _ptr(noul), _ptr(max_p))
+        tp = None
+        if taps is not None:
+            tp = C.byref(jd_taps(_ptr(taps.get("encoder_out")), _ptr(taps.get("marker_state"))))
+        _check(lib().jd_decide(self.h, C.byref(batch), C.byref(out), tp, _stream(stream)))
+
+    def jd_forward(self, batch: jd_batch, logits, stream=None):
+        _check(lib().jd_forward(self.h, C.byref(batch), _ptr(logits), _stream(stream)))
+
+    def jd_check_status(self):
+        _check(lib().jd_check_status(self.h))
+
+    def jd_set_graph_mode(self, enable):
+        _check(lib().jd_set_graph_mode(self.h, int(bool(enable))))
+
+    def _host_out(self, n_rows, n_markers):
+        o = dict(logits=np.zeros(n_markers, np.float32), probs=np.zeros(n_markers, np.float32),
+                 choice=np.zeros(n_rows, np.int32), score=np.zeros(n_rows, np.float32),
+                 noul=np.zeros(n_rows, np.float32), max_p=np.zeros(n_rows, np.float32))
+        s = jd_host_outputs(o["logits"].ctypes.data_as(f32p), o["probs"].ctypes.data_as(f32p),
+                            o["choice"].ctypes.data_as(i32p), o["score"].ctypes.data_as(f32p),
+                            o["noul"].ctypes.data_as(f32p), o["max_p"].ctypes.data_as(f32p), 0, 0)
+        return o, s
+
+    def jd_decide_host(self, rows, opts: jd_encode_opts, stream=None):
+        keep = _RowKeep(rows)
+        n_m = sum(len(r.options) for r in rows)
+        o, s = self._host_out(len(rows), n_m)
+        _check(lib().jd_decide_host(self.h, keep.arr, len(rows), C.byref(opts), C.byref(s), _stream(stream)))
+        return o
+
+    def jd_decide_packed_host(self, hb: HostBatch, stream=None):
+        o, s = self._host_out(hb.n_rows, hb.n_markers)
+        bs = hb.as_struct()
+        _check(lib().jd_decide_packed_host(self.h, C.byref(bs), C.byref(s), _stream(stream)))
+        return o

@@ -1,0 +1,80 @@
+// Launchers of the library's kernels (host side).  Every launcher queues work
+// on the given stream and returns the launch status; none allocates memory.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "epilogue.cuh"
+
+namespace jd {
+
+// Opt-in shared-memory sizes of every kernel that needs more than 48 KB; call
+// once per device before the first launch (not during stream capture).
+cudaError_t init_kernel_attributes();
+
+// One projection: out = epilogue(A[rows, K] . W[N, K]^T).
+struct GemmOp {
+    int epi;                  // EpiKind
+    int bn;                   // tile width: 384 (QKV, RESID_LN) or 256 (GEGLU, BIAS_ACT)
+    int K, N;
+    const CUtensorMap *tmA;   // BF16 path: A box 64 x 128
+    const CUtensorMap *tmB;   // BF16 path: W box 64 x (bn == 384 ? 192 : 256)
+    const float *A32;         // FP32 path: A [rows, lda]
+    int lda;
+    const float *W32;         // FP32 path: W [N, K]
+    EpiParams ep;
+};
+cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st);
+
+// Per-token row index / position and per-row attention tile offsets.
+cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
+                        cudaStream_t st);
+
+// x = LN(E[token]) (gain only); xn = x in the activation type.
+cudaError_t launch_embed_ln(const int *tokens, int n_tokens, const float *E, int vocab, const float *g, float eps,
+                            float *x, void *xn, bool fp32, unsigned *status, cudaStream_t st);
+
+// Varlen bidirectional attention inside each row.  qkv [T, 1152] holds
+// q | k | v per token (head h at column h * 64 of each part); window < 0
+// means global.  o [T, 384].
+struct AttnArgs {
+    const void *qkv;
+    void *o;
+    const int *cu_seqlens;
+    const int *qb_off;        // [B + 1] prefix sums of ceil(len / 64)
+    int n_rows, n_tokens;
+    int window;
+    const CUtensorMap *tm_qkv; // BF16 path: box 64 x 64 over [T_cap, 1152]
+    unsigned *status;
+};
+cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st);
+
+// Gather the marker rows: hm[m] = h[mask_pos[m]] (FP32), xm[m] = xn[mask_pos[m]].
+cudaError_t launch_gather_markers(const int *mask_pos, int n_markers, int n_tokens, const float *h, const void *xn,
+                                  float *hm, void *xm, bool fp32, unsigned *status, cudaStream_t st);
+
+// Marker-only attention of the last head layer: the queries of each row's
+// markers qm [M, 384] against all keys / values of that row (qkv columns 384..).
+cudaError_t launch_marker_attention(const void *qm, const void *qkv, void *om, const int *cu_seqlens,
+                                    const int *opt_off, const int *mask_pos, int n_rows, bool fp32, cudaStream_t st);
+
+// Scorer: logits[m] from the marker states hm [M, 384].
+struct ScorerArgs {
+    const float *hm;
+    int n_markers;
+    const float *ln_g, *ln_b;
+    const float *w1t, *b1;     // MLP: W1 transposed [384 in][384 out], bias [384]
+    const float *w2, *b2;      // MLP: [384], [1]; linear variant: W [384], b [1]
+    int linear;
+    float eps;
+    float *logits;
+    float *tap;                // optional copy of hm
+};
+cudaError_t launch_scorer(const ScorerArgs &a, cudaStream_t st);
+
+// Per-row softmax and read-outs.
+cudaError_t launch_readout(const float *logits, const int *opt_off, const int *row_type, int n_rows, float *probs,
+                           int *choice, float *score, float *noul, float *max_p, cudaStream_t st);
+
+}  // namespace jd

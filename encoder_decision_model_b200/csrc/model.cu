@@ -1,0 +1,790 @@
+// jd_model: device weights, workspace and the launch sequence of the forward
+// pass ("Julia-1: one score per mask token", "The decision head").
+//
+// Per encoder layer l (global iff l % 3 == 0; "Julia-1 MLX", "Performance"):
+//   QKV GEMM + RoPE      xn -> qkv                 (theta 160000 global / 10000 local)
+//   attention            qkv -> o                  (global, or keys with |i - j| <= 64)
+//   Wo GEMM + residual   x += o Wo^T; xn = LN_mlp(x)
+//   Wi GEMM + GEGLU      y = GELU(u) * g
+//   Wo2 GEMM + residual  x += y Wo2^T; xn = LN_attn(l+1)(x)
+//     (last layer: h = LN_final(x) + type row, xn = LN1 of head layer 0)
+// Head layer 0 (all tokens) and head layer 1 (keys / values for all tokens,
+// everything else only at the markers), scorer, read-outs.
+//
+// Weights file: .jdw (see workloads/gen.py for the writer), FP32.  The
+// library keeps the embedding table, norms, biases, type table and scorer in
+// FP32 and stores projection weights as BF16 (BF16 mode) or FP32 (validation
+// mode).  Wi rows are interleaved in blocks of 128 ([u_j | g_j]) so that one
+// 256-wide GEMM tile holds both halves of 128 GEGLU outputs.
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "host_common.h"
+#include "kernels.h"
+
+using namespace jd;
+
+namespace {
+
+constexpr int NL = 22;
+constexpr int VOCAB = 256000;
+constexpr float EPS = 1e-5f;
+
+#define CK(call)                                                                                       \
+    do {                                                                                               \
+        cudaError_t e_ = (call);                                                                       \
+        if (e_ != cudaSuccess) return jd::fail(JD_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+    } while (0)
+
+// ---------------------------------------------------------------- weights file
+
+struct TensorRec {
+    std::vector<uint32_t> shape;
+    uint64_t offset;  // absolute
+    uint64_t count;
+};
+
+struct WeightFile {
+    std::map<std::string, TensorRec> idx;
+    FILE *fh = nullptr;
+    ~WeightFile() {
+        if (fh) fclose(fh);
+    }
+};
+
+jd_status open_weights(const char *path, WeightFile &wf) {
+    wf.fh = fopen(path, "rb");
+    if (!wf.fh) return fail(JD_ERR_IO, "cannot open weights file %s", path);
+    char magic[8];
+    uint32_t n = 0;
+    if (fread(magic, 1, 8, wf.fh) != 8 || memcmp(magic, "JDWGT001", 8) != 0 || fread(&n, 4, 1, wf.fh) != 1)
+        return fail(JD_ERR_IO, "%s is not a .jdw weights file", path);
+    const uint64_t header = 12ull + 96ull * n;
+    const uint64_t data0 = (header + 255) / 256 * 256;
+    for (uint32_t i = 0; i < n; ++i) {
+        unsigned char rec[96];
+        if (fread(rec, 1, 96, wf.fh) != 96) return fail(JD_ERR_IO, "truncated weights header");
+        char name[65];
+        memcpy(name, rec, 64);
+        name[64] = 0;
+        uint32_t ndim, dims[4];
+        uint64_t off;
+        memcpy(&ndim, rec + 64, 4);
+        memcpy(dims, rec + 68, 16);
+        memcpy(&off, rec + 84, 8);
+        TensorRec t;
+        t.count = 1;
+        for (uint32_t d = 0; d < ndim && d < 4; ++d) {
+            t.shape.push_back(dims[d]);
+            t.count *= dims[d];
+        }
+        t.offset = data0 + off;
+        wf.idx[name] = t;
+    }
+    return JD_OK;
+}
+
+jd_status read_tensor(WeightFile &wf, const std::string &name, std::vector<uint32_t> shape, std::vector<float> &out) {
+    auto it = wf.idx.find(name);
+    if (it == wf.idx.end()) return fail(JD_ERR_IO, "weights file has no tensor %s", name.c_str());
+    if (it->second.shape != shape) return fail(JD_ERR_IO, "tensor %s has an unexpected shape", name.c_str());
+    out.resize(it->second.count);
+    if (fseeko(wf.fh, (off_t)it->second.offset, SEEK_SET) != 0 ||
+        fread(out.data(), 4, out.size(), wf.fh) != out.size())
+        return fail(JD_ERR_IO, "cannot read tensor %s", name.c_str());
+    return JD_OK;
+}
+
+// FP32 -> BF16, round to nearest even (NaN kept quiet).
+uint16_t to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x40);
+    const uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 map over [rows, cols] with row stride ld (elements); box = box_cols x box_rows, 128-byte swizzle.
+jd_status make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_cols,
+                   uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(JD_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(JD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return JD_OK;
+}
+
+struct ProjW {            // one projection weight [N, K]
+    void *w = nullptr;    // bf16 or f32 on device
+    CUtensorMap tm{};     // BF16 mode only
+    int N = 0, K = 0;
+};
+
+}  // namespace
+
+struct jd_model {
+    jd_model_config cfg{};
+    int device = 0;
+    bool fp32 = false;
+    int T_cap = 0, B_cap = 0, M_cap = 0;
+    size_t bytes = 0;
+    std::vector<void *> allocs;
+
+    // weights
+    float *E = nullptr, *emb_g = nullptr, *fin_g = nullptr, *type_tab = nullptr;
+    float *attn_g[NL] = {}, *mlp_g[NL] = {};
+    ProjW Wqkv[NL], Wo[NL], Wi[NL], Wo2[NL];
+    float *n1g[2] = {}, *n1b[2] = {}, *n2g[2] = {}, *n2b[2] = {};
+    ProjW in_full[2], in_q[2], in_kv[2], out_p[2], lin1[2], lin2[2];
+    float *in_b[2] = {}, *out_b[2] = {}, *l1_b[2] = {}, *l2_b[2] = {};
+    float *sc_g = nullptr, *sc_b = nullptr, *sc_w1t = nullptr, *sc_b1 = nullptr, *sc_w2 = nullptr, *sc_b2 = nullptr;
+    float *lin_w = nullptr, *lin_b = nullptr;
+    float2 *rope_g = nullptr, *rope_l = nullptr;
+
+    // workspace
+    float *x = nullptr;
+    void *xn = nullptr, *qkv = nullptr, *o = nullptr, *y = nullptr;
+    int *tok_row = nullptr, *pos = nullptr, *qb_off = nullptr;
+    float *hm = nullptr;
+    void *xm = nullptr, *qm = nullptr, *om = nullptr, *xnm = nullptr, *ym = nullptr;
+    unsigned *status = nullptr;
+    CUtensorMap tm_xn{}, tm_o{}, tm_y_enc{}, tm_y_head{}, tm_qkv{}, tm_xm{}, tm_om{}, tm_xnm{}, tm_ym{};
+
+    // internal outputs (jd_forward, host entry points) and device batch staging
+    float *i_logits = nullptr, *i_probs = nullptr, *i_score = nullptr, *i_noul = nullptr, *i_maxp = nullptr;
+    int *i_choice = nullptr;
+    int *d_tokens = nullptr, *d_cu = nullptr, *d_mask = nullptr, *d_opt = nullptr, *d_type = nullptr;
+    // pinned host staging
+    int *h_tokens = nullptr, *h_cu = nullptr, *h_mask = nullptr, *h_opt = nullptr, *h_type = nullptr;
+    float *h_logits = nullptr, *h_probs = nullptr, *h_score = nullptr, *h_noul = nullptr, *h_maxp = nullptr;
+    int *h_choice = nullptr;
+
+    cudaStream_t last_stream = nullptr;
+
+    // CUDA graph cache (one entry)
+    bool graph_mode = false;
+    cudaGraphExec_t gexec = nullptr;
+    std::vector<uintptr_t> gkey;
+
+    template <class T>
+    jd_status dalloc(T **p, size_t n) {
+        void *q = nullptr;
+        size_t b = std::max<size_t>(n, 1) * sizeof(T);
+        cudaError_t e = cudaMalloc(&q, b);
+        if (e != cudaSuccess) return fail(JD_ERR_CUDA, "cudaMalloc(%zu): %s", b, cudaGetErrorString(e));
+        e = cudaMemset(q, 0, b);
+        if (e != cudaSuccess) return fail(JD_ERR_CUDA, "cudaMemset: %s", cudaGetErrorString(e));
+        allocs.push_back(q);
+        bytes += b;
+        *p = static_cast<T *>(q);
+        return JD_OK;
+    }
+    template <class T>
+    jd_status halloc(T **p, size_t n) {
+        void *q = nullptr;
+        cudaError_t e = cudaHostAlloc(&q, std::max<size_t>(n, 1) * sizeof(T), cudaHostAllocDefault);
+        if (e != cudaSuccess) return fail(JD_ERR_CUDA, "cudaHostAlloc: %s", cudaGetErrorString(e));
+        hallocs.push_back(q);
+        *p = static_cast<T *>(q);
+        return JD_OK;
+    }
+    std::vector<void *> hallocs;
+};
+
+namespace {
+
+#define TRY(call)                    \
+    do {                             \
+        jd_status s_ = (call);       \
+        if (s_ != JD_OK) return s_;  \
+    } while (0)
+
+jd_status upload_f32(jd_model *m, WeightFile &wf, const std::string &name, std::vector<uint32_t> shape, float **dst) {
+    std::vector<float> h;
+    TRY(read_tensor(wf, name, shape, h));
+    TRY(m->dalloc(dst, h.size()));
+    CK(cudaMemcpy(*dst, h.data(), h.size() * 4, cudaMemcpyHostToDevice));
+    return JD_OK;
+}
+
+// Upload rows [r0, r0 + N) of a host [*, K] matrix as a projection weight.
+jd_status upload_proj(jd_model *m, const std::vector<float> &h, int r0, int N, int K, int bn, ProjW &p) {
+    p.N = N;
+    p.K = K;
+    const float *src = h.data() + (size_t)r0 * K;
+    if (m->fp32) {
+        float *d = nullptr;
+        TRY(m->dalloc(&d, (size_t)N * K));
+        CK(cudaMemcpy(d, src, (size_t)N * K * 4, cudaMemcpyHostToDevice));
+        p.w = d;
+    } else {
+        std::vector<uint16_t> b((size_t)N * K);
+        for (size_t i = 0; i < b.size(); ++i) b[i] = to_bf16(src[i]);
+        uint16_t *d = nullptr;
+        TRY(m->dalloc(&d, b.size()));
+        CK(cudaMemcpy(d, b.data(), b.size() * 2, cudaMemcpyHostToDevice));
+        p.w = d;
+        // one TMA box per MMA: 192 rows for 384-wide tiles (two N=192 MMAs), else the tile width
+        const uint32_t box_rows = bn == 384 ? 192 : (uint32_t)bn;
+        TRY(make_map(&p.tm, d, K, N, K, 64, box_rows));
+    }
+    return JD_OK;
+}
+
+jd_status load_proj(jd_model *m, WeightFile &wf, const std::string &name, int N, int K, int bn, ProjW &p) {
+    std::vector<float> h;
+    TRY(read_tensor(wf, name, {(uint32_t)N, (uint32_t)K}, h));
+    return upload_proj(m, h, 0, N, K, bn, p);
+}
+
+jd_status make_rope_table(jd_model *m, double theta, float2 **dst) {
+    std::vector<float2> h((size_t)MAX_POS * 32);
+    for (int p = 0; p < MAX_POS; ++p)
+        for (int i = 0; i < 32; ++i) {
+            const double ang = (double)p * std::pow(theta, -2.0 * i / 64.0);
+            h[(size_t)p * 32 + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+        }
+    TRY(m->dalloc(dst, h.size()));
+    CK(cudaMemcpy(*dst, h.data(), h.size() * sizeof(float2), cudaMemcpyHostToDevice));
+    return JD_OK;
+}
+
+jd_status load_weights(jd_model *m, const char *path) {
+    WeightFile wf;
+    TRY(open_weights(path, wf));
+    const uint32_t d = D;
+    TRY(upload_f32(m, wf, "embed.E", {VOCAB, d}, &m->E));
+    TRY(upload_f32(m, wf, "embed.norm.g", {d}, &m->emb_g));
+    for (int l = 0; l < NL; ++l) {
+        const std::string p = "enc." + std::to_string(l) + ".";
+        if (l != 0) TRY(upload_f32(m, wf, p + "attn_norm.g", {d}, &m->attn_g[l]));
+        TRY(upload_f32(m, wf, p + "mlp_norm.g", {d}, &m->mlp_g[l]));
+        TRY(load_proj(m, wf, p + "Wqkv", QKV, D, 384, m->Wqkv[l]));
+        TRY(load_proj(m, wf, p + "Wo", D, D, 384, m->Wo[l]));
+        TRY(load_proj(m, wf, p + "Wo2", D, FF, 384, m->Wo2[l]));
+        std::vector<float> wi, il((size_t)2 * FF * D);
+        TRY(read_tensor(wf, p + "Wi", {2 * FF, d}, wi));
+        for (int j = 0; j < FF / 128; ++j) {  // [u_j (128 rows) | g_j (128 rows)]
+            memcpy(&il[(size_t)(j * 256) * D], &wi[(size_t)(j * 128) * D], sizeof(float) * 128 * D);
+            memcpy(&il[(size_t)(j * 256 + 128) * D], &wi[(size_t)(FF + j * 128) * D], sizeof(float) * 128 * D);
+        }
+        TRY(upload_proj(m, il, 0, 2 * FF, D, 256, m->Wi[l]));
+    }
+    TRY(upload_f32(m, wf, "enc.final_norm.g", {d}, &m->fin_g));
+    TRY(upload_f32(m, wf, "head.type_table", {3, d}, &m->type_tab));
+    for (int i = 0; i < 2; ++i) {
+        const std::string p = "head." + std::to_string(i) + ".";
+        TRY(upload_f32(m, wf, p + "norm1.g", {d}, &m->n1g[i]));
+        TRY(upload_f32(m, wf, p + "norm1.b", {d}, &m->n1b[i]));
+        TRY(upload_f32(m, wf, p + "norm2.g", {d}, &m->n2g[i]));
+        TRY(upload_f32(m, wf, p + "norm2.b", {d}, &m->n2b[i]));
+        std::vector<float> win;
+        TRY(read_tensor(wf, p + "in_proj.W", {QKV, d}, win));
+        if (i == 0) {
+            TRY(upload_proj(m, win, 0, QKV, D, 384, m->in_full[i]));
+        } else {
+            TRY(upload_proj(m, win, 0, D, D, 384, m->in_q[i]));
+            TRY(upload_proj(m, win, D, 2 * D, D, 384, m->in_kv[i]));
+        }
+        TRY(upload_f32(m, wf, p + "in_proj.b", {QKV}, &m->in_b[i]));
+        TRY(load_proj(m, wf, p + "out_proj.W", D, D, 384, m->out_p[i]));
+        TRY(upload_f32(m, wf, p + "out_proj.b", {d}, &m->out_b[i]));
+        TRY(load_proj(m, wf, p + "linear1.W", HFF, D, 256, m->lin1[i]));
+        TRY(upload_f32(m, wf, p + "linear1.b", {HFF}, &m->l1_b[i]));
+        TRY(load_proj(m, wf, p + "linear2.W", D, HFF, 384, m->lin2[i]));
+        TRY(upload_f32(m, wf, p + "linear2.b", {d}, &m->l2_b[i]));
+    }
+    TRY(upload_f32(m, wf, "scorer.norm.g", {d}, &m->sc_g));
+    TRY(upload_f32(m, wf, "scorer.norm.b", {d}, &m->sc_b));
+    {
+        std::vector<float> w1, w1t((size_t)D * D);
+        TRY(read_tensor(wf, "scorer.linear1.W", {d, d}, w1));
+        for (int o = 0; o < D; ++o)
+            for (int k = 0; k < D; ++k) w1t[(size_t)k * D + o] = w1[(size_t)o * D + k];
+        TRY(m->dalloc(&m->sc_w1t, w1t.size()));
+        CK(cudaMemcpy(m->sc_w1t, w1t.data(), w1t.size() * 4, cudaMemcpyHostToDevice));
+    }
+    TRY(upload_f32(m, wf, "scorer.linear1.b", {d}, &m->sc_b1));
+    TRY(upload_f32(m, wf, "scorer.linear2.W", {1, d}, &m->sc_w2));
+    TRY(upload_f32(m, wf, "scorer.linear2.b", {1}, &m->sc_b2));
+    TRY(upload_f32(m, wf, "scorer_lin.W", {1, d}, &m->lin_w));
+    TRY(upload_f32(m, wf, "scorer_lin.b", {1}, &m->lin_b));
+    TRY(make_rope_table(m, 160000.0, &m->rope_g));
+    TRY(make_rope_table(m, 10000.0, &m->rope_l));
+    return JD_OK;
+}
+
+jd_status alloc_workspace(jd_model *m) {
+    const size_t T = m->T_cap, M = m->M_cap, B = m->B_cap;
+    const size_t es = m->fp32 ? 4 : 2;
+    TRY(m->dalloc(&m->x, T * D));
+    uint8_t *p = nullptr;
+    TRY(m->dalloc(&p, T * D * es)); m->xn = p;
+    TRY(m->dalloc(&p, T * QKV * es)); m->qkv = p;
+    TRY(m->dalloc(&p, T * D * es)); m->o = p;
+    TRY(m->dalloc(&p, T * HFF * es)); m->y = p;
+    TRY(m->dalloc(&m->tok_row, T));
+    TRY(m->dalloc(&m->pos, T));
+    TRY(m->dalloc(&m->qb_off, B + 1));
+    TRY(m->dalloc(&m->hm, M * D));
+    TRY(m->dalloc(&p, M * D * es)); m->xm = p;
+    TRY(m->dalloc(&p, M * D * es)); m->qm = p;
+    TRY(m->dalloc(&p, M * D * es)); m->om = p;
+    TRY(m->dalloc(&p, M * D * es)); m->xnm = p;
+    TRY(m->dalloc(&p, M * HFF * es)); m->ym = p;
+    TRY(m->dalloc(&m->status, 1));
+    TRY(m->dalloc(&m->i_logits, M));
+    TRY(m->dalloc(&m->i_probs, M));
+    TRY(m->dalloc(&m->i_choice, B));
+    TRY(m->dalloc(&m->i_score, B));
+    TRY(m->dalloc(&m->i_noul, B));
+    TRY(m->dalloc(&m->i_maxp, B));
+    TRY(m->dalloc(&m->d_tokens, T));
+    TRY(m->dalloc(&m->d_cu, B + 1));
+    TRY(m->dalloc(&m->d_mask, M));
+    TRY(m->dalloc(&m->d_opt, B + 1));
+    TRY(m->dalloc(&m->d_type, B));
+    TRY(m->halloc(&m->h_tokens, T));
+    TRY(m->halloc(&m->h_cu, B + 1));
+    TRY(m->halloc(&m->h_mask, M));
+    TRY(m->halloc(&m->h_opt, B + 1));
+    TRY(m->halloc(&m->h_type, B));
+    TRY(m->halloc(&m->h_logits, M));
+    TRY(m->halloc(&m->h_probs, M));
+    TRY(m->halloc(&m->h_choice, B));
+    TRY(m->halloc(&m->h_score, B));
+    TRY(m->halloc(&m->h_noul, B));
+    TRY(m->halloc(&m->h_maxp, B));
+    if (!m->fp32) {
+        TRY(make_map(&m->tm_xn, m->xn, D, T, D, 64, 128));
+        TRY(make_map(&m->tm_o, m->o, D, T, D, 64, 128));
+        TRY(make_map(&m->tm_y_enc, m->y, FF, T, FF, 64, 128));
+        TRY(make_map(&m->tm_y_head, m->y, HFF, T, HFF, 64, 128));
+        TRY(make_map(&m->tm_qkv, m->qkv, QKV, T, QKV, 64, 64));
+        TRY(make_map(&m->tm_xm, m->xm, D, M, D, 64, 128));
+        TRY(make_map(&m->tm_om, m->om, D, M, D, 64, 128));
+        TRY(make_map(&m->tm_xnm, m->xnm, D, M, D, 64, 128));
+        TRY(make_map(&m->tm_ym, m->ym, HFF, M, HFF, 64, 128));
+    }
+    return JD_OK;
+}
+
+EpiParams base_ep(jd_model *m, int rows) {
+    EpiParams e;
+    memset(&e, 0, sizeof(e));
+    e.rows = rows;
+    e.eps = EPS;
+    e.status = m->status;
+    e.act = m->cfg.head_act;
+    return e;
+}
+
+GemmOp make_op(int epi, int bn, const ProjW &w, const CUtensorMap *tmA, const void *A, int lda, const EpiParams &ep) {
+    GemmOp op;
+    op.epi = epi;
+    op.bn = bn;
+    op.K = w.K;
+    op.N = w.N;
+    op.tmA = tmA;
+    op.tmB = &w.tm;
+    op.A32 = static_cast<const float *>(A);
+    op.lda = lda;
+    op.W32 = static_cast<const float *>(w.w);
+    op.ep = ep;
+    return op;
+}
+
+template <class T>
+T *offset(void *p, size_t elems, bool fp32) {
+    return reinterpret_cast<T *>(static_cast<uint8_t *>(p) + elems * (fp32 ? 4 : 2));
+}
+
+#define LK(call)                                                                                  \
+    do {                                                                                          \
+        cudaError_t e_ = (call);                                                                  \
+        if (e_ != cudaSuccess) return fail(JD_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+    } while (0)
+
+// The whole launch sequence (no allocation, no synchronisation).
+jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out, const jd_taps *taps,
+                          cudaStream_t st) {
+    const bool f32 = m->fp32;
+    const int T = b->n_tokens, B = b->n_rows, M = b->n_markers;
+    LK(cudaMemsetAsync(m->status, 0, sizeof(unsigned), st));
+    LK(launch_prep(b->cu_seqlens, B, T, m->tok_row, m->pos, m->qb_off, st));
+    LK(launch_embed_ln(b->tokens, T, m->E, VOCAB, m->emb_g, EPS, m->x, m->xn, f32, m->status, st));
+
+    AttnArgs aa;
+    aa.qkv = m->qkv;
+    aa.o = m->o;
+    aa.cu_seqlens = b->cu_seqlens;
+    aa.qb_off = m->qb_off;
+    aa.n_rows = B;
+    aa.n_tokens = T;
+    aa.tm_qkv = &m->tm_qkv;
+    aa.status = m->status;
+
+    for (int l = 0; l < NL; ++l) {
+        const bool glob = (l % 3) == 0;
+        EpiParams e = base_ep(m, T);
+        e.out = m->qkv;
+        e.ldo = QKV;
+        e.rope = glob ? m->rope_g : m->rope_l;
+        e.pos = m->pos;
+        e.rope_cols = 2 * D;
+        LK(launch_gemm(make_op(EPI_QKV, 384, m->Wqkv[l], &m->tm_xn, m->xn, D, e), f32, st));
+
+        aa.window = glob ? -1 : 64;
+        LK(launch_attention(aa, f32, st));
+
+        e = base_ep(m, T);
+        e.out = m->xn;
+        e.ldo = D;
+        e.resid = m->x;
+        e.ln_g = m->mlp_g[l];
+        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo[l], &m->tm_o, m->o, D, e), f32, st));
+
+        e = base_ep(m, T);
+        e.out = m->y;
+        e.ldo = FF;
+        LK(launch_gemm(make_op(EPI_GEGLU, 256, m->Wi[l], &m->tm_xn, m->xn, D, e), f32, st));
+
+        e = base_ep(m, T);
+        e.out = m->xn;
+        e.ldo = D;
+        e.resid = m->x;
+        if (l + 1 < NL) {
+            e.ln_g = m->attn_g[l + 1];
+        } else {
+            e.fin_g = m->fin_g;
+            e.type_tab = m->type_tab;
+            e.tok_row = m->tok_row;
+            e.row_type = b->row_type;
+            e.tap = taps ? taps->encoder_out : nullptr;
+            e.ln_g = m->n1g[0];
+            e.ln_b = m->n1b[0];
+        }
+        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo2[l], &m->tm_y_enc, m->y, FF, e), f32, st));
+    }
+
+    // ---- head layer 0 (all tokens)
+    {
+        EpiParams e = base_ep(m, T);
+        e.out = m->qkv;
+        e.ldo = QKV;
+        e.bias = m->in_b[0];
+        LK(launch_gemm(make_op(EPI_QKV, 384, m->in_full[0], &m->tm_xn, m->xn, D, e), f32, st));
+        aa.window = -1;
+        LK(launch_attention(aa, f32, st));
+        e = base_ep(m, T);
+        e.out = m->xn;
+        e.ldo = D;
+        e.bias = m->out_b[0];
+        e.resid = m->x;
+        e.ln_g = m->n2g[0];
+        e.ln_b = m->n2b[0];
+        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->out_p[0], &m->tm_o, m->o, D, e), f32, st));
+        e = base_ep(m, T);
+        e.out = m->y;
+        e.ldo = HFF;
+        e.bias = m->l1_b[0];
+        LK(launch_gemm(make_op(EPI_BIAS_ACT, 256, m->lin1[0], &m->tm_xn, m->xn, D, e), f32, st));
+        e = base_ep(m, T);
+        e.out = m->xn;
+        e.ldo = D;
+        e.bias = m->l2_b[0];
+        e.resid = m->x;
+        e.ln_g = m->n1g[1];
+        e.ln_b = m->n1b[1];
+        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[0], &m->tm_y_head, m->y, HFF, e), f32, st));
+    }
+    // ---- head layer 1: keys / values for every token, the rest at the markers only
+    {
+        EpiParams e = base_ep(m, T);
+        e.out = offset<uint8_t>(m->qkv, D, f32);
+        e.ldo = QKV;
+        e.bias = m->in_b[1] + D;
+        LK(launch_gemm(make_op(EPI_QKV, 384, m->in_kv[1], &m->tm_xn, m->xn, D, e), f32, st));
+        LK(launch_gather_markers(b->mask_pos, M, T, m->x, m->xn, m->hm, m->xm, f32, m->status, st));
+        e = base_ep(m, M);
+        e.out = m->qm;
+        e.ldo = D;
+        e.bias = m->in_b[1];
+        LK(launch_gemm(make_op(EPI_QKV, 384, m->in_q[1], &m->tm_xm, m->xm, D, e), f32, st));
+        LK(launch_marker_attention(m->qm, m->qkv, m->om, b->cu_seqlens, b->opt_off, b->mask_pos, B, f32, st));
+        e = base_ep(m, M);
+        e.out = m->xnm;
+        e.ldo = D;
+        e.bias = m->out_b[1];
+        e.resid = m->hm;
+        e.ln_g = m->n2g[1];
+        e.ln_b = m->n2b[1];
+        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->out_p[1], &m->tm_om, m->om, D, e), f32, st));
+        e = base_ep(m, M);
+        e.out = m->ym;
+        e.ldo = HFF;
+        e.bias = m->l1_b[1];
+        LK(launch_gemm(make_op(EPI_BIAS_ACT, 256, m->lin1[1], &m->tm_xnm, m->xnm, D, e), f32, st));
+        e = base_ep(m, M);
+        e.bias = m->l2_b[1];
+        e.resid = m->hm;
+        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[1], &m->tm_ym, m->ym, HFF, e), f32, st));
+    }
+    // ---- scorer + read-outs
+    ScorerArgs sa;
+    sa.hm = m->hm;
+    sa.n_markers = M;
+    sa.ln_g = m->sc_g;
+    sa.ln_b = m->sc_b;
+    sa.w1t = m->sc_w1t;
+    sa.b1 = m->sc_b1;
+    sa.linear = m->cfg.scorer == JD_SCORER_LINEAR;
+    sa.w2 = sa.linear ? m->lin_w : m->sc_w2;
+    sa.b2 = sa.linear ? m->lin_b : m->sc_b2;
+    sa.eps = EPS;
+    sa.logits = out->logits;
+    sa.tap = taps ? taps->marker_state : nullptr;
+    LK(launch_scorer(sa, st));
+    LK(launch_readout(out->logits, b->opt_off, b->row_type, B, out->probs, out->choice, out->score, out->noul,
+                      out->max_p, st));
+    return JD_OK;
+}
+
+jd_status check_batch(jd_model *m, const jd_batch *b) {
+    if (!b) return fail(JD_ERR_INVALID_ARG, "batch is NULL");
+    if (b->n_rows < 1 || b->n_tokens < 1 || b->n_markers < 1)
+        return fail(JD_ERR_INVALID_ARG, "empty batch (rows %d, tokens %d, markers %d)", b->n_rows, b->n_tokens,
+                    b->n_markers);
+    if (b->n_tokens > m->cfg.max_tokens || b->n_rows > m->cfg.max_rows || b->n_markers > m->cfg.max_markers)
+        return fail(JD_ERR_CAPACITY, "batch (%d tokens, %d rows, %d markers) exceeds capacity (%d, %d, %d)",
+                    b->n_tokens, b->n_rows, b->n_markers, m->cfg.max_tokens, m->cfg.max_rows, m->cfg.max_markers);
+    if (b->max_row_len > MAX_POS) return fail(JD_ERR_INVALID_ARG, "a row is longer than 8192 tokens");
+    if (!b->tokens || !b->cu_seqlens || !b->mask_pos || !b->opt_off || !b->row_type)
+        return fail(JD_ERR_INVALID_ARG, "batch has a NULL array");
+    return JD_OK;
+}
+
+}  // namespace
+
+// ================================================================== C ABI
+
+extern "C" jd_status jd_model_create(const jd_model_config *cfg, const char *weights_path, int device,
+                                     jd_model **out) {
+    clear_error();
+    if (!out || !cfg || !weights_path) return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    *out = nullptr;
+    if (cfg->max_tokens < 1 || cfg->max_rows < 1 || cfg->max_markers < 1)
+        return fail(JD_ERR_INVALID_ARG, "capacities must be positive");
+    if (cfg->precision != JD_PREC_BF16 && cfg->precision != JD_PREC_FP32)
+        return fail(JD_ERR_INVALID_ARG, "unknown precision %d", cfg->precision);
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) return fail(JD_ERR_CUDA, "no CUDA device");
+    if (device < 0 || device >= ndev) return fail(JD_ERR_INVALID_ARG, "device %d out of range", device);
+    CK(cudaSetDevice(device));
+    cudaDeviceProp prop;
+    CK(cudaGetDeviceProperties(&prop, device));
+    if (prop.major != 10) return fail(JD_ERR_CUDA, "this library is built for sm_100a; device is sm_%d%d", prop.major, prop.minor);
+
+    jd_model *m = new jd_model();
+    m->cfg = *cfg;
+    m->device = device;
+    m->fp32 = cfg->precision == JD_PREC_FP32;
+    m->T_cap = (cfg->max_tokens + 127) / 128 * 128;
+    m->B_cap = cfg->max_rows;
+    m->M_cap = (cfg->max_markers + 127) / 128 * 128;
+    jd_status s = JD_OK;
+    {
+        cudaError_t e = init_kernel_attributes();
+        if (e != cudaSuccess) s = fail(JD_ERR_CUDA, "kernel attributes: %s", cudaGetErrorString(e));
+    }
+    if (s == JD_OK) s = load_weights(m, weights_path);
+    if (s == JD_OK) s = alloc_workspace(m);
+    if (s == JD_OK) {
+        cudaError_t e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) s = fail(JD_ERR_CUDA, "setup: %s", cudaGetErrorString(e));
+    }
+    if (s != JD_OK) {
+        jd_model_destroy(m);
+        return s;
+    }
+    *out = m;
+    return JD_OK;
+}
+
+extern "C" void jd_model_destroy(jd_model *m) {
+    if (!m) return;
+    cudaSetDevice(m->device);
+    if (m->gexec) cudaGraphExecDestroy(m->gexec);
+    for (void *p : m->allocs) cudaFree(p);
+    for (void *p : m->hallocs) cudaFreeHost(p);
+    delete m;
+}
+
+extern "C" size_t jd_model_device_bytes(const jd_model *m) { return m ? m->bytes : 0; }
+
+extern "C" jd_status jd_set_graph_mode(jd_model *m, int enable) {
+    clear_error();
+    if (!m) return fail(JD_ERR_INVALID_ARG, "model is NULL");
+    m->graph_mode = enable != 0;
+    return JD_OK;
+}
+
+extern "C" jd_status jd_decide(jd_model *m, const jd_batch *b, const jd_outputs *out, const jd_taps *taps,
+                               void *stream) {
+    clear_error();
+    if (!m || !out) return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    TRY(check_batch(m, b));
+    if (!out->logits || !out->probs || !out->choice || !out->score || !out->noul || !out->max_p)
+        return fail(JD_ERR_INVALID_ARG, "an output pointer is NULL");
+    CK(cudaSetDevice(m->device));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    m->last_stream = st;
+    if (!m->graph_mode) return enqueue_forward(m, b, out, taps, st);
+
+    std::vector<uintptr_t> key = {(uintptr_t)b->n_tokens,  (uintptr_t)b->n_rows,     (uintptr_t)b->n_markers,
+                                  (uintptr_t)b->tokens,    (uintptr_t)b->cu_seqlens, (uintptr_t)b->mask_pos,
+                                  (uintptr_t)b->opt_off,   (uintptr_t)b->row_type,   (uintptr_t)out->logits,
+                                  (uintptr_t)out->probs,   (uintptr_t)out->choice,   (uintptr_t)out->score,
+                                  (uintptr_t)out->noul,    (uintptr_t)out->max_p,
+                                  (uintptr_t)(taps ? taps->encoder_out : nullptr),
+                                  (uintptr_t)(taps ? taps->marker_state : nullptr)};
+    if (!m->gexec || key != m->gkey) {
+        if (m->gexec) {
+            cudaGraphExecDestroy(m->gexec);
+            m->gexec = nullptr;
+        }
+        cudaStream_t cap = st;
+        bool own = false;
+        if (cap == nullptr) {  // the legacy stream cannot be captured: capture on a private one
+            CK(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
+            own = true;
+        }
+        CK(cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal));
+        jd_status s = enqueue_forward(m, b, out, taps, cap);
+        cudaGraph_t g = nullptr;
+        cudaError_t e = cudaStreamEndCapture(cap, &g);
+        if (own) cudaStreamDestroy(cap);
+        if (s != JD_OK) {
+            if (g) cudaGraphDestroy(g);
+            return s;
+        }
+        if (e != cudaSuccess) return fail(JD_ERR_CUDA, "graph capture: %s", cudaGetErrorString(e));
+        e = cudaGraphInstantiate(&m->gexec, g, 0);
+        cudaGraphDestroy(g);
+        if (e != cudaSuccess) return fail(JD_ERR_CUDA, "graph instantiate: %s", cudaGetErrorString(e));
+        m->gkey = key;
+    }
+    CK(cudaGraphLaunch(m->gexec, st));
+    return JD_OK;
+}
+
+extern "C" jd_status jd_forward(jd_model *m, const jd_batch *b, float *logits, void *stream) {
+    clear_error();
+    if (!m || !logits) return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    TRY(check_batch(m, b));
+    jd_outputs o{logits, m->i_probs, m->i_choice, m->i_score, m->i_noul, m->i_maxp};
+    return jd_decide(m, b, &o, nullptr, stream);
+}
+
+extern "C" jd_status jd_decide_packed_host(jd_model *m, const jd_batch *hb, jd_host_outputs *ho, void *stream) {
+    clear_error();
+    if (!m || !hb || !ho) return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    TRY(check_batch(m, hb));
+    CK(cudaSetDevice(m->device));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int T = hb->n_tokens, B = hb->n_rows, M = hb->n_markers;
+    memcpy(m->h_tokens, hb->tokens, sizeof(int) * T);
+    memcpy(m->h_cu, hb->cu_seqlens, sizeof(int) * (B + 1));
+    memcpy(m->h_mask, hb->mask_pos, sizeof(int) * M);
+    memcpy(m->h_opt, hb->opt_off, sizeof(int) * (B + 1));
+    memcpy(m->h_type, hb->row_type, sizeof(int) * B);
+    CK(cudaMemcpyAsync(m->d_tokens, m->h_tokens, sizeof(int) * T, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_cu, m->h_cu, sizeof(int) * (B + 1), cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_mask, m->h_mask, sizeof(int) * M, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_opt, m->h_opt, sizeof(int) * (B + 1), cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_type, m->h_type, sizeof(int) * B, cudaMemcpyHostToDevice, st));
+    jd_batch db = *hb;
+    db.tokens = m->d_tokens;
+    db.cu_seqlens = m->d_cu;
+    db.mask_pos = m->d_mask;
+    db.opt_off = m->d_opt;
+    db.row_type = m->d_type;
+    db.head_len = nullptr;
+    db.trunc = nullptr;
+    jd_outputs o{m->i_logits, m->i_probs, m->i_choice, m->i_score, m->i_noul, m->i_maxp};
+    TRY(jd_decide(m, &db, &o, nullptr, stream));
+    CK(cudaMemcpyAsync(m->h_logits, m->i_logits, sizeof(float) * M, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(m->h_probs, m->i_probs, sizeof(float) * M, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(m->h_choice, m->i_choice, sizeof(int) * B, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(m->h_score, m->i_score, sizeof(float) * B, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(m->h_noul, m->i_noul, sizeof(float) * B, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(m->h_maxp, m->i_maxp, sizeof(float) * B, cudaMemcpyDeviceToHost, st));
+    CK(cudaStreamSynchronize(st));
+    unsigned stv = 0;
+    CK(cudaMemcpy(&stv, m->status, sizeof(unsigned), cudaMemcpyDeviceToHost));
+    if (stv) return fail(JD_ERR_DEVICE_STATUS, "device status 0x%x (1: wait timeout, 2: token id range, 4: index)", stv);
+    if (ho->logits) memcpy(ho->logits, m->h_logits, sizeof(float) * M);
+    if (ho->probs) memcpy(ho->probs, m->h_probs, sizeof(float) * M);
+    if (ho->choice) memcpy(ho->choice, m->h_choice, sizeof(int) * B);
+    if (ho->score) memcpy(ho->score, m->h_score, sizeof(float) * B);
+    if (ho->noul) memcpy(ho->noul, m->h_noul, sizeof(float) * B);
+    if (ho->max_p) memcpy(ho->max_p, m->h_maxp, sizeof(float) * B);
+    ho->n_rows = B;
+    ho->n_markers = M;
+    return JD_OK;
+}
+
+extern "C" jd_status jd_decide_host(jd_model *m, const jd_row *rows, int32_t n_rows, const jd_encode_opts *opts,
+                                    jd_host_outputs *ho, void *stream) {
+    jd_batch *hb = nullptr;
+    int32_t bad = -1;
+    jd_status s = jd_serialize(rows, n_rows, opts, &hb, &bad);
+    if (s != JD_OK) return s;
+    s = jd_decide_packed_host(m, hb, ho, stream);
+    jd_batch_free(hb);
+    return s;
+}
+
+extern "C" jd_status jd_check_status(jd_model *m) {
+    clear_error();
+    if (!m) return fail(JD_ERR_INVALID_ARG, "model is NULL");
+    CK(cudaSetDevice(m->device));
+    CK(cudaStreamSynchronize(m->last_stream));
+    unsigned stv = 0;
+    CK(cudaMemcpy(&stv, m->status, sizeof(unsigned), cudaMemcpyDeviceToHost));
+    if (stv) return fail(JD_ERR_DEVICE_STATUS, "device status 0x%x (1: wait timeout, 2: token id range, 4: index)", stv);
+    return JD_OK;
+}

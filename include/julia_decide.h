@@ -1,0 +1,211 @@
+/*
+ * julia_decide.h -- C ABI of the B200 (sm_100a) Julia-1 decision-model library.
+ *
+ * The library computes the Julia-1 forward pass on pre-tokenized requests:
+ * (state, question, 2..20 options, type) rows in; raw option logits,
+ * per-question softmax probabilities and the choice / score / noul read-outs
+ * out.  Sources (page title, section):
+ *   "Julia-1: one score per mask token" -- "From a state to one decision"
+ *       (marker layout, budgets, strict mode), "The decision head" (forward
+ *       steps), "Three modes through one head" (read-outs);
+ *   "Julia-1 MLX" -- "API" (predict / logits / encoding_info over rows),
+ *       "Performance" (alternating attention, FP32 residual stream);
+ *   "julia1 -- Rust runtime for Julia-1" -- "Use" (validation errors match the
+ *       Python ValueError cases), "Why it is faster" (varlen packing, fused
+ *       epilogues, marker-only last head layer).
+ *
+ * Conventions
+ *   - Every call returns a jd_status; JD_OK is 0.  On failure a message for
+ *     the calling thread is available from jd_last_error().
+ *   - Host pointers are read during the call only.  Device pointers must stay
+ *     valid until the work queued on the caller's stream has completed.
+ *   - "stream" is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Device work is asynchronous on that stream; a kernel-side
+ *     check failure (bounded wait expired, id out of range) is recorded in a
+ *     device status word and reported by jd_check_status().
+ *   - One jd_model serves one stream at a time: its workspace is shared by
+ *     all calls on it.
+ *   - Nothing in the library falls back to the CPU: without a CUDA device
+ *     jd_model_create fails with JD_ERR_CUDA.
+ */
+#ifndef JULIA_DECIDE_H
+#define JULIA_DECIDE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    JD_OK = 0,
+    JD_ERR_INVALID_ARG = 1,    /* null pointer, bad option value, mismatched sizes */
+    JD_ERR_OPTION_COUNT = 2,   /* K outside [2, 20], or a noul row with K != 2 */
+    JD_ERR_OVERFLOW = 3,       /* strict budget violated, or nothing fits when truncating */
+    JD_ERR_TOKEN_RANGE = 4,    /* a token id outside [0, vocab) */
+    JD_ERR_CAPACITY = 5,       /* batch larger than the capacity given at jd_model_create */
+    JD_ERR_CUDA = 6,           /* a CUDA runtime / driver call failed */
+    JD_ERR_DEVICE_STATUS = 7,  /* a kernel reported a failed check (see jd_check_status) */
+    JD_ERR_IO = 8              /* weights file missing or malformed */
+} jd_status;
+
+/* Decision type = row index of the 3x384 type table ("The decision head", step 1). */
+typedef enum { JD_CHOICE = 0, JD_SCORE = 1, JD_NOUL = 2 } jd_type;
+
+/* Per-row truncation bits (non-strict encoding only; "Julia-1 MLX", "API":
+ * encoding_info reports whether anything was truncated). */
+enum {
+    JD_TRUNC_OPTION_48 = 1,   /* an option was clipped to 48 ids */
+    JD_TRUNC_OPTION_CAP = 2,  /* options were capped to fit the head budget */
+    JD_TRUNC_QUESTION = 4,    /* the question was clipped from its end */
+    JD_TRUNC_STATE = 8        /* the state was clipped to fit max_length */
+};
+
+/* One pre-tokenized request row (host memory).  The type prefix in words
+ * ("choice question: ...") is part of the caller's question ids.  For a noul
+ * row the options are [false, true] in that order. */
+typedef struct {
+    const int32_t *state;          /* [n_state] */
+    int32_t n_state;
+    const int32_t *question;       /* [n_question] */
+    int32_t n_question;
+    const int32_t *const *options; /* [k] pointers to each option's ids */
+    const int32_t *n_option_ids;   /* [k] */
+    int32_t k;                     /* number of options, 2..20 */
+    int32_t type;                  /* jd_type */
+} jd_row;
+
+/* Encoding options ("From a state to one decision": options <= 48 tokens,
+ * head budget 256 by default / 512 in the card's example, 8192 in all). */
+typedef struct {
+    int32_t max_length;   /* 1..8192 */
+    int32_t head_budget;  /* >= 1; tokens before the state */
+    int32_t strict;       /* nonzero: raise JD_ERR_OVERFLOW instead of truncating */
+    int32_t bos, eos, mask;
+    int32_t vocab;        /* ids must lie in [0, vocab) */
+} jd_encode_opts;
+
+/* A packed (unpadded, row after row) batch.  jd_serialize fills one in host
+ * memory that the library owns until jd_batch_free.  The same struct with
+ * DEVICE pointers (caller-owned) is the input of jd_forward / jd_decide. */
+typedef struct {
+    int32_t n_rows;         /* B */
+    int32_t n_tokens;       /* T = cu_seqlens[B] */
+    int32_t n_markers;      /* M = opt_off[B] */
+    int32_t max_row_len;    /* longest row, <= 8192 */
+    int32_t *tokens;        /* [T]   serialized ids, rows back to back */
+    int32_t *cu_seqlens;    /* [B+1] row r spans tokens [cu_seqlens[r], cu_seqlens[r+1]) */
+    int32_t *mask_pos;      /* [M]   absolute token index of each <mask> marker, row order */
+    int32_t *opt_off;       /* [B+1] row r's markers are mask_pos[opt_off[r] .. opt_off[r+1]) */
+    int32_t *row_type;      /* [B]   jd_type of each row */
+    int32_t *head_len;      /* [B]   tokens before the state (host batches only; may be NULL) */
+    uint8_t *trunc;         /* [B]   JD_TRUNC_* bits (host batches only; may be NULL) */
+} jd_batch;
+
+/* Device outputs (caller-owned device memory). */
+typedef struct {
+    float *logits;     /* [M] raw option logits, row order */
+    float *probs;      /* [M] softmax over each row's options (temperature 1) */
+    int32_t *choice;   /* [B] argmax option index (lowest index on ties) */
+    float *score;      /* [B] expected index sum_i i * p_i */
+    float *noul;       /* [B] p(true) = probs of option 1 for noul rows, NaN otherwise */
+    float *max_p;      /* [B] largest probability */
+} jd_outputs;
+
+/* Optional intermediate taps for validation (device memory, any may be NULL). */
+typedef struct {
+    float *encoder_out;   /* [T, 384] encoder output after the final norm (before the type row) */
+    float *marker_state;  /* [M, 384] marker states after both head layers (scorer input) */
+} jd_taps;
+
+enum { JD_PREC_BF16 = 0, JD_PREC_FP32 = 1 };
+enum { JD_SCORER_MLP = 0, JD_SCORER_LINEAR = 1 };
+enum { JD_ACT_RELU = 0, JD_ACT_GELU = 1 };
+
+typedef struct {
+    int32_t max_tokens;    /* capacity: packed tokens per call */
+    int32_t max_rows;      /* capacity: rows per call */
+    int32_t max_markers;   /* capacity: markers per call */
+    int32_t precision;     /* JD_PREC_BF16: BF16 tensor-core GEMMs / attention with FP32
+                              accumulation and an FP32 residual stream;
+                              JD_PREC_FP32: FP32 everywhere (validation mode) */
+    int32_t scorer;        /* JD_SCORER_MLP: LayerNorm -> Linear(384,384) -> GELU -> Linear(384,1)
+                              ("The decision head", step 4); JD_SCORER_LINEAR: LayerNorm -> Linear(384,1) */
+    int32_t head_act;      /* feed-forward activation of the two head layers (default ReLU) */
+} jd_model_config;
+
+typedef struct jd_model jd_model;
+
+/* Thread-local message of the last failed call on this thread ("" if none). */
+const char *jd_last_error(void);
+
+/* Library version string. */
+const char *jd_version(void);
+
+/* Serialize rows into a packed host batch ("From a state to one decision").
+ * Layout per row: <bos> question <eos> (<mask> option)_k <eos> state <eos>.
+ * Always errors: K outside [2,20] or noul with K != 2 (JD_ERR_OPTION_COUNT),
+ * an id outside [0, vocab) (JD_ERR_TOKEN_RANGE).  Strict: an option over 48
+ * ids, head over budget or total over max_length -> JD_ERR_OVERFLOW.
+ * Non-strict: clip options to 48 ids; if the head is over budget cap every
+ * option at the largest common length that fits (clip the question from its
+ * end if even one id per option does not fit); clip the state to fit
+ * max_length; report the JD_TRUNC_* bits per row.  On error *out is NULL and
+ * *bad_row (if non-NULL) receives the failing row index. */
+jd_status jd_serialize(const jd_row *rows, int32_t n_rows, const jd_encode_opts *opts,
+                       jd_batch **out, int32_t *bad_row);
+void jd_batch_free(jd_batch *batch);
+
+/* Load the .jdw weights file and allocate the device workspace for the given
+ * capacity on `device`.  BF16 copies of the projection weights are made here;
+ * the embedding table, norms, biases and head stay FP32. */
+jd_status jd_model_create(const jd_model_config *cfg, const char *weights_path, int device,
+                          jd_model **out);
+void jd_model_destroy(jd_model *model);
+
+/* Device bytes held by the model (weights + workspace). */
+size_t jd_model_device_bytes(const jd_model *model);
+
+/* Full forward pass and read-outs on a packed batch in device memory.
+ * `batch` is a host struct whose array pointers are device pointers (tokens,
+ * cu_seqlens, mask_pos, opt_off, row_type; head_len / trunc are ignored).
+ * n_tokens, n_rows, n_markers must not exceed the model's capacity
+ * (JD_ERR_CAPACITY).  All outputs of `out` are written; `taps` may be NULL. */
+jd_status jd_decide(jd_model *model, const jd_batch *batch, const jd_outputs *out,
+                    const jd_taps *taps, void *stream);
+
+/* Raw logits only (the "logits(rows)" call): writes logits[M]. */
+jd_status jd_forward(jd_model *model, const jd_batch *batch, float *logits, void *stream);
+
+/* Host outputs of jd_decide_host (caller-owned host memory, sizes as jd_outputs). */
+typedef struct {
+    float *logits; float *probs; int32_t *choice; float *score; float *noul; float *max_p;
+    int32_t n_rows, n_markers;    /* written by the call */
+} jd_host_outputs;
+
+/* End-to-end call: serialize `rows`, copy the packed batch to the device
+ * through the model's pinned staging buffers, run jd_decide, copy the
+ * outputs back and synchronize `stream`.  Output arrays must hold the total
+ * number of options (logits/probs) and n_rows entries. */
+jd_status jd_decide_host(jd_model *model, const jd_row *rows, int32_t n_rows,
+                         const jd_encode_opts *opts, jd_host_outputs *out, void *stream);
+
+/* Same as jd_decide_host, starting from an already serialized host batch. */
+jd_status jd_decide_packed_host(jd_model *model, const jd_batch *host_batch,
+                                jd_host_outputs *out, void *stream);
+
+/* Synchronize the model's last stream and read the device status word;
+ * JD_ERR_DEVICE_STATUS with a message if a kernel recorded a failure. */
+jd_status jd_check_status(jd_model *model);
+
+/* CUDA-graph replay for repeated calls of one batch shape: the first call
+ * with a given (n_tokens, n_rows, n_markers, batch pointers, outputs)
+ * captures the whole jd_decide launch sequence on `stream`; later calls with
+ * the same key replay it.  enable = 0 turns capture off (the default). */
+jd_status jd_set_graph_mode(jd_model *model, int enable);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* JULIA_DECIDE_H */

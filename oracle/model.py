@@ -230,3 +230,13 @@ class OracleModel:
         """Raw option logits for one serialised row (oracle.serialize.Encoded)."""
         h = self.hidden(enc.ids, enc.qtype)
         return scorer(h[np.asarray(enc.mask_pos, dtype=np.int64)], self.W, self.mo)
+
+    def forward_all(self, enc):
+        """The same pass, returning the encoder output (after the final norm),
+        the marker states after both head layers, and the logits."""
+        e = self.encode(enc.ids)
+        h = e + self.W["head.type_table"][enc.qtype]
+        for i in range(2):
+            h = head_layer(h, self.W, i, self.mo)
+        hm = h[np.asarray(enc.mask_pos, dtype=np.int64)]
+        return dict(encoder_out=e, marker_state=hm, logits=scorer(hm, self.W, self.mo))

@@ -1,0 +1,145 @@
+"""CPU tests of the C ABI: exported symbols, the host serializer against the
+oracle serializer (bit-exact) and loud failure without a CUDA device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from encoder_decision_model_b200 import _lib as jl
+from oracle import serialize_row, EncodeOptions, EncodingError
+from workloads import Row, rows_config0, rows_config1, rows_config2, rows_config3, requests_config4, worked_example_rows
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from encoder_decision_model_b200.build import build
+    build()
+    return jl.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    hdr = open(os.path.join(ROOT, "include", "julia_decide.h")).read()
+    names = set(re.findall(r"\b(jd_[a-z_]+)\s*\(", hdr))
+    assert len(names) >= 13
+    cdll = ctypes.CDLL(str(jl.LIB_PATH))
+    missing = [n for n in sorted(names) if not hasattr(cdll, n)]
+    assert not missing, missing
+
+
+def _oracle_pack(rows, opt):
+    encs = [serialize_row(r, opt) for r in rows]
+    ids = np.concatenate([e.ids for e in encs])
+    cu = np.cumsum([0] + [len(e.ids) for e in encs]).astype(np.int32)
+    mp = np.concatenate([e.mask_pos + cu[i] for i, e in enumerate(encs)]).astype(np.int32)
+    oo = np.cumsum([0] + [len(e.mask_pos) for e in encs]).astype(np.int32)
+    return encs, ids, cu, mp, oo
+
+
+def _compare(rows, max_length, head_budget, strict):
+    o = EncodeOptions(max_length=max_length, head_budget=head_budget, strict=strict)
+    encs, ids, cu, mp, oo = _oracle_pack(rows, o)
+    hb = jl.jd_serialize(rows, jl.encode_opts(max_length, head_budget, strict))
+    assert hb.n_rows == len(rows) and hb.n_tokens == len(ids) and hb.n_markers == len(mp)
+    np.testing.assert_array_equal(hb.tokens, ids)
+    np.testing.assert_array_equal(hb.cu_seqlens, cu)
+    np.testing.assert_array_equal(hb.mask_pos, mp)
+    np.testing.assert_array_equal(hb.opt_off, oo)
+    np.testing.assert_array_equal(hb.row_type, [r.qtype for r in rows])
+    np.testing.assert_array_equal(hb.trunc, [e.trunc for e in encs])
+    np.testing.assert_array_equal(hb.head_len, [e.head_len for e in encs])
+    assert hb.max_row_len == max(len(e.ids) for e in encs)
+
+
+def test_serializer_configs_bit_exact(L):
+    _compare(worked_example_rows(), 1024, 512, True)
+    _compare(rows_config0(), 8192, 256, True)
+    _compare(rows_config1(), 1024, 512, True)
+    _compare(rows_config2(256), 1024, 512, True)
+    _compare(rows_config3(4), 8192, 256, False)
+    reqs = requests_config4(8)
+    rows = [Row(state=r.state, question=r.question, options=r.labels[g:g + 20], qtype=0)
+            for r in reqs for g in range(0, 72, 20)]
+    _compare(rows, 1024, 512, True)
+
+
+def _rand_rows(rng, n):
+    rows = []
+    for _ in range(n):
+        k = int(rng.integers(2, 21))
+        qtype = int(rng.integers(0, 3))
+        if qtype == 2:
+            k = 2
+        rows.append(Row(state=rng.integers(10, 1000, size=int(rng.integers(0, 300))).astype(np.int32),
+                        question=rng.integers(10, 1000, size=int(rng.integers(0, 40))).astype(np.int32),
+                        options=[rng.integers(10, 1000, size=int(rng.integers(0, 70))).astype(np.int32)
+                                 for _ in range(k)], qtype=qtype))
+    return rows
+
+
+def test_serializer_random_nonstrict_bit_exact(L):
+    rng = np.random.default_rng(5)
+    for budget, maxlen in ((64, 128), (40, 100), (256, 300), (30, 35), (512, 8192)):
+        rows = _rand_rows(rng, 60)
+        ok = []
+        for r in rows:
+            try:
+                serialize_row(r, EncodeOptions(max_length=maxlen, head_budget=budget, strict=False))
+                ok.append(r)
+            except EncodingError:
+                pass
+        if ok:
+            _compare(ok, maxlen, budget, False)
+
+
+def test_serializer_error_codes_match_oracle(L):
+    rng = np.random.default_rng(9)
+    cases = []
+    base = _rand_rows(rng, 1)[0]
+    cases.append(Row(state=base.state, question=base.question, options=base.options[:1], qtype=0))
+    cases.append(Row(state=base.state, question=base.question, options=[base.question] * 21, qtype=0))
+    cases.append(Row(state=base.state, question=base.question, options=[base.question] * 3, qtype=2))
+    bad = base.state.copy() if len(base.state) else np.array([5], np.int32)
+    bad[0] = 256000
+    cases.append(Row(state=bad, question=base.question, options=base.options, qtype=base.qtype))
+    cases.append(Row(state=base.state, question=base.question, options=[np.arange(10, 60, dtype=np.int32)] * 2, qtype=1))
+    cases.append(Row(state=np.arange(10, 2000, dtype=np.int32), question=base.question, options=base.options[:2], qtype=0))
+    for strict in (True, False):
+        for r in cases:
+            o = EncodeOptions(max_length=512, head_budget=64, strict=strict)
+            try:
+                serialize_row(r, o)
+                want = 0
+            except EncodingError as e:
+                want = e.code
+            try:
+                jl.jd_serialize([r], jl.encode_opts(512, 64, strict))
+                got = 0
+            except jl.JDError as e:
+                got = e.code
+                assert e.bad_row == 0
+            assert got == want, (strict, got, want)
+
+
+def test_serializer_reports_failing_row(L):
+    rows = rows_config1()
+    bad = Row(state=rows[0].state, question=rows[0].question, options=rows[0].options[:1], qtype=0)
+    with pytest.raises(jl.JDError) as ei:
+        jl.jd_serialize(rows + [bad], jl.encode_opts(1024, 512, True))
+    assert ei.value.code == jl.JD_ERR_OPTION_COUNT and ei.value.bad_row == 3
+
+
+def test_model_create_fails_loudly_without_gpu(L, weights_file):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(jl.JDError) as ei:
+        jl.Model(weights_file, 1024, 4, 64)
+    assert ei.value.code == jl.JD_ERR_CUDA
+
+
+def test_version(L):
+    assert "sm_100a" in jl.jd_version()
