@@ -1,0 +1,462 @@
+#!/usr/bin/env python
+"""Benchmark of the Julia-1 decision-model forward pass on B200.
+
+One step = one full forward pass (serialised rows -> logits, probabilities,
+choice / score / noul) over one batch of the throughput workload: 1024 packed
+rows of 64..1024 tokens (2..20 options, head budget 512, strict), synthetic
+ids and random-init weights.  Multi-GPU: one process per GPU, each rank runs
+its own 1024 rows (rows are independent decisions; no collective on the data
+path), value = all ranks' decisions / max over ranks of the device time.
+
+Prints one JSON line on rank 0.  --impl reference times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decisions/s batched and p50 ms/call, Julia-1 forward on 1 B200 (BF16)"
+UNIT = "decisions/s"
+D, FF, HFF, NH = 384, 1152, 1536, 6
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--rows", type=int, default=1024, help="rows per rank and step")
+    ap.add_argument("--workload", default="throughput", choices=["throughput", "long"],
+                    help="throughput: 1024 rows of 64..1024 tokens; long: 16 rows of 8192 tokens")
+    ap.add_argument("--latency-calls", type=int, default=1000)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-steps", type=int, default=3)
+    ap.add_argument("--json-out", default=None)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- workload
+
+
+def workload(args, rank):
+    from workloads import rows_config2, rows_config3
+    if args.workload == "long":
+        rows = rows_config3(16, seed=103 + 1000 * rank)
+        opts = dict(max_length=8192, head_budget=256, strict=False)
+        desc = ("long context: 16 rows x 8192 tokens, 20 options (capped to the 256-token head budget, "
+                "non-strict), choice/score")
+    else:
+        rows = rows_config2(args.rows, seed=102 + 1000 * rank)
+        opts = dict(max_length=1024, head_budget=512, strict=True)
+        desc = (f"batched throughput: {args.rows} packed rows, lengths U[64,1024], 2..20 options of 1..48 ids, "
+                "types uniform, head budget 512, strict")
+    return rows, opts, desc
+
+
+def algorithmic_cost(name, lens, n_markers):
+    """(bytes, flops) per launch of kernel `name` for rows of lengths `lens`."""
+    lens = np.asarray(lens, dtype=np.float64)
+    T = lens.sum()
+    if name == "embed_ln":
+        return T * (4 + 1536 + 1536 + 768), T * 3 * D
+    if name in ("gemm_qkv_rope", "head0_gemm_in"):
+        return T * (768 + 2304), T * 2 * D * 3 * D
+    if name in ("gemm_wo_res_ln", "head0_gemm_out"):
+        return T * (768 + 1536 + 1536 + 768), T * 2 * D * D
+    if name == "gemm_wi_geglu":
+        return T * (768 + 2304), T * 2 * D * 2 * FF
+    if name == "gemm_wo2_res_ln":
+        return T * (2304 + 1536 + 1536 + 768), T * 2 * FF * D
+    if name == "head0_gemm_ffn1":
+        return T * (768 + 3072), T * 2 * D * HFF
+    if name == "head0_gemm_ffn2":
+        return T * (3072 + 1536 + 1536 + 768), T * 2 * HFF * D
+    if name in ("attn_global", "head0_attn"):
+        return T * (3 * 768 + 768), 4.0 * 64 * NH * float((lens ** 2).sum())
+    if name == "attn_local":
+        vis = 0.0
+        for L in lens.astype(np.int64):
+            i = np.arange(L)
+            vis += float((np.minimum(L - 1, i + 64) - np.maximum(0, i - 64) + 1).sum())
+        return T * (3 * 768 + 768), 4.0 * 64 * NH * vis
+    if name == "head1_gemm_kv":
+        return T * (768 + 1536), T * 2 * D * 2 * D
+    return None
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), tc_burst=float(d["bf16_tflops"]),
+                    tc_sust=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, tc_burst=1590.0, tc_sust=1400.0, src="fallback")
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "encoder_decision_model_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload_tag):
+    """DRAM bytes per token from a committed ncu summary, if its source hash
+    matches the current kernels (else None)."""
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    sha = kernel_source_sha()
+    for f in sorted(os.listdir(pdir)):
+        if not f.endswith(".md"):
+            continue
+        txt = open(os.path.join(pdir, f)).read()
+        for m in re.finditer(r"traffic\s+kernel=(\S+)\s+workload=(\S+)\s+dram_bytes_per_token=([0-9.eE+-]+)"
+                             r"\s+source_sha=(\S+)", txt):
+            if m.group(1) == kernel and m.group(2) == workload_tag and m.group(4) == sha:
+                return float(m.group(3))
+    return None
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = [l.split(",") for l in open(self.f.name).read().strip().splitlines() if l.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=mx, reasons=sorted(reasons), samples=len(sm))
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+
+def oracle_sample(rows, opts, seconds, min_rows=2):
+    """Time the oracle as it stands on the first rows until `seconds` elapse."""
+    from oracle import EncodeOptions, OracleModel, serialize_row, readouts
+    from workloads import weights_path
+    m = OracleModel(weights_path(0))
+    eo = EncodeOptions(max_length=opts["max_length"], head_budget=opts["head_budget"], strict=opts["strict"])
+    t0 = time.perf_counter()
+    n = toks = 0
+    for r in rows:
+        e = serialize_row(r, eo)
+        readouts(m.logits(e), e.qtype)
+        n += 1
+        toks += len(e.ids)
+        if time.perf_counter() - t0 >= seconds and n >= min_rows:
+            break
+    return n, toks, time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        th = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if th:
+            return int(max(th))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    rows, opts, desc = workload(args, 0)
+    per_step = 2 if args.workload == "throughput" else 1
+    cores = blas_threads()
+    for w in range(args.warmup):
+        oracle_sample(rows[w * per_step:(w + 1) * per_step], opts, 0.0, per_step)
+    n = toks = 0
+    el = 0.0
+    base = args.warmup * per_step
+    for s in range(args.steps):
+        sl = rows[(base + s * per_step) % len(rows):][:per_step]
+        a, b, t = oracle_sample(sl, opts, 0.0, per_step)
+        n += a
+        toks += b
+        el += t
+    v = n / el
+    sample = f"{n} rows ({toks} tokens) of the workload, {per_step} per step, float64 NumPy oracle"
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": desc, "rows_per_step": per_step},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    from encoder_decision_model_b200.build import build
+    if rank == 0:
+        build()
+    barrier()
+    from encoder_decision_model_b200 import _lib as jl
+    from workloads import weights_path
+
+    if rank == 0:
+        weights_path(0)
+    barrier()
+    rows, opts, desc = workload(args, rank)
+    hb = jl.jd_serialize(rows, jl.encode_opts(**opts))
+    T, B, M = hb.n_tokens, hb.n_rows, hb.n_markers
+    lens = np.diff(hb.cu_seqlens)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, toks, el = oracle_sample(rows, opts, args.cpu_seconds)
+        cpu = {"value": n / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"first {n} rows ({toks} tokens) of this workload, float64 NumPy oracle, {el:.1f} s"}
+
+    model = jl.Model(weights_path(0), T, B, M, precision=jl.JD_PREC_BF16, device=local)
+    up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    keep = [up(hb.tokens), up(hb.cu_seqlens), up(hb.mask_pos), up(hb.opt_off), up(hb.row_type)]
+    batch = jl.Model.device_batch(B, T, M, hb.max_row_len, *keep)
+    outs = dict(logits=torch.empty(M, device=dev), probs=torch.empty(M, device=dev),
+                choice=torch.empty(B, dtype=torch.int32, device=dev), score=torch.empty(B, device=dev),
+                noul=torch.empty(B, device=dev), max_p=torch.empty(B, device=dev))
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        model.jd_decide(batch, **outs, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        model.jd_check_status()
+        launches_per_step = model.jd_last_launch_count()
+
+        clocks = ClockSampler(local)
+        barrier()
+        torch.cuda.synchronize()
+        clocks.start()
+        time.sleep(0.3)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ck = clocks.stop()
+        ms = e0.elapsed_time(e1)
+        ms_max = max_over_ranks(ms)
+        model.jd_check_status()
+
+        # per-kernel event timing on the launching stream (separate profiled steps)
+        model.jd_set_profiling(True)
+        for _ in range(args.profile_steps):
+            step()
+        prof = model.jd_profile_report()
+        model.jd_set_profiling(False)
+        torch.cuda.synchronize()
+
+    decisions = sum_over_ranks(float(B * args.steps))
+    tokens = sum_over_ranks(float(T * args.steps))
+    value = decisions / (ms_max / 1000.0)
+
+    # ---- end to end through the host entry point: serialise + H2D + forward + D2H
+    e2e_steps = max(3, min(args.steps, 10))
+    hopts = jl.encode_opts(**opts)
+    model.jd_decide_host(rows, hopts)  # warm
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        model.jd_decide_host(rows, hopts)
+    e2e_s = max_over_ranks(time.perf_counter() - t0)
+    e2e_val = sum_over_ranks(float(B * e2e_steps)) / e2e_s
+    h2d = 4 * (T + (B + 1) + M + (B + 1) + B)
+    d2h = 4 * (2 * M + 4 * B)
+
+    # ---- batch-1 latency: the 3-question request on one 200-token state, graph replay
+    lat = {}
+    if rank == 0 and args.latency_calls > 0:
+        from workloads import rows_config1
+        r1 = rows_config1()
+        o1 = jl.encode_opts(1024, 512, True)
+        lm = jl.Model(weights_path(0), 2048, 8, 64, precision=jl.JD_PREC_BF16, device=local)
+        lm.jd_set_graph_mode(True)
+        for _ in range(20):
+            lm.jd_decide_host(r1, o1)
+        ts = []
+        for _ in range(args.latency_calls):
+            t = time.perf_counter()
+            lm.jd_decide_host(r1, o1)
+            ts.append(1000 * (time.perf_counter() - t))
+        lat = dict(p50_ms_per_call=float(np.percentile(ts, 50)), p99_ms_per_call=float(np.percentile(ts, 99)),
+                   latency_workload="3 questions (choice/4, score/3, noul/2) on one 200-token state, "
+                                    "jd_decide_host with CUDA-graph replay, host serialisation and copies included")
+        lm.close()
+
+    # ---- roofline of the dominant kernel
+    peaks = read_peaks()
+    roof = None
+    per_kernel = {}
+    for name, (n, tot) in prof.items():
+        per_kernel[name] = dict(launches_per_step=n // max(1, args.profile_steps), ms_per_step=tot / args.profile_steps)
+    if prof:
+        top = max(prof, key=lambda k: prof[k][1])
+        n, tot = prof[top]
+        avg_s = tot / n / 1000.0
+        cost = algorithmic_cost(top, lens, M)
+        if cost is not None:
+            byt, fl = cost
+            t_hbm = byt / (peaks["hbm"] * 1e9)
+            t_tc = fl / (peaks["tc_sust"] * 1e12)
+            wl_tag = args.workload
+            tr = recorded_traffic(top, wl_tag)
+            if t_tc > t_hbm:
+                ach = fl / avg_s / 1e12
+                roof = {"bound": "tensor", "achieved": ach, "peak": peaks["tc_sust"], "unit": "TFLOP/s",
+                        "frac": ach / peaks["tc_sust"], "traffic": None if tr is None else tr * T,
+                        "kernel": top, "peak_source": f"{peaks['src']} sustained bf16 (cuBLAS)"}
+            else:
+                ach = byt / avg_s / 1e9
+                roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                        "frac": ach / peaks["hbm"], "traffic": None if tr is None else tr * T,
+                        "kernel": top, "peak_source": f"{peaks['src']} copy bandwidth"}
+            roof["algorithmic_per_launch"] = {"bytes": byt, "flops": fl}
+            roof["avg_launch_ms"] = avg_s * 1000.0
+            roof["kernel_source_sha"] = kernel_source_sha()
+        for name, d in per_kernel.items():
+            c = algorithmic_cost(name, lens, M)
+            if c is None or d["launches_per_step"] == 0:
+                continue
+            a = d["ms_per_step"] / d["launches_per_step"] / 1000.0
+            d["hbm_frac"] = c[0] / a / 1e9 / peaks["hbm"]
+            d["tensor_frac"] = c[1] / a / 1e12 / peaks["tc_sust"]
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": desc, "global_batch": int(B * world), "rows_per_gpu": int(B),
+                       "tokens_per_gpu_step": int(T), "markers_per_gpu_step": int(M),
+                       "parallelism": f"dp{world} (independent rows per rank, no collective)",
+                       "l2": "inputs larger than L2 (FP32 residual stream of one step alone is "
+                             f"{T * 1536 / 1e6:.0f} MB)",
+                       "weights": "random init N(0,0.02), seed 0"},
+            "tokens_per_s": tokens / (ms_max / 1000.0),
+            **lat,
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "call": "jd_decide_host (serialise + H2D from pinned staging + forward + D2H + sync)"},
+            "gpu_launches": int(launches_per_step * args.steps),
+            "clocks": ck, "per_kernel": per_kernel}
+    if rank == 0:
+        s = json.dumps(line)
+        print(s, flush=True)
+        if args.json_out:
+            open(args.json_out, "w").write(s + "\n")
+    model.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -97,8 +97,13 @@ def lib():
     L.jd_decide_packed_host.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.POINTER(jd_host_outputs), C.c_void_p]
     L.jd_check_status.argtypes = [C.c_void_p]
     L.jd_set_graph_mode.argtypes = [C.c_void_p, C.c_int]
+    L.jd_last_launch_count.argtypes = [C.c_void_p]
+    L.jd_last_launch_count.restype = C.c_int32
+    L.jd_set_profiling.argtypes = [C.c_void_p, C.c_int]
+    L.jd_profile_report.argtypes = [C.c_void_p, C.c_char_p, C.c_size_t]
     for name in ("jd_serialize", "jd_model_create", "jd_decide", "jd_forward", "jd_decide_host",
-                 "jd_decide_packed_host", "jd_check_status", "jd_set_graph_mode"):
+                 "jd_decide_packed_host", "jd_check_status", "jd_set_graph_mode", "jd_set_profiling",
+                 "jd_profile_report"):
         getattr(L, name).restype = C.c_int
     _lib = L
     return L
@@ -245,6 +250,22 @@ class Model:
 
     def jd_set_graph_mode(self, enable):
         _check(lib().jd_set_graph_mode(self.h, int(bool(enable))))
+
+    def jd_last_launch_count(self):
+        return lib().jd_last_launch_count(self.h)
+
+    def jd_set_profiling(self, enable):
+        _check(lib().jd_set_profiling(self.h, int(bool(enable))))
+
+    def jd_profile_report(self):
+        """{kernel name: (launches, total ms)} summed since profiling was enabled."""
+        buf = C.create_string_buffer(1 << 16)
+        _check(lib().jd_profile_report(self.h, buf, len(buf)))
+        out = {}
+        for line in buf.value.decode().splitlines():
+            name, n, ms = line.split()
+            out[name] = (int(n), float(ms))
+        return out
 
     def _host_out(self, n_rows, n_markers):
         o = dict(logits=np.zeros(n_markers, np.float32), probs=np.zeros(n_markers, np.float32),

@@ -193,6 +193,14 @@ struct jd_model {
     int *h_choice = nullptr;
 
     cudaStream_t last_stream = nullptr;
+    int launches = 0;
+
+    // per-kernel event timing (profiling mode)
+    bool prof = false;
+    std::vector<cudaEvent_t> ev;
+    std::vector<const char *> ev_name;
+    int n_ev = 0;
+    std::map<std::string, std::pair<long, double>> prof_acc;
 
     // CUDA graph cache (one entry)
     bool graph_mode = false;
@@ -438,14 +446,27 @@ T *offset(void *p, size_t elems, bool fp32) {
         if (e_ != cudaSuccess) return fail(JD_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
     } while (0)
 
+// Launch with optional per-kernel event timing and a launch count.
+#define KL(name, nk, call)                                                     \
+    do {                                                                       \
+        if (m->prof && m->n_ev < (int)m->ev.size()) {                          \
+            LK(cudaEventRecord(m->ev[m->n_ev], st));                           \
+            m->ev_name[m->n_ev++] = (name);                                    \
+        }                                                                      \
+        LK(call);                                                              \
+        m->launches += (nk);                                                   \
+    } while (0)
+
 // The whole launch sequence (no allocation, no synchronisation).
 jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out, const jd_taps *taps,
                           cudaStream_t st) {
     const bool f32 = m->fp32;
+    m->launches = 0;
+    m->n_ev = 0;
     const int T = b->n_tokens, B = b->n_rows, M = b->n_markers;
     LK(cudaMemsetAsync(m->status, 0, sizeof(unsigned), st));
-    LK(launch_prep(b->cu_seqlens, B, T, m->tok_row, m->pos, m->qb_off, st));
-    LK(launch_embed_ln(b->tokens, T, m->E, VOCAB, m->emb_g, EPS, m->x, m->xn, f32, m->status, st));
+    KL("prep", 2, launch_prep(b->cu_seqlens, B, T, m->tok_row, m->pos, m->qb_off, st));
+    KL("embed_ln", 1, launch_embed_ln(b->tokens, T, m->E, VOCAB, m->emb_g, EPS, m->x, m->xn, f32, m->status, st));
 
     AttnArgs aa;
     aa.qkv = m->qkv;
@@ -465,22 +486,22 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.rope = glob ? m->rope_g : m->rope_l;
         e.pos = m->pos;
         e.rope_cols = 2 * D;
-        LK(launch_gemm(make_op(EPI_QKV, 384, m->Wqkv[l], &m->tm_xn, m->xn, D, e), f32, st));
+        KL("gemm_qkv_rope", 1, launch_gemm(make_op(EPI_QKV, 384, m->Wqkv[l], &m->tm_xn, m->xn, D, e), f32, st));
 
         aa.window = glob ? -1 : 64;
-        LK(launch_attention(aa, f32, st));
+        KL(glob ? "attn_global" : "attn_local", 1, launch_attention(aa, f32, st));
 
         e = base_ep(m, T);
         e.out = m->xn;
         e.ldo = D;
         e.resid = m->x;
         e.ln_g = m->mlp_g[l];
-        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo[l], &m->tm_o, m->o, D, e), f32, st));
+        KL("gemm_wo_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo[l], &m->tm_o, m->o, D, e), f32, st));
 
         e = base_ep(m, T);
         e.out = m->y;
         e.ldo = FF;
-        LK(launch_gemm(make_op(EPI_GEGLU, 256, m->Wi[l], &m->tm_xn, m->xn, D, e), f32, st));
+        KL("gemm_wi_geglu", 1, launch_gemm(make_op(EPI_GEGLU, 256, m->Wi[l], &m->tm_xn, m->xn, D, e), f32, st));
 
         e = base_ep(m, T);
         e.out = m->xn;
@@ -497,7 +518,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
             e.ln_g = m->n1g[0];
             e.ln_b = m->n1b[0];
         }
-        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo2[l], &m->tm_y_enc, m->y, FF, e), f32, st));
+        KL("gemm_wo2_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo2[l], &m->tm_y_enc, m->y, FF, e), f32, st));
     }
 
     // ---- head layer 0 (all tokens)
@@ -506,9 +527,9 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.out = m->qkv;
         e.ldo = QKV;
         e.bias = m->in_b[0];
-        LK(launch_gemm(make_op(EPI_QKV, 384, m->in_full[0], &m->tm_xn, m->xn, D, e), f32, st));
+        KL("head0_gemm_in", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_full[0], &m->tm_xn, m->xn, D, e), f32, st));
         aa.window = -1;
-        LK(launch_attention(aa, f32, st));
+        KL("head0_attn", 1, launch_attention(aa, f32, st));
         e = base_ep(m, T);
         e.out = m->xn;
         e.ldo = D;
@@ -516,12 +537,12 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.resid = m->x;
         e.ln_g = m->n2g[0];
         e.ln_b = m->n2b[0];
-        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->out_p[0], &m->tm_o, m->o, D, e), f32, st));
+        KL("head0_gemm_out", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->out_p[0], &m->tm_o, m->o, D, e), f32, st));
         e = base_ep(m, T);
         e.out = m->y;
         e.ldo = HFF;
         e.bias = m->l1_b[0];
-        LK(launch_gemm(make_op(EPI_BIAS_ACT, 256, m->lin1[0], &m->tm_xn, m->xn, D, e), f32, st));
+        KL("head0_gemm_ffn1", 1, launch_gemm(make_op(EPI_BIAS_ACT, 256, m->lin1[0], &m->tm_xn, m->xn, D, e), f32, st));
         e = base_ep(m, T);
         e.out = m->xn;
         e.ldo = D;
@@ -529,7 +550,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.resid = m->x;
         e.ln_g = m->n1g[1];
         e.ln_b = m->n1b[1];
-        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[0], &m->tm_y_head, m->y, HFF, e), f32, st));
+        KL("head0_gemm_ffn2", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[0], &m->tm_y_head, m->y, HFF, e), f32, st));
     }
     // ---- head layer 1: keys / values for every token, the rest at the markers only
     {
@@ -537,14 +558,14 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.out = offset<uint8_t>(m->qkv, D, f32);
         e.ldo = QKV;
         e.bias = m->in_b[1] + D;
-        LK(launch_gemm(make_op(EPI_QKV, 384, m->in_kv[1], &m->tm_xn, m->xn, D, e), f32, st));
-        LK(launch_gather_markers(b->mask_pos, M, T, m->x, m->xn, m->hm, m->xm, f32, m->status, st));
+        KL("head1_gemm_kv", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_kv[1], &m->tm_xn, m->xn, D, e), f32, st));
+        KL("head1_gather", 1, launch_gather_markers(b->mask_pos, M, T, m->x, m->xn, m->hm, m->xm, f32, m->status, st));
         e = base_ep(m, M);
         e.out = m->qm;
         e.ldo = D;
         e.bias = m->in_b[1];
-        LK(launch_gemm(make_op(EPI_QKV, 384, m->in_q[1], &m->tm_xm, m->xm, D, e), f32, st));
-        LK(launch_marker_attention(m->qm, m->qkv, m->om, b->cu_seqlens, b->opt_off, b->mask_pos, B, f32, st));
+        KL("head1_gemm_q", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_q[1], &m->tm_xm, m->xm, D, e), f32, st));
+        KL("head1_marker_attn", 1, launch_marker_attention(m->qm, m->qkv, m->om, b->cu_seqlens, b->opt_off, b->mask_pos, B, f32, st));
         e = base_ep(m, M);
         e.out = m->xnm;
         e.ldo = D;
@@ -552,16 +573,16 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.resid = m->hm;
         e.ln_g = m->n2g[1];
         e.ln_b = m->n2b[1];
-        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->out_p[1], &m->tm_om, m->om, D, e), f32, st));
+        KL("head1_gemm_out", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->out_p[1], &m->tm_om, m->om, D, e), f32, st));
         e = base_ep(m, M);
         e.out = m->ym;
         e.ldo = HFF;
         e.bias = m->l1_b[1];
-        LK(launch_gemm(make_op(EPI_BIAS_ACT, 256, m->lin1[1], &m->tm_xnm, m->xnm, D, e), f32, st));
+        KL("head1_gemm_ffn1", 1, launch_gemm(make_op(EPI_BIAS_ACT, 256, m->lin1[1], &m->tm_xnm, m->xnm, D, e), f32, st));
         e = base_ep(m, M);
         e.bias = m->l2_b[1];
         e.resid = m->hm;
-        LK(launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[1], &m->tm_ym, m->ym, HFF, e), f32, st));
+        KL("head1_gemm_ffn2", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[1], &m->tm_ym, m->ym, HFF, e), f32, st));
     }
     // ---- scorer + read-outs
     ScorerArgs sa;
@@ -577,9 +598,26 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
     sa.eps = EPS;
     sa.logits = out->logits;
     sa.tap = taps ? taps->marker_state : nullptr;
-    LK(launch_scorer(sa, st));
-    LK(launch_readout(out->logits, b->opt_off, b->row_type, B, out->probs, out->choice, out->score, out->noul,
+    KL("scorer", 1, launch_scorer(sa, st));
+    KL("readout", 1, launch_readout(out->logits, b->opt_off, b->row_type, B, out->probs, out->choice, out->score, out->noul,
                       out->max_p, st));
+    if (m->prof && m->n_ev < (int)m->ev.size()) {
+        LK(cudaEventRecord(m->ev[m->n_ev], st));
+        m->ev_name[m->n_ev++] = nullptr;
+    }
+    return JD_OK;
+}
+
+// Fold the events of the last profiled call into the per-kernel totals.
+jd_status collect_profile(jd_model *m, cudaStream_t st) {
+    CK(cudaStreamSynchronize(st));
+    for (int i = 0; i + 1 < m->n_ev; ++i) {
+        float ms = 0.f;
+        CK(cudaEventElapsedTime(&ms, m->ev[i], m->ev[i + 1]));
+        auto &acc = m->prof_acc[m->ev_name[i]];
+        acc.first += 1;
+        acc.second += ms;
+    }
     return JD_OK;
 }
 
@@ -648,6 +686,7 @@ extern "C" void jd_model_destroy(jd_model *m) {
     if (!m) return;
     cudaSetDevice(m->device);
     if (m->gexec) cudaGraphExecDestroy(m->gexec);
+    for (cudaEvent_t e : m->ev) cudaEventDestroy(e);
     for (void *p : m->allocs) cudaFree(p);
     for (void *p : m->hallocs) cudaFreeHost(p);
     delete m;
@@ -672,6 +711,10 @@ extern "C" jd_status jd_decide(jd_model *m, const jd_batch *b, const jd_outputs 
     CK(cudaSetDevice(m->device));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     m->last_stream = st;
+    if (m->prof) {
+        TRY(enqueue_forward(m, b, out, taps, st));
+        return collect_profile(m, st);
+    }
     if (!m->graph_mode) return enqueue_forward(m, b, out, taps, st);
 
     std::vector<uintptr_t> key = {(uintptr_t)b->n_tokens,  (uintptr_t)b->n_rows,     (uintptr_t)b->n_markers,
@@ -786,5 +829,35 @@ extern "C" jd_status jd_check_status(jd_model *m) {
     unsigned stv = 0;
     CK(cudaMemcpy(&stv, m->status, sizeof(unsigned), cudaMemcpyDeviceToHost));
     if (stv) return fail(JD_ERR_DEVICE_STATUS, "device status 0x%x (1: wait timeout, 2: token id range, 4: index)", stv);
+    return JD_OK;
+}
+
+extern "C" int32_t jd_last_launch_count(const jd_model *m) { return m ? m->launches : 0; }
+
+extern "C" jd_status jd_set_profiling(jd_model *m, int enable) {
+    clear_error();
+    if (!m) return fail(JD_ERR_INVALID_ARG, "model is NULL");
+    CK(cudaSetDevice(m->device));
+    if (enable && m->ev.empty()) {
+        m->ev.resize(192);
+        m->ev_name.resize(192);
+        for (auto &e : m->ev) CK(cudaEventCreate(&e));
+    }
+    m->prof = enable != 0;
+    m->prof_acc.clear();
+    return JD_OK;
+}
+
+extern "C" jd_status jd_profile_report(jd_model *m, char *buf, size_t n) {
+    clear_error();
+    if (!m || !buf || n == 0) return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    std::string s;
+    char line[160];
+    for (auto &kv : m->prof_acc) {
+        snprintf(line, sizeof(line), "%s %ld %.6f\n", kv.first.c_str(), kv.second.first, kv.second.second);
+        s += line;
+    }
+    if (s.size() + 1 > n) return fail(JD_ERR_INVALID_ARG, "buffer too small (%zu bytes needed)", s.size() + 1);
+    memcpy(buf, s.c_str(), s.size() + 1);
     return JD_OK;
 }

@@ -205,6 +205,21 @@ jd_status jd_check_status(jd_model *model);
  * the same key replay it.  enable = 0 turns capture off (the default). */
 jd_status jd_set_graph_mode(jd_model *model, int enable);
 
+/* Number of kernels the last jd_decide / jd_forward call launched (the same
+ * sequence whether replayed from a graph or launched eagerly). */
+int32_t jd_last_launch_count(const jd_model *model);
+
+/* Per-kernel timing for measurement: when enabled, every launch of the
+ * sequence is bracketed by CUDA events on the caller's stream, each call
+ * synchronizes that stream before returning, and the elapsed times are summed
+ * per kernel name.  Enabling (or disabling) clears the sums.  Graph replay is
+ * not used while profiling. */
+jd_status jd_set_profiling(jd_model *model, int enable);
+
+/* Write the sums as text lines "name launches total_ms" into buf (size n).
+ * JD_ERR_INVALID_ARG if buf is too small. */
+jd_status jd_profile_report(jd_model *model, char *buf, size_t n);
+
 #ifdef __cplusplus
 }
 #endif
