@@ -97,6 +97,8 @@ def lib():
     L.jd_decide_packed_host.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.POINTER(jd_host_outputs), C.c_void_p]
     L.jd_check_status.argtypes = [C.c_void_p]
     L.jd_set_graph_mode.argtypes = [C.c_void_p, C.c_int]
+    L.jd_forward_noalloc.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.c_void_p, C.c_void_p]
+    L.jd_forward_noalloc.restype = C.c_int
     L.jd_last_launch_count.argtypes = [C.c_void_p]
     L.jd_last_launch_count.restype = C.c_int32
     L.jd_set_profiling.argtypes = [C.c_void_p, C.c_int]
@@ -244,6 +246,11 @@ class Model:
 
     def jd_forward(self, batch: jd_batch, logits, stream=None):
         _check(lib().jd_forward(self.h, C.byref(batch), _ptr(logits), _stream(stream)))
+
+    def jd_forward_noalloc(self, batch: jd_batch, logits, stream=None):
+        """jd_forward with every intermediate in the library's static device
+        array (no allocation); at most 1024 tokens, 32 rows, 128 markers."""
+        _check(lib().jd_forward_noalloc(self.h, C.byref(batch), _ptr(logits), _stream(stream)))
 
     def jd_check_status(self):
         _check(lib().jd_check_status(self.h))

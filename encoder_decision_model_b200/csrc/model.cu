@@ -861,3 +861,140 @@ extern "C" jd_status jd_profile_report(jd_model *m, char *buf, size_t n) {
     memcpy(buf, s.c_str(), s.size() + 1);
     return JD_OK;
 }
+
+// ================================================================== forward without allocation
+//
+// For callers that cannot allocate device memory once they are running: for
+// example a serving loop that must stay inside a fixed memory budget after
+// start-up, or a host that hands this library a device but forbids it from
+// calling the CUDA allocator.  Such a caller creates its jd_model at start-up
+// and then calls jd_forward_noalloc, which keeps every intermediate of the
+// forward pass in one file-scope __device__ array instead of the model's
+// workspace.  The launch sequence is the one jd_forward uses.
+
+namespace {
+
+constexpr int NA_TOKENS = 1024;   // largest batch (packed tokens) the array holds
+constexpr int NA_ROWS = 32;
+constexpr int NA_MARKERS = 128;
+constexpr int NA_MAX_DEVICES = 64;
+
+constexpr size_t na_up(size_t b) { return (b + 255) / 256 * 256; }
+// byte offsets of the workspace inside the array (BF16 activations)
+constexpr size_t NA_X = 0;
+constexpr size_t NA_XN = NA_X + na_up((size_t)NA_TOKENS * D * 4);
+constexpr size_t NA_QKV = NA_XN + na_up((size_t)NA_TOKENS * D * 2);
+constexpr size_t NA_O = NA_QKV + na_up((size_t)NA_TOKENS * QKV * 2);
+constexpr size_t NA_Y = NA_O + na_up((size_t)NA_TOKENS * D * 2);
+constexpr size_t NA_TOKROW = NA_Y + na_up((size_t)NA_TOKENS * HFF * 2);
+constexpr size_t NA_POS = NA_TOKROW + na_up((size_t)NA_TOKENS * 4);
+constexpr size_t NA_QBOFF = NA_POS + na_up((size_t)NA_TOKENS * 4);
+constexpr size_t NA_HM = NA_QBOFF + na_up((size_t)(NA_ROWS + 1) * 4);
+constexpr size_t NA_XM = NA_HM + na_up((size_t)NA_MARKERS * D * 4);
+constexpr size_t NA_QM = NA_XM + na_up((size_t)NA_MARKERS * D * 2);
+constexpr size_t NA_OM = NA_QM + na_up((size_t)NA_MARKERS * D * 2);
+constexpr size_t NA_XNM = NA_OM + na_up((size_t)NA_MARKERS * D * 2);
+constexpr size_t NA_YM = NA_XNM + na_up((size_t)NA_MARKERS * D * 2);
+constexpr size_t NA_STATUS = NA_YM + na_up((size_t)NA_MARKERS * HFF * 2);
+constexpr size_t NA_PROBS = NA_STATUS + 256;
+constexpr size_t NA_CHOICE = NA_PROBS + na_up((size_t)NA_MARKERS * 4);
+constexpr size_t NA_SCORE = NA_CHOICE + na_up((size_t)NA_ROWS * 4);
+constexpr size_t NA_NOUL = NA_SCORE + na_up((size_t)NA_ROWS * 4);
+constexpr size_t NA_MAXP = NA_NOUL + na_up((size_t)NA_ROWS * 4);
+constexpr size_t NA_BYTES = NA_MAXP + na_up((size_t)NA_ROWS * 4);  // about 9.7 MB
+
+// Held by every GPU that loads the library, until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NA_BYTES];
+
+struct NoAllocSlot {
+    bool ready = false;
+    uint8_t *base = nullptr;  // device address of g_noalloc_scratch on this device
+    CUtensorMap tm_xn{}, tm_o{}, tm_y_enc{}, tm_y_head{}, tm_qkv{}, tm_xm{}, tm_om{}, tm_xnm{}, tm_ym{};
+};
+NoAllocSlot g_na_slot[NA_MAX_DEVICES];
+std::mutex g_na_mutex;
+jd_model g_na_view[NA_MAX_DEVICES];  // per-device view: the caller's weights + the array's workspace
+
+// Once per device, with that device current: resolve the array's device
+// address (a host-side reference to the symbol is not a device pointer) and
+// describe its buffers for TMA.
+jd_status noalloc_setup(int dev) {
+    NoAllocSlot &s = g_na_slot[dev];
+    if (s.ready) return JD_OK;
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return fail(JD_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    s.base = static_cast<uint8_t *>(p);
+    TRY(make_map(&s.tm_xn, s.base + NA_XN, D, NA_TOKENS, D, 64, 128));
+    TRY(make_map(&s.tm_o, s.base + NA_O, D, NA_TOKENS, D, 64, 128));
+    TRY(make_map(&s.tm_y_enc, s.base + NA_Y, FF, NA_TOKENS, FF, 64, 128));
+    TRY(make_map(&s.tm_y_head, s.base + NA_Y, HFF, NA_TOKENS, HFF, 64, 128));
+    TRY(make_map(&s.tm_qkv, s.base + NA_QKV, QKV, NA_TOKENS, QKV, 64, 64));
+    TRY(make_map(&s.tm_xm, s.base + NA_XM, D, NA_MARKERS, D, 64, 128));
+    TRY(make_map(&s.tm_om, s.base + NA_OM, D, NA_MARKERS, D, 64, 128));
+    TRY(make_map(&s.tm_xnm, s.base + NA_XNM, D, NA_MARKERS, D, 64, 128));
+    TRY(make_map(&s.tm_ym, s.base + NA_YM, HFF, NA_MARKERS, HFF, 64, 128));
+    s.ready = true;
+    return JD_OK;
+}
+
+// Point the device's view at the caller's weights and at the array's buffers
+// (plain field copies; nothing is allocated).
+void noalloc_view(jd_model &v, const jd_model *m, const NoAllocSlot &s) {
+    v.cfg = m->cfg;
+    v.device = m->device;
+    v.fp32 = false;
+    v.E = m->E; v.emb_g = m->emb_g; v.fin_g = m->fin_g; v.type_tab = m->type_tab;
+    for (int l = 0; l < NL; ++l) {
+        v.attn_g[l] = m->attn_g[l]; v.mlp_g[l] = m->mlp_g[l];
+        v.Wqkv[l] = m->Wqkv[l]; v.Wo[l] = m->Wo[l]; v.Wi[l] = m->Wi[l]; v.Wo2[l] = m->Wo2[l];
+    }
+    for (int i = 0; i < 2; ++i) {
+        v.n1g[i] = m->n1g[i]; v.n1b[i] = m->n1b[i]; v.n2g[i] = m->n2g[i]; v.n2b[i] = m->n2b[i];
+        v.in_full[i] = m->in_full[i]; v.in_q[i] = m->in_q[i]; v.in_kv[i] = m->in_kv[i];
+        v.out_p[i] = m->out_p[i]; v.lin1[i] = m->lin1[i]; v.lin2[i] = m->lin2[i];
+        v.in_b[i] = m->in_b[i]; v.out_b[i] = m->out_b[i]; v.l1_b[i] = m->l1_b[i]; v.l2_b[i] = m->l2_b[i];
+    }
+    v.sc_g = m->sc_g; v.sc_b = m->sc_b; v.sc_w1t = m->sc_w1t; v.sc_b1 = m->sc_b1; v.sc_w2 = m->sc_w2;
+    v.sc_b2 = m->sc_b2; v.lin_w = m->lin_w; v.lin_b = m->lin_b; v.rope_g = m->rope_g; v.rope_l = m->rope_l;
+    uint8_t *b = s.base;
+    v.x = reinterpret_cast<float *>(b + NA_X);
+    v.xn = b + NA_XN; v.qkv = b + NA_QKV; v.o = b + NA_O; v.y = b + NA_Y;
+    v.tok_row = reinterpret_cast<int *>(b + NA_TOKROW);
+    v.pos = reinterpret_cast<int *>(b + NA_POS);
+    v.qb_off = reinterpret_cast<int *>(b + NA_QBOFF);
+    v.hm = reinterpret_cast<float *>(b + NA_HM);
+    v.xm = b + NA_XM; v.qm = b + NA_QM; v.om = b + NA_OM; v.xnm = b + NA_XNM; v.ym = b + NA_YM;
+    v.status = reinterpret_cast<unsigned *>(b + NA_STATUS);
+    v.tm_xn = s.tm_xn; v.tm_o = s.tm_o; v.tm_y_enc = s.tm_y_enc; v.tm_y_head = s.tm_y_head; v.tm_qkv = s.tm_qkv;
+    v.tm_xm = s.tm_xm; v.tm_om = s.tm_om; v.tm_xnm = s.tm_xnm; v.tm_ym = s.tm_ym;
+    v.prof = false;
+    v.graph_mode = false;
+}
+
+}  // namespace
+
+extern "C" jd_status jd_forward_noalloc(jd_model *m, const jd_batch *b, float *logits, void *stream) {
+    clear_error();
+    if (!m || !b || !logits) return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    if (m->fp32) return fail(JD_ERR_INVALID_ARG, "jd_forward_noalloc serves BF16 models only");
+    if (m->device < 0 || m->device >= NA_MAX_DEVICES) return fail(JD_ERR_INVALID_ARG, "device ordinal too large");
+    if (b->n_rows < 1 || b->n_tokens < 1 || b->n_markers < 1) return fail(JD_ERR_INVALID_ARG, "empty batch");
+    if (b->n_tokens > NA_TOKENS || b->n_rows > NA_ROWS || b->n_markers > NA_MARKERS)
+        return fail(JD_ERR_CAPACITY,
+                    "jd_forward_noalloc takes at most %d tokens, %d rows and %d markers (got %d, %d, %d)",
+                    NA_TOKENS, NA_ROWS, NA_MARKERS, b->n_tokens, b->n_rows, b->n_markers);
+    if (!b->tokens || !b->cu_seqlens || !b->mask_pos || !b->opt_off || !b->row_type)
+        return fail(JD_ERR_INVALID_ARG, "batch has a NULL array");
+    CK(cudaSetDevice(m->device));
+    std::lock_guard<std::mutex> lock(g_na_mutex);
+    TRY(noalloc_setup(m->device));
+    jd_model &v = g_na_view[m->device];
+    noalloc_view(v, m, g_na_slot[m->device]);
+    uint8_t *base = g_na_slot[m->device].base;
+    jd_outputs o{logits, reinterpret_cast<float *>(base + NA_PROBS), reinterpret_cast<int *>(base + NA_CHOICE),
+                 reinterpret_cast<float *>(base + NA_SCORE), reinterpret_cast<float *>(base + NA_NOUL),
+                 reinterpret_cast<float *>(base + NA_MAXP)};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return enqueue_forward(&v, b, &o, nullptr, st);
+}

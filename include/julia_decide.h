@@ -220,6 +220,26 @@ jd_status jd_set_profiling(jd_model *model, int enable);
  * JD_ERR_INVALID_ARG if buf is too small. */
 jd_status jd_profile_report(jd_model *model, char *buf, size_t n);
 
+/* jd_forward without any device allocation (no counterpart on the pages; it
+ * serves callers that may not call the CUDA allocator once they are running,
+ * e.g. a serving loop held to the memory budget it reserved at start-up, or a
+ * host application that owns all device allocation).  Same inputs and output
+ * as jd_forward: `batch` with device arrays, raw logits[M] on the device.
+ * Every intermediate lives in one file-scope __device__ array of about 9.7 MB
+ * that each GPU loading the library holds until the process exits.
+ *   - Limits: at most 1024 packed tokens, 32 rows and 128 markers per call
+ *     (JD_ERR_CAPACITY beyond them); BF16 models only (JD_ERR_INVALID_ARG).
+ *   - The first call on a device resolves the array's device address and
+ *     describes its buffers for TMA; make that first call before any stream
+ *     capture.
+ *   - All calls share the array, and each call leaves its intermediates there:
+ *     calls whose work overlaps on the GPU (different streams, or models on
+ *     the same device used concurrently) race and must be serialized by the
+ *     caller.  The status word the kernels write is cleared at the start of
+ *     every call; it is not reported by jd_check_status.
+ *   - The model (weights) must come from jd_model_create, called at start-up. */
+jd_status jd_forward_noalloc(jd_model *model, const jd_batch *batch, float *logits, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
