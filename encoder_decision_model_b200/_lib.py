@@ -61,6 +61,16 @@ class jd_host_outputs(C.Structure):
                 ("max_p", f32p), ("n_rows", C.c_int32), ("n_markers", C.c_int32)]
 
 
+class jd_route_request(C.Structure):
+    _fields_ = [("state", i32p), ("n_state", C.c_int32), ("question", i32p), ("n_question", C.c_int32),
+                ("labels", C.POINTER(i32p)), ("n_label_ids", i32p), ("n_labels", C.c_int32)]
+
+
+class jd_route_outputs(C.Structure):
+    _fields_ = [("winner", i32p), ("winner_p", f32p), ("final_candidates", i32p), ("final_probs", f32p),
+                ("rows_per_round", i32p), ("max_rounds", C.c_int32), ("n_rounds", C.c_int32)]
+
+
 class JDError(RuntimeError):
     def __init__(self, code, msg):
         super().__init__(f"[{code}] {msg}")
@@ -97,6 +107,9 @@ def lib():
     L.jd_decide_packed_host.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.POINTER(jd_host_outputs), C.c_void_p]
     L.jd_check_status.argtypes = [C.c_void_p]
     L.jd_set_graph_mode.argtypes = [C.c_void_p, C.c_int]
+    L.jd_route_host.argtypes = [C.c_void_p, C.POINTER(jd_route_request), C.c_int32, C.POINTER(jd_encode_opts),
+                                C.c_int32, C.c_int32, C.c_int32, C.POINTER(jd_route_outputs), C.c_void_p]
+    L.jd_route_host.restype = C.c_int
     L.jd_forward_noalloc.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.c_void_p, C.c_void_p]
     L.jd_forward_noalloc.restype = C.c_int
     L.jd_last_launch_count.argtypes = [C.c_void_p]
@@ -246,6 +259,35 @@ class Model:
 
     def jd_forward(self, batch: jd_batch, logits, stream=None):
         _check(lib().jd_forward(self.h, C.byref(batch), _ptr(logits), _stream(stream)))
+
+    def jd_route_host(self, requests, opts: jd_encode_opts, max_tokens=None, max_rows=None, max_markers=None,
+                      stream=None):
+        """Route requests (objects with state/question/labels); returns dict of
+        winner, winner_p, final_candidates [n, 20], final_probs [n, 20], rows_per_round."""
+        keep = []
+        arr = (jd_route_request * max(1, len(requests)))()
+        for i, r in enumerate(requests):
+            st = np.ascontiguousarray(r.state, dtype=np.int32)
+            q = np.ascontiguousarray(r.question, dtype=np.int32)
+            labs = [np.ascontiguousarray(x, dtype=np.int32) for x in r.labels]
+            lp = (i32p * len(labs))(*[x.ctypes.data_as(i32p) for x in labs])
+            ln = np.asarray([len(x) for x in labs], dtype=np.int32)
+            keep += [st, q, labs, lp, ln]
+            arr[i] = jd_route_request(st.ctypes.data_as(i32p), len(st), q.ctypes.data_as(i32p), len(q), lp,
+                                      ln.ctypes.data_as(i32p), len(labs))
+        n = len(requests)
+        o = dict(winner=np.zeros(n, np.int32), winner_p=np.zeros(n, np.float32),
+                 final_candidates=np.zeros((n, 20), np.int32), final_probs=np.zeros((n, 20), np.float32),
+                 rows_per_round=np.zeros(16, np.int32))
+        s = jd_route_outputs(o["winner"].ctypes.data_as(i32p), o["winner_p"].ctypes.data_as(f32p),
+                             o["final_candidates"].ctypes.data_as(i32p), o["final_probs"].ctypes.data_as(f32p),
+                             o["rows_per_round"].ctypes.data_as(i32p), 16, 0)
+        c = self.cfg
+        _check(lib().jd_route_host(self.h, arr, n, C.byref(opts), int(max_tokens or c.max_tokens),
+                                   int(max_rows or c.max_rows), int(max_markers or c.max_markers), C.byref(s),
+                                   _stream(stream)))
+        o["rows_per_round"] = o["rows_per_round"][:s.n_rounds]
+        return o
 
     def jd_forward_noalloc(self, batch: jd_batch, logits, stream=None):
         """jd_forward with every intermediate in the library's static device

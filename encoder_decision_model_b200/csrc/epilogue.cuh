@@ -72,6 +72,10 @@ __device__ __forceinline__ void ln_regs(float (&v)[12], const float *g, const fl
     }
 }
 
+// Second half of the residual epilogue for one row whose sum v = x + acc (+ bias) is in registers.
+template <typename OutT>
+__device__ __forceinline__ void epi_resid_ln_finish(float (&v)[12], int row, const EpiParams &ep, int lane);
+
 template <typename OutT>
 __device__ __forceinline__ void epi_resid_ln_row(const float *acc, int row, const EpiParams &ep, int lane) {
     float v[12];
@@ -88,6 +92,50 @@ __device__ __forceinline__ void epi_resid_ln_row(const float *acc, int row, cons
         v[4 * j + 2] = x.z + a.z + b.z;
         v[4 * j + 3] = x.w + a.w + b.w;
     }
+    epi_resid_ln_finish<OutT>(v, row, ep, lane);
+}
+
+// R rows (row0 + u * rstep, u < n) per warp with every global load issued
+// before the first use, so that a warp keeps R residual rows in flight.
+template <typename OutT, int R>
+__device__ __forceinline__ void epi_resid_ln_rows(const float *acc0, int pitch, int row0, int rstep, int n,
+                                                  const EpiParams &ep, int lane) {
+    float v[R][12];
+    float4 b[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+        b[j] = ep.bias ? *reinterpret_cast<const float4 *>(ep.bias + j * 128 + lane * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < R; ++u) {
+        if (u < n) {
+            const float *xr = ep.resid + (size_t)(row0 + u * rstep) * D;
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                const float4 x = *reinterpret_cast<const float4 *>(xr + j * 128 + lane * 4);
+                v[u][4 * j + 0] = x.x; v[u][4 * j + 1] = x.y; v[u][4 * j + 2] = x.z; v[u][4 * j + 3] = x.w;
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < R; ++u) {
+        if (u < n) {
+            const float *acc = acc0 + (size_t)u * rstep * pitch;
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                const float4 a = *reinterpret_cast<const float4 *>(acc + j * 128 + lane * 4);
+                v[u][4 * j + 0] += a.x + b[j].x;
+                v[u][4 * j + 1] += a.y + b[j].y;
+                v[u][4 * j + 2] += a.z + b[j].z;
+                v[u][4 * j + 3] += a.w + b[j].w;
+            }
+            epi_resid_ln_finish<OutT>(v[u], row0 + u * rstep, ep, lane);
+        }
+    }
+}
+
+template <typename OutT>
+__device__ __forceinline__ void epi_resid_ln_finish(float (&v)[12], int row, const EpiParams &ep, int lane) {
+    float *xr = ep.resid + (size_t)row * D;
     if (ep.fin_g) {
         ln_regs(v, ep.fin_g, nullptr, lane, ep.eps);
         const int t = ep.row_type[ep.tok_row[row]];

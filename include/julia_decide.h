@@ -195,6 +195,41 @@ jd_status jd_decide_host(jd_model *model, const jd_row *rows, int32_t n_rows,
 jd_status jd_decide_packed_host(jd_model *model, const jd_batch *host_batch,
                                 jd_host_outputs *out, void *stream);
 
+/* A choice question over up to 4096 candidate labels (host memory). */
+typedef struct {
+    const int32_t *state;
+    int32_t n_state;
+    const int32_t *question;
+    int32_t n_question;
+    const int32_t *const *labels;  /* [n_labels] pointers to each label's ids */
+    const int32_t *n_label_ids;    /* [n_labels] */
+    int32_t n_labels;              /* 1..4096 */
+} jd_route_request;
+
+/* Router outputs (host memory, caller-owned; optional arrays may be NULL). */
+typedef struct {
+    int32_t *winner;            /* [n_requests] index of the chosen label */
+    float *winner_p;            /* [n_requests] its probability in the final call (1 if unscored) */
+    int32_t *final_candidates;  /* optional [n_requests * 20] label indices of the final call, -1 padded */
+    float *final_probs;         /* optional [n_requests * 20] their probabilities */
+    int32_t *rows_per_round;    /* optional [max_rounds] rows scored per round, all requests together */
+    int32_t max_rounds;
+    int32_t n_rounds;           /* written: rounds including the final call */
+} jd_route_outputs;
+
+/* Router ("Julia-1: one score per mask token", "More than 20 options: the
+ * Router"): per round, each request with more than 20 candidates is split in
+ * order into consecutive groups of at most 20; all groups of all requests are
+ * scored together (one batch per round, chunked to max_tokens / max_rows /
+ * max_markers, which must not exceed the model's capacity); a group keeps its
+ * winner alone if its probability is above 0.95 and every other is below 0.045,
+ * else its two most probable candidates, in their original order; a group of
+ * one passes through unscored.  With 20 or fewer left, one final call per
+ * request picks the winner.  Rows are encoded with `opts` as choice rows. */
+jd_status jd_route_host(jd_model *model, const jd_route_request *requests, int32_t n_requests,
+                        const jd_encode_opts *opts, int32_t max_tokens, int32_t max_rows, int32_t max_markers,
+                        jd_route_outputs *out, void *stream);
+
 /* Synchronize the model's last stream and read the device status word;
  * JD_ERR_DEVICE_STATUS with a message if a kernel recorded a failure. */
 jd_status jd_check_status(jd_model *model);
