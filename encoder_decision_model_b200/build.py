@@ -45,16 +45,19 @@ def _stale():
     return any(p.stat().st_mtime > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> Path:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False, defines=(), out=None,
+          objdir=None) -> Path:
+    target = Path(out) if out else OUT
+    if not force and out is None and not _stale():
         return OUT
     nvcc = _nvcc()
-    BUILD.mkdir(parents=True, exist_ok=True)
+    bdir = Path(objdir) if objdir else BUILD
+    bdir.mkdir(parents=True, exist_ok=True)
     inc = ["-I", str(INCLUDE), "-I", str(CSRC)]
-    extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+    extra = (["-Xptxas", "-v"] if ptxas_verbose else []) + [f"-D{d}" for d in defines]
 
     def compile_one(src: Path):
-        obj = BUILD / (src.name + ".o")
+        obj = bdir / (src.name + ".o")
         cmd = [nvcc, *ARCH, *NVCC_FLAGS, *inc, *extra, "-c", str(src), "-o", str(obj)]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -66,14 +69,14 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     for _, log in results:
         if log.strip() and (verbose or ptxas_verbose):
             print(log, file=sys.stderr)
-    tmp = OUT.with_suffix(".so.tmp")
+    tmp = target.with_suffix(".so.tmp")
     cmd = [nvcc, *ARCH, "-shared", "-o", str(tmp), *[str(o) for o, _ in results], "-lcuda" if False else "-lcudart_static",
            "-lpthread", "-ldl", "-lrt"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
-    os.replace(tmp, OUT)
-    return OUT
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

@@ -232,6 +232,146 @@ __global__ void __launch_bounds__(128)
     }
 }
 
+
+// Sliding-window (+-64) variant: the CTA's 64 queries need the 192-key band
+// [q0 - 64, q0 + 128), loaded once by TMA (three 64 x 64 tiles of K and of V);
+// warp w's 16 queries need only the 144 keys [q0 + 16w - 64, q0 + 16w + 80),
+// i.e. nine 16-key chunks, so each warp visits just those and runs an exact
+// two-pass softmax over them in registers (no running rescale).
+constexpr int LW_CHUNKS = 9;  // (16 + 2 * 64) / 16
+
+__global__ void __launch_bounds__(128)
+    k_attn_local_bf16(const __grid_constant__ CUtensorMap tm, __nv_bfloat16 *__restrict__ out,
+                      const int *__restrict__ cu, const int *__restrict__ qb_off, int n_rows, unsigned *status) {
+    extern __shared__ uint8_t sm_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = sm;                  // 64 x 64
+    uint8_t *sK = sm + 8192;           // 3 tiles of 64 x 64
+    uint8_t *sV = sm + 4 * 8192;       // 3 tiles
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 7 * 8192);
+
+    const int tile = blockIdx.x, h = blockIdx.y;
+    if (tile >= qb_off[n_rows]) return;
+    const int row = find_row(qb_off, n_rows, tile);
+    const int cs = cu[row], ce = cu[row + 1];
+    const int q0 = cs + (tile - qb_off[row]) * BQ;
+    const int kbase = q0 - 64;         // band start (may precede the row: masked)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar, 7 * 8192);
+        tma_load_2d(sQ, &tm, bar, h * DH, q0);
+        for (int t = 0; t < 3; ++t) {
+            tma_load_2d(sK + t * 8192, &tm, bar, D + h * DH, kbase + t * 64);
+            tma_load_2d(sV + t * 8192, &tm, bar, 2 * D + h * DH, kbase + t * 64);
+        }
+    }
+    __syncthreads();
+    if (!mbar_wait(bar, 0, status)) return;
+
+    const float sl2 = 0.125f * 1.4426950408889634f;
+    const int g = lane >> 2, tq = lane & 3;
+    const int qi0 = q0 + warp * 16 + g, qi1 = qi0 + 8;
+    uint32_t qf[4][4];
+    {
+        const uint32_t base = smem_u32(sQ);
+        const int r = warp * 16 + (lane & 15);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            ldsm_x4(base + sw128(r, kk * 2 + (lane >> 4)), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+    }
+    // S over the warp's nine 16-key chunks (band chunks warp .. warp + 8)
+    float sc[2 * LW_CHUNKS][4];
+#pragma unroll
+    for (int j = 0; j < 2 * LW_CHUNKS; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < LW_CHUNKS; ++cc) {
+        const int kc = warp + cc;                  // 16-key chunk inside the band
+        const uint32_t kb = smem_u32(sK + (kc >> 2) * 8192);
+        const int kr = (kc & 3) * 16 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kb + sw128(kr, kk * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
+            mma_bf16(sc[2 * cc], qf[kk], b0, b1);
+            mma_bf16(sc[2 * cc + 1], qf[kk], b2, b3);
+        }
+    }
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int kj = kbase + (warp * 2 + j) * 8 + 2 * tq + e;
+            const bool in_row = kj >= cs && kj < ce;
+            const bool v0 = in_row && abs(qi0 - kj) <= 64, v1 = in_row && abs(qi1 - kj) <= 64;
+            sc[j][e] = v0 ? sc[j][e] * sl2 : -INFINITY;
+            sc[j][2 + e] = v1 ? sc[j][2 + e] * sl2 : -INFINITY;
+            mx0 = fmaxf(mx0, sc[j][e]);
+            mx1 = fmaxf(mx1, sc[j][2 + e]);
+        }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float mu0 = mx0 == -INFINITY ? 0.f : mx0, mu1 = mx1 == -INFINITY ? 0.f : mx1;
+    float l0 = 0.f, l1 = 0.f;
+    uint32_t pa[LW_CHUNKS][4];
+#pragma unroll
+    for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
+        const float p0 = exp2f(sc[j][0] - mu0), p1 = exp2f(sc[j][1] - mu0);
+        const float p2 = exp2f(sc[j][2] - mu1), p3 = exp2f(sc[j][3] - mu1);
+        l0 += p0 + p1;
+        l1 += p2 + p3;
+        pa[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p0, p1);
+        pa[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+    }
+    float o[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < LW_CHUNKS; ++cc) {
+        const int kc = warp + cc;
+        const uint32_t vb = smem_u32(sV + (kc >> 2) * 8192);
+        const int vr = (kc & 3) * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+        for (int dp = 0; dp < 4; ++dp) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(vb + sw128(vr, dp * 2 + (lane >> 4)), b0, b1, b2, b3);
+            mma_bf16(o[2 * dp], pa[cc], b0, b1);
+            mma_bf16(o[2 * dp + 1], pa[cc], b2, b3);
+        }
+    }
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    uint8_t *stg = sQ;  // the warp's own 16 rows of the Q tile (its Q fragments are in registers)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int col = j * 8 + 2 * tq;
+        const int r0 = warp * 16 + g, r1 = r0 + 8;
+        *reinterpret_cast<uint32_t *>(stg + sw128(r0, col >> 3) + (col & 7) * 2) = pack_bf16x2(o[j][0] * i0, o[j][1] * i0);
+        *reinterpret_cast<uint32_t *>(stg + sw128(r1, col >> 3) + (col & 7) * 2) = pack_bf16x2(o[j][2] * i1, o[j][3] * i1);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int e = lane + 32 * it;
+        const int r = e >> 3, c = e & 7;
+        const int qi = q0 + warp * 16 + r;
+        if (qi < ce) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(stg + sw128(warp * 16 + r, c));
+            *reinterpret_cast<uint4 *>(out + (size_t)qi * D + h * DH + c * 8) = v;
+        }
+    }
+}
+
 // ------------------------------------------------------------------ FP32 validation attention
 
 template <bool LOCAL>
@@ -297,6 +437,10 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+cudaError_t attn_init_attributes() {
+    return cudaFuncSetAttribute(k_attn_local_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, 7 * 8192 + 64 + 1024);
+}
+
 cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st) {
     if (a.n_rows <= 0 || a.n_tokens <= 0) return cudaSuccess;
     const int max_tiles = (a.n_tokens + BQ - 1) / BQ + a.n_rows;
@@ -311,7 +455,10 @@ cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st) {
                                                     a.n_rows, a.window);
     } else {
         const int smem = 5 * 8192 + 64 + 1024;
-        if (local)
+        if (local && a.window == 64)
+            k_attn_local_bf16<<<grid, 128, 7 * 8192 + 64 + 1024, st>>>(*a.tm_qkv, (__nv_bfloat16 *)a.o, a.cu_seqlens,
+                                                                       a.qb_off, a.n_rows, a.status);
+        else if (local)
             k_attn_bf16<true><<<grid, 128, smem, st>>>(*a.tm_qkv, (__nv_bfloat16 *)a.o, a.cu_seqlens, a.qb_off,
                                                        a.n_rows, a.window, a.status);
         else

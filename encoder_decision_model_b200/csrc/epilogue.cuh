@@ -31,6 +31,7 @@ struct EpiParams {
     int ldo;
     const float *bias;       // [N] by weight row, or null
     const float2 *rope;      // [MAX_POS][32] (cos, sin), or null
+    int out_col0;            // column offset of this launch's output inside the tensor map (BF16 path)
     const int *pos;          // [rows] position within the request row
     int rope_cols;           // output columns [0, rope_cols) are rotated
     float *resid;            // [rows, 384] FP32 residual stream (RESID_LN)

@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(256, 1)
     }
 }
 
-// ---------------------------------------------------------------- persistent BF16 GEMM (N-split epilogues)
+// ---------------------------------------------------------------- persistent BF16 GEMM (column-split epilogues)
 //
 // One CTA per SM loops over 128 x BN tiles (tile t -> m = t / NB, n = t % NB,
 // so the NB column blocks of one row block run side by side and share A in
@@ -172,42 +172,82 @@ __global__ void __launch_bounds__(256, 1)
 //   warp 0 lane 0  TMA producer (A 128 x 64, W BN x 64 per stage)
 //   warp 1         TMEM allocation; lane 0 issues tcgen05.mma
 //   warps 2..5     epilogue, one accumulator row per thread (TMEM lane
-//                  quarter = warp % 4), results stored straight to global
+//                  quarter = warp % 4); QKV and bias+activation outputs are
+//                  staged per warp as 32 rows x 64 columns (bf16, 128-byte
+//                  swizzle) in shared memory and written by one TMA bulk
+//                  store each (double-buffered); GEGLU outputs go straight
+//                  from registers to global memory.
 template <int BN>
 struct PcCfg {
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (BN <= 192) ? 5 : 4;
-    static constexpr int DATA = STAGES * STAGE;
+    static constexpr int STAGES = 4;
+    static constexpr int RING = STAGES * STAGE;
+    static constexpr int OUT_BOX = 32 * 128;           // 32 rows x 64 bf16
+    static constexpr int OUT = 4 * 2 * OUT_BOX;        // 4 warps x 2 buffers
+    static constexpr int DATA = RING + OUT;
     static constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 8;
     static constexpr int SMEM = DATA + BAR_BYTES + 1024;
-    static constexpr uint32_t BUF_COLS = 256;  // column stride of the two accumulators
+    static constexpr uint32_t BUF_COLS = 256;          // column stride of the two accumulators
 };
 
+// Per-warp double-buffered staging of 32 x 64 bf16 boxes for TMA stores.
+struct OutStage {
+    uint8_t *base;   // this warp's two 4 KB buffers
+    uint32_t count;  // boxes issued so far
+    __device__ __forceinline__ uint8_t *begin(int lane) {
+        if (count >= 2) {
+            if (lane == 0) bulk_wait_read<1>();  // the store that used this buffer has read it
+            __syncwarp();
+        }
+        return base + (count & 1) * 4096;
+    }
+    __device__ __forceinline__ void commit(uint8_t *buf, const CUtensorMap *map, int x, int y, int lane) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(map, buf, x, y);
+            bulk_commit();
+        }
+        ++count;
+    }
+};
+
+// Write 4 x 16 bytes (32 bf16) of row r into 16-byte chunks c0..c0+3 of a swizzled box.
+__device__ __forceinline__ void stage_row32(uint8_t *box, int r, int c0, const uint32_t (&w)[16]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4 *>(box + r * 128 + (((c0 + q) ^ (r & 7)) << 4)) =
+            make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+}
+
 template <int EPI, int BN>
-__device__ __forceinline__ void pc_epilogue_row(uint32_t tacc, int row, bool valid, int n0, const EpiParams &ep,
-                                                const float2 (&cs)[32], bool have_cs) {
-    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(ep.out) + (size_t)row * ep.ldo;
+__device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0, int n0, const EpiParams &ep,
+                                                 const CUtensorMap *tmO, OutStage &os, int lane,
+                                                 const float2 (&cs)[32], bool have_cs) {
     if constexpr (EPI == EPI_GEGLU) {
+        // stored straight from registers: a shared-memory staging pass here
+        // competes with the 256-wide MMAs for shared-memory bandwidth
         constexpr int G = BN / 2;
+        const int row = row0 + r;
+        __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(ep.out) + (size_t)row * ep.ldo + n0 / 2;
 #pragma unroll 1
         for (int c = 0; c < G; c += 32) {
             uint32_t u[32], g[32];
             tmem_ld32(tacc + c, u);
             tmem_ld32(tacc + G + c, g);
             tmem_ld_wait();
-            if (valid) {
-                uint4 *dst = reinterpret_cast<uint4 *>(o + n0 / 2 + c);
+            if (row < ep.rows) {
+                uint4 *dst = reinterpret_cast<uint4 *>(o + c);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int j = q * 8 + e * 2;
-                        const float y0 = gelu_erf(__uint_as_float(u[j])) * __uint_as_float(g[j]);
-                        const float y1 = gelu_erf(__uint_as_float(u[j + 1])) * __uint_as_float(g[j + 1]);
-                        w[e] = pack_bf16x2(y0, y1);
+                        w[e] = pack_bf16x2(gelu_erf(__uint_as_float(u[j])) * __uint_as_float(g[j]),
+                                           gelu_erf(__uint_as_float(u[j + 1])) * __uint_as_float(g[j + 1]));
                     }
                     dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
@@ -215,75 +255,79 @@ __device__ __forceinline__ void pc_epilogue_row(uint32_t tacc, int row, bool val
         }
     } else if constexpr (EPI == EPI_BIAS_ACT) {
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-            uint32_t a[32];
-            tmem_ld32(tacc + c, a);
-            tmem_ld_wait();
-            if (valid) {
-                uint4 *dst = reinterpret_cast<uint4 *>(o + n0 + c);
-                const float *bb = ep.bias + n0 + c;
+        for (int c = 0; c < BN; c += 64) {
+            uint8_t *box = os.begin(lane);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t w[4];
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t a[32], w[16];
+                tmem_ld32(tacc + c + 32 * hh, a);
+                tmem_ld_wait();
+                const float4 *bb = reinterpret_cast<const float4 *>(ep.bias + n0 + c + 32 * hh);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = q * 8 + e * 2;
-                        float y0 = __uint_as_float(a[j]) + (bb ? bb[j] : 0.f);
-                        float y1 = __uint_as_float(a[j + 1]) + (bb ? bb[j + 1] : 0.f);
-                        if (ep.act == 0) { y0 = fmaxf(y0, 0.f); y1 = fmaxf(y1, 0.f); }
-                        else { y0 = gelu_erf(y0); y1 = gelu_erf(y1); }
-                        w[e] = pack_bf16x2(y0, y1);
-                    }
-                    dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 b = ep.bias ? bb[j4] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    float y[4] = {__uint_as_float(a[4 * j4]) + b.x, __uint_as_float(a[4 * j4 + 1]) + b.y,
+                                  __uint_as_float(a[4 * j4 + 2]) + b.z, __uint_as_float(a[4 * j4 + 3]) + b.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) y[e] = ep.act == 0 ? fmaxf(y[e], 0.f) : gelu_erf(y[e]);
+                    w[2 * j4] = pack_bf16x2(y[0], y[1]);
+                    w[2 * j4 + 1] = pack_bf16x2(y[2], y[3]);
                 }
+                stage_row32(box, r, 4 * hh, w);
             }
+            os.commit(box, tmO, ep.out_col0 + n0 + c, row0, lane);
         }
     } else {  // EPI_QKV: 64-column heads, rotary pairs (i, i + 32) on columns < rope_cols
 #pragma unroll 1
         for (int h = 0; h < BN; h += 64) {
-            uint32_t a[32], b[32];
+            uint8_t *box = os.begin(lane);
+            uint32_t a[32], b[32], w1[16], w2[16];
             tmem_ld32(tacc + h, a);
             tmem_ld32(tacc + h + 32, b);
             tmem_ld_wait();
-            if (!valid) continue;
             const int n = n0 + h;
             const bool rot = have_cs && n < ep.rope_cols;
-            uint4 *d1 = reinterpret_cast<uint4 *>(o + n);
-            uint4 *d2 = reinterpret_cast<uint4 *>(o + n + 32);
+            float ba[32], bb[32];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t w1[4], w2[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float r[2], s[2];
-#pragma unroll
-                    for (int t = 0; t < 2; ++t) {
-                        const int j = q * 8 + e * 2 + t;
-                        float x1 = __uint_as_float(a[j]), x2 = __uint_as_float(b[j]);
-                        if (ep.bias) { x1 += ep.bias[n + j]; x2 += ep.bias[n + 32 + j]; }
-                        if (rot) {
-                            const float2 c2 = cs[j];
-                            r[t] = x1 * c2.x - x2 * c2.y;
-                            s[t] = x2 * c2.x + x1 * c2.y;
-                        } else {
-                            r[t] = x1;
-                            s[t] = x2;
-                        }
-                    }
-                    w1[e] = pack_bf16x2(r[0], r[1]);
-                    w2[e] = pack_bf16x2(s[0], s[1]);
+            for (int j4 = 0; j4 < 8; ++j4) {
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+                if (ep.bias) {
+                    x = reinterpret_cast<const float4 *>(ep.bias + n)[j4];
+                    y = reinterpret_cast<const float4 *>(ep.bias + n + 32)[j4];
                 }
-                d1[q] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-                d2[q] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+                ba[4 * j4] = x.x; ba[4 * j4 + 1] = x.y; ba[4 * j4 + 2] = x.z; ba[4 * j4 + 3] = x.w;
+                bb[4 * j4] = y.x; bb[4 * j4 + 1] = y.y; bb[4 * j4 + 2] = y.z; bb[4 * j4 + 3] = y.w;
             }
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                float r2[2], s2[2];
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const int jj = j + t;
+                    const float x1 = __uint_as_float(a[jj]) + ba[jj];
+                    const float x2 = __uint_as_float(b[jj]) + bb[jj];
+                    if (rot) {
+                        r2[t] = x1 * cs[jj].x - x2 * cs[jj].y;
+                        s2[t] = x2 * cs[jj].x + x1 * cs[jj].y;
+                    } else {
+                        r2[t] = x1;
+                        s2[t] = x2;
+                    }
+                }
+                w1[j >> 1] = pack_bf16x2(r2[0], r2[1]);
+                w2[j >> 1] = pack_bf16x2(s2[0], s2[1]);
+            }
+            stage_row32(box, r, 0, w1);
+            stage_row32(box, r, 4, w2);
+            os.commit(box, tmO, ep.out_col0 + n, row0, lane);
         }
     }
 }
 
 template <int EPI, int BN>
 __global__ void __launch_bounds__(192, 1)
-    k_gemm_pc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int K, int n_tiles,
-              int nblk, EpiParams ep) {
+    k_gemm_pc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmO, int K, int n_tiles, int nblk, EpiParams ep) {
     using C = PcCfg<BN>;
     static_assert(BN <= 256, "one MMA per k-step");
     extern __shared__ uint8_t smem_raw[];
@@ -310,6 +354,7 @@ __global__ void __launch_bounds__(192, 1)
         fence_proxy_async_smem();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        prefetch_tmap(&tmO);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -366,17 +411,17 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else {
         const int q = warp & 3;  // TMEM lane quarter of this warp
+        OutStage os{smem + C::RING + (warp - 2) * 2 * C::OUT_BOX, 0u};
         uint32_t tc = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tc) {
             const int m0 = (t / nblk) * 128, n0 = (t % nblk) * BN;
-            const int row = m0 + q * 32 + lane;
-            const bool valid = row < ep.rows;
+            const int row0 = m0 + q * 32;
             float2 cs[32];
             bool have_cs = false;
             if constexpr (EPI == EPI_QKV) {
                 if (ep.rope && n0 < ep.rope_cols) {
-                    const int pos = valid ? ep.pos[row] : 0;
-                    const float4 *src = reinterpret_cast<const float4 *>(ep.rope + (size_t)pos * 32);
+                    const int row = row0 + lane;
+                    const float4 *src = reinterpret_cast<const float4 *>(ep.rope + (size_t)(row < ep.rows ? ep.pos[row] : 0) * 32);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const float4 v = src[i];
@@ -391,11 +436,274 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
             tc_fence_after();
             const uint32_t tacc = tmem + buf * C::BUF_COLS + ((uint32_t)(q * 32) << 16);
-            pc_epilogue_row<EPI, BN>(tacc, row, valid, n0, ep, cs, have_cs);
+            pc_epilogue_rows<EPI, BN>(tacc, lane, row0, n0, ep, &tmO, os, lane, cs, have_cs);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acce[buf]);
         }
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- persistent residual + LayerNorm GEMM
+//
+// x[rows, 384] += A . W^T (+ bias);  xn = LN(x) * g (+ b), one CTA per SM
+// looping over 128-row tiles; the 384 accumulator columns stay in one TMEM
+// buffer, so the overlap comes from the producer running ahead (the next
+// tile's A / W stages load while this tile's epilogue streams the residual).
+//   warp 0 lane 0  TMA producer: A box 128 x 64, W as two 192 x 64 boxes
+//   warp 1         TMEM allocation; lane 0 issues the N = 2 x 192 MMAs
+//   warps 2..5     epilogue, one row per thread:
+//     pass 1  per 32-column chunk: the residual chunk (128 x 32 FP32, 128-byte
+//             swizzle) arrives by TMA (three buffers, prefetched across
+//             tiles); v = x + acc (+ bias) is written back in place, stored to
+//             x by TMA and parked in TMEM; row mean and M2 are merged chunk by
+//             chunk (Chan's pairwise update), so one pass yields the moments;
+//     pass 2  xn = LN(v) from TMEM into 128 x 64 bf16 boxes, TMA-stored.
+struct RlCfg {
+    static constexpr int A_BYTES = 128 * 128;
+    static constexpr int B_BYTES = 384 * 128;
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int STAGES = 2;
+    static constexpr int RING = STAGES * STAGE;
+    static constexpr int XCH = 128 * 32 * 4;   // residual chunk: 128 rows x 32 FP32
+    static constexpr int NXB = 3;
+    static constexpr int XNB = 128 * 64 * 2;   // output box: 128 rows x 64 bf16
+    static constexpr int NXN = 2;
+    static constexpr int DATA = RING + NXB * XCH + NXN * XNB;
+    static constexpr int BAR_BYTES = (2 * STAGES + 2 + NXB) * 8 + 8;
+    static constexpr int SMEM = DATA + BAR_BYTES + 1024;
+};
+
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_rl(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXN, int K, int n_tiles,
+              EpiParams ep) {
+    using C = RlCfg;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *xbuf = smem + C::RING;
+    uint8_t *xnbuf = xbuf + C::NXB * C::XCH;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::DATA);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *accf = empty + C::STAGES;
+    uint64_t *acce = accf + 1;
+    uint64_t *xfull = acce + 1;  // [NXB]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xfull + C::NXB);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KB = K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        mbar_init(acce, 4);
+        for (int b = 0; b < C::NXB; ++b) mbar_init(&xfull[b], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmX);
+        prefetch_tmap(&tmXN);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                const int m0 = t * 128;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const uint32_t s = it % C::STAGES;
+                    if (it >= (uint32_t)C::STAGES && !mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1, ep.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = smem + s * C::STAGE;
+                    mbar_arrive_expect_tx(&full[s], C::STAGE);
+                    tma_load_2d(sa, &tmA, &full[s], kb * 64, m0);
+                    tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * 64, 0);
+                    tma_load_2d(sa + C::A_BYTES + 192 * 128, &tmB, &full[s], kb * 64, 192);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(192);
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tc) {
+                if (tc >= 1 && !mbar_wait(acce, (tc - 1) & 1, ep.status)) break;
+                tc_fence_after();
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const uint32_t s = it % C::STAGES;
+                    if (!mbar_wait(&full[s], (it / C::STAGES) & 1, ep.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smem + s * C::STAGE);
+                    const uint32_t b_base = a_base + C::A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        tc_mma_bf16(tmem, sdesc_sw128(a_base + k * 32), sdesc_sw128(b_base + k * 32), idesc,
+                                    (kb | k) != 0);
+                        tc_mma_bf16(tmem + 192, sdesc_sw128(a_base + k * 32),
+                                    sdesc_sw128(b_base + 192 * 128 + k * 32), idesc, (kb | k) != 0);
+                    }
+                    tc_commit(&empty[s]);
+                }
+                tc_commit(accf);
+            }
+        }
+    } else {
+        const int q = warp & 3;             // TMEM lane quarter
+        const int r = q * 32 + lane;        // row inside the tile
+        const bool leader = threadIdx.x == 64;
+        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+        const int first = blockIdx.x;
+        // residual chunk loads: chunk index g = (local tile) * 12 + c into buffer g % 3
+        if (leader && first < n_tiles) {
+            for (int c = 0; c < C::NXB; ++c) {
+                mbar_arrive_expect_tx(&xfull[c], C::XCH);
+                tma_load_2d(xbuf + c * C::XCH, &tmX, &xfull[c], c * 32, first * 128);
+            }
+        }
+        // every epilogue thread runs the same sequence of named barriers: a wait
+        // that gives up does not leave the loop (later waits then return at once)
+        uint32_t tc = 0;
+        for (int t = first; t < n_tiles; t += gridDim.x, ++tc) {
+            const int m0 = t * 128;
+            const int tnext = t + gridDim.x;
+            mbar_wait(accf, tc & 1, ep.status);
+            __syncwarp();
+            tc_fence_after();
+            float cnt = 0.f, mean = 0.f, m2 = 0.f;
+            // ---- pass 1
+#pragma unroll 1
+            for (int c = 0; c < 12; ++c) {
+                const uint32_t g = tc * 12 + c, b = g % C::NXB;
+                uint32_t a[32];
+                tmem_ld32(tl + c * 32, a);
+                mbar_wait(&xfull[b], (g / C::NXB) & 1, ep.status);
+                tmem_ld_wait();
+                uint8_t *xb = xbuf + b * C::XCH;
+                float v[32];
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(xb + r * 128 + ((j4 ^ (r & 7)) << 4));
+                    float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (ep.bias) bb = reinterpret_cast<const float4 *>(ep.bias + c * 32)[j4];
+                    v[4 * j4 + 0] = x.x + __uint_as_float(a[4 * j4 + 0]) + bb.x;
+                    v[4 * j4 + 1] = x.y + __uint_as_float(a[4 * j4 + 1]) + bb.y;
+                    v[4 * j4 + 2] = x.z + __uint_as_float(a[4 * j4 + 2]) + bb.z;
+                    v[4 * j4 + 3] = x.w + __uint_as_float(a[4 * j4 + 3]) + bb.w;
+                }
+                float s = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) s += v[j];
+                const float cm = s * (1.0f / 32.f);
+                float cq = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) cq += (v[j] - cm) * (v[j] - cm);
+                if (c == 0) {
+                    mean = cm;
+                    m2 = cq;
+                    cnt = 32.f;
+                } else {
+                    const float tot = cnt + 32.f, dl = cm - mean;
+                    mean += dl * (32.f / tot);
+                    m2 += cq + dl * dl * (cnt * 32.f / tot);
+                    cnt = tot;
+                }
+                uint32_t w[32];
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    *reinterpret_cast<float4 *>(xb + r * 128 + ((j4 ^ (r & 7)) << 4)) =
+                        make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
+                tmem_st32(tl + c * 32, w);
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (leader) {
+                    tma_store_2d(&tmX, xb, c * 32, m0);
+                    bulk_commit();
+                    // refill this buffer with the chunk three ahead (this tile, else the next one)
+                    const int cn = c + C::NXB;
+                    const int tt = cn < 12 ? t : tnext;
+                    if (tt < n_tiles) {
+                        bulk_wait_read<0>();
+                        mbar_arrive_expect_tx(&xfull[b], C::XCH);
+                        tma_load_2d(xb, &tmX, &xfull[b], (cn % 12) * 32, tt * 128);
+                    }
+                }
+            }
+            tmem_st_wait();
+            const float rstd = 1.0f / sqrtf(m2 * (1.0f / D) + ep.eps);
+            // ---- pass 2
+#pragma unroll 1
+            for (int j = 0; j < 6; ++j) {
+                const uint32_t g2 = tc * 6 + j;
+                uint8_t *ob = xnbuf + (g2 & 1) * C::XNB;
+                if (g2 >= 2) {
+                    if (leader) bulk_wait_read<0>();
+                    named_bar_sync(1, 128);
+                }
+                uint32_t a[32], b2[32];
+                tmem_ld32(tl + j * 64, a);
+                tmem_ld32(tl + j * 64 + 32, b2);
+                tmem_ld_wait();
+                uint32_t w[32];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const int col = j * 64 + h * 32 + j4 * 4;
+                        const float4 gg = *reinterpret_cast<const float4 *>(ep.ln_g + col);
+                        float4 be = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (ep.ln_b) be = *reinterpret_cast<const float4 *>(ep.ln_b + col);
+                        const uint32_t *src = h ? b2 : a;
+                        const float y0 = (__uint_as_float(src[4 * j4 + 0]) - mean) * rstd * gg.x + be.x;
+                        const float y1 = (__uint_as_float(src[4 * j4 + 1]) - mean) * rstd * gg.y + be.y;
+                        const float y2 = (__uint_as_float(src[4 * j4 + 2]) - mean) * rstd * gg.z + be.z;
+                        const float y3 = (__uint_as_float(src[4 * j4 + 3]) - mean) * rstd * gg.w + be.w;
+                        w[h * 16 + 2 * j4] = pack_bf16x2(y0, y1);
+                        w[h * 16 + 2 * j4 + 1] = pack_bf16x2(y2, y3);
+                    }
+                }
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc)
+                    *reinterpret_cast<uint4 *>(ob + r * 128 + ((cc ^ (r & 7)) << 4)) =
+                        make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (leader) {
+                    tma_store_2d(&tmXN, ob, j * 64, m0);
+                    bulk_commit();
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce);
+        }
+        if (leader) bulk_wait_all();
+        __syncwarp();
     }
     __syncthreads();
     if (warp == 1) {
@@ -487,6 +795,8 @@ cudaError_t gemm_init_attributes() {
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(k_gemm_rl, cudaFuncAttributeMaxDynamicSharedMemorySize, RlCfg::SMEM)) != cudaSuccess)
+        return e;
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<192>::SMEM)) != cudaSuccess)
         return e;
@@ -524,13 +834,23 @@ static cudaError_t launch_pc(const GemmOp &op, cudaStream_t st) {
     const int nblk = op.N / BN;
     const int n_tiles = nblk * ((op.ep.rows + 127) / 128);
     const int grid = n_tiles < g_num_sms ? n_tiles : g_num_sms;
-    k_gemm_pc<EPI, BN><<<grid, 192, PcCfg<BN>::SMEM, st>>>(*op.tmA, *op.tmB, op.K, n_tiles, nblk, op.ep);
+    if (!op.tmO) return cudaErrorInvalidValue;
+    k_gemm_pc<EPI, BN><<<grid, 192, PcCfg<BN>::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmO, op.K, n_tiles, nblk, op.ep);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st) {
     if (op.ep.rows <= 0) return cudaSuccess;
     if (op.N % op.bn != 0 || op.K % 64 != 0) return cudaErrorInvalidValue;
+    // the streaming residual kernel keeps a 2-stage operand ring; for K > 384 the
+    // 3-stage single-tile kernel (weights streamed per tile) measured faster
+    if (!fp32 && op.epi == EPI_RESID_LN && op.tmX && op.tmXN && op.ep.ln_g && !op.ep.fin_g && op.N == D &&
+        op.K <= 384) {
+        const int n_tiles = (op.ep.rows + 127) / 128;
+        const int grid = n_tiles < g_num_sms ? n_tiles : g_num_sms;
+        k_gemm_rl<<<grid, 192, RlCfg::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmX, *op.tmXN, op.K, n_tiles, op.ep);
+        return cudaGetLastError();
+    }
     if (!fp32) {  // persistent tcgen05 kernels for the column-split epilogues
         if (op.epi == EPI_QKV) return launch_pc<EPI_QKV, 192>(op, st);
         if (op.epi == EPI_GEGLU) return launch_pc<EPI_GEGLU, 256>(op, st);

@@ -20,6 +20,9 @@ struct GemmOp {
     int K, N;
     const CUtensorMap *tmA;   // BF16 path: A box 64 x 128
     const CUtensorMap *tmB;   // BF16 path: W box 64 x (bn == 384 ? 192 : 256)
+    const CUtensorMap *tmO;   // BF16 column-split epilogues: output, box 64 x 32, 128-byte swizzle
+    const CUtensorMap *tmX;   // BF16 residual epilogue: FP32 residual, box 32 x 128, 128-byte swizzle
+    const CUtensorMap *tmXN;  // BF16 residual epilogue: LayerNorm output, box 64 x 128, 128-byte swizzle
     const float *A32;         // FP32 path: A [rows, lda]
     int lda;
     const float *W32;         // FP32 path: W [N, K]

@@ -131,16 +131,16 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 map over [rows, cols] with row stride ld (elements); box = box_cols x box_rows, 128-byte swizzle.
+// 2-D map over [rows, cols] with row stride ld (elements); box = box_cols x box_rows, 128-byte swizzle.
 jd_status make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_cols,
-                   uint32_t box_rows) {
+                   uint32_t box_rows, bool fp32 = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(JD_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {ld * 2};
+    cuuint64_t strides[1] = {ld * (fp32 ? 4 : 2)};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t es[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+    CUresult r = fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(JD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -182,6 +182,9 @@ struct jd_model {
     void *xm = nullptr, *qm = nullptr, *om = nullptr, *xnm = nullptr, *ym = nullptr;
     unsigned *status = nullptr;
     CUtensorMap tm_xn{}, tm_o{}, tm_y_enc{}, tm_y_head{}, tm_qkv{}, tm_xm{}, tm_om{}, tm_xnm{}, tm_ym{};
+    // output maps of the column-split epilogues (box 64 x 32)
+    CUtensorMap to_qkv{}, to_y_enc{}, to_y_head{}, to_qm{}, to_ym{};
+    CUtensorMap tm_x32{};  // FP32 residual stream, box 32 x 128
 
     // internal outputs (jd_forward, host entry points) and device batch staging
     float *i_logits = nullptr, *i_probs = nullptr, *i_score = nullptr, *i_noul = nullptr, *i_maxp = nullptr;
@@ -406,6 +409,12 @@ jd_status alloc_workspace(jd_model *m) {
         TRY(make_map(&m->tm_om, m->om, D, M, D, 64, 128));
         TRY(make_map(&m->tm_xnm, m->xnm, D, M, D, 64, 128));
         TRY(make_map(&m->tm_ym, m->ym, HFF, M, HFF, 64, 128));
+        TRY(make_map(&m->to_qkv, m->qkv, QKV, T, QKV, 64, 32));
+        TRY(make_map(&m->tm_x32, m->x, D, T, D, 32, 128, true));
+        TRY(make_map(&m->to_y_enc, m->y, FF, T, FF, 64, 32));
+        TRY(make_map(&m->to_y_head, m->y, HFF, T, HFF, 64, 32));
+        TRY(make_map(&m->to_qm, m->qm, D, M, D, 64, 32));
+        TRY(make_map(&m->to_ym, m->ym, HFF, M, HFF, 64, 32));
     }
     return JD_OK;
 }
@@ -420,8 +429,12 @@ EpiParams base_ep(jd_model *m, int rows) {
     return e;
 }
 
-GemmOp make_op(int epi, int bn, const ProjW &w, const CUtensorMap *tmA, const void *A, int lda, const EpiParams &ep) {
+GemmOp make_op(int epi, int bn, const ProjW &w, const CUtensorMap *tmA, const void *A, int lda, const EpiParams &ep,
+               const CUtensorMap *tmO = nullptr, const CUtensorMap *tmX = nullptr, const CUtensorMap *tmXN = nullptr) {
     GemmOp op;
+    op.tmO = tmO;
+    op.tmX = tmX;
+    op.tmXN = tmXN;
     op.epi = epi;
     op.bn = bn;
     op.K = w.K;
@@ -486,7 +499,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.rope = glob ? m->rope_g : m->rope_l;
         e.pos = m->pos;
         e.rope_cols = 2 * D;
-        KL("gemm_qkv_rope", 1, launch_gemm(make_op(EPI_QKV, 384, m->Wqkv[l], &m->tm_xn, m->xn, D, e), f32, st));
+        KL("gemm_qkv_rope", 1, launch_gemm(make_op(EPI_QKV, 384, m->Wqkv[l], &m->tm_xn, m->xn, D, e, &m->to_qkv), f32, st));
 
         aa.window = glob ? -1 : 64;
         KL(glob ? "attn_global" : "attn_local", 1, launch_attention(aa, f32, st));
@@ -496,12 +509,12 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.ldo = D;
         e.resid = m->x;
         e.ln_g = m->mlp_g[l];
-        KL("gemm_wo_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo[l], &m->tm_o, m->o, D, e), f32, st));
+        KL("gemm_wo_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo[l], &m->tm_o, m->o, D, e, nullptr, &m->tm_x32, &m->tm_xn), f32, st));
 
         e = base_ep(m, T);
         e.out = m->y;
         e.ldo = FF;
-        KL("gemm_wi_geglu", 1, launch_gemm(make_op(EPI_GEGLU, 256, m->Wi[l], &m->tm_xn, m->xn, D, e), f32, st));
+        KL("gemm_wi_geglu", 1, launch_gemm(make_op(EPI_GEGLU, 256, m->Wi[l], &m->tm_xn, m->xn, D, e, &m->to_y_enc), f32, st));
 
         e = base_ep(m, T);
         e.out = m->xn;
@@ -518,7 +531,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
             e.ln_g = m->n1g[0];
             e.ln_b = m->n1b[0];
         }
-        KL("gemm_wo2_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo2[l], &m->tm_y_enc, m->y, FF, e), f32, st));
+        KL("gemm_wo2_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo2[l], &m->tm_y_enc, m->y, FF, e, nullptr, &m->tm_x32, &m->tm_xn), f32, st));
     }
 
     // ---- head layer 0 (all tokens)
@@ -527,7 +540,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.out = m->qkv;
         e.ldo = QKV;
         e.bias = m->in_b[0];
-        KL("head0_gemm_in", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_full[0], &m->tm_xn, m->xn, D, e), f32, st));
+        KL("head0_gemm_in", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_full[0], &m->tm_xn, m->xn, D, e, &m->to_qkv), f32, st));
         aa.window = -1;
         KL("head0_attn", 1, launch_attention(aa, f32, st));
         e = base_ep(m, T);
@@ -537,12 +550,12 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.resid = m->x;
         e.ln_g = m->n2g[0];
         e.ln_b = m->n2b[0];
-        KL("head0_gemm_out", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->out_p[0], &m->tm_o, m->o, D, e), f32, st));
+        KL("head0_gemm_out", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->out_p[0], &m->tm_o, m->o, D, e, nullptr, &m->tm_x32, &m->tm_xn), f32, st));
         e = base_ep(m, T);
         e.out = m->y;
         e.ldo = HFF;
         e.bias = m->l1_b[0];
-        KL("head0_gemm_ffn1", 1, launch_gemm(make_op(EPI_BIAS_ACT, 256, m->lin1[0], &m->tm_xn, m->xn, D, e), f32, st));
+        KL("head0_gemm_ffn1", 1, launch_gemm(make_op(EPI_BIAS_ACT, 256, m->lin1[0], &m->tm_xn, m->xn, D, e, &m->to_y_head), f32, st));
         e = base_ep(m, T);
         e.out = m->xn;
         e.ldo = D;
@@ -550,7 +563,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.resid = m->x;
         e.ln_g = m->n1g[1];
         e.ln_b = m->n1b[1];
-        KL("head0_gemm_ffn2", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[0], &m->tm_y_head, m->y, HFF, e), f32, st));
+        KL("head0_gemm_ffn2", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[0], &m->tm_y_head, m->y, HFF, e, nullptr, &m->tm_x32, &m->tm_xn), f32, st));
     }
     // ---- head layer 1: keys / values for every token, the rest at the markers only
     {
@@ -558,13 +571,14 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.out = offset<uint8_t>(m->qkv, D, f32);
         e.ldo = QKV;
         e.bias = m->in_b[1] + D;
-        KL("head1_gemm_kv", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_kv[1], &m->tm_xn, m->xn, D, e), f32, st));
+        e.out_col0 = D;  // keys / values land in columns 384..1151 of qkv
+        KL("head1_gemm_kv", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_kv[1], &m->tm_xn, m->xn, D, e, &m->to_qkv), f32, st));
         KL("head1_gather", 1, launch_gather_markers(b->mask_pos, M, T, m->x, m->xn, m->hm, m->xm, f32, m->status, st));
         e = base_ep(m, M);
         e.out = m->qm;
         e.ldo = D;
         e.bias = m->in_b[1];
-        KL("head1_gemm_q", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_q[1], &m->tm_xm, m->xm, D, e), f32, st));
+        KL("head1_gemm_q", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_q[1], &m->tm_xm, m->xm, D, e, &m->to_qm), f32, st));
         KL("head1_marker_attn", 1, launch_marker_attention(m->qm, m->qkv, m->om, b->cu_seqlens, b->opt_off, b->mask_pos, B, f32, st));
         e = base_ep(m, M);
         e.out = m->xnm;
@@ -578,7 +592,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.out = m->ym;
         e.ldo = HFF;
         e.bias = m->l1_b[1];
-        KL("head1_gemm_ffn1", 1, launch_gemm(make_op(EPI_BIAS_ACT, 256, m->lin1[1], &m->tm_xnm, m->xnm, D, e), f32, st));
+        KL("head1_gemm_ffn1", 1, launch_gemm(make_op(EPI_BIAS_ACT, 256, m->lin1[1], &m->tm_xnm, m->xnm, D, e, &m->to_ym), f32, st));
         e = base_ep(m, M);
         e.bias = m->l2_b[1];
         e.resid = m->hm;
@@ -910,6 +924,8 @@ struct NoAllocSlot {
     bool ready = false;
     uint8_t *base = nullptr;  // device address of g_noalloc_scratch on this device
     CUtensorMap tm_xn{}, tm_o{}, tm_y_enc{}, tm_y_head{}, tm_qkv{}, tm_xm{}, tm_om{}, tm_xnm{}, tm_ym{};
+    CUtensorMap to_qkv{}, to_y_enc{}, to_y_head{}, to_qm{}, to_ym{};
+    CUtensorMap tm_x32{};  // FP32 residual stream, box 32 x 128
 };
 NoAllocSlot g_na_slot[NA_MAX_DEVICES];
 std::mutex g_na_mutex;
@@ -934,6 +950,12 @@ jd_status noalloc_setup(int dev) {
     TRY(make_map(&s.tm_om, s.base + NA_OM, D, NA_MARKERS, D, 64, 128));
     TRY(make_map(&s.tm_xnm, s.base + NA_XNM, D, NA_MARKERS, D, 64, 128));
     TRY(make_map(&s.tm_ym, s.base + NA_YM, HFF, NA_MARKERS, HFF, 64, 128));
+    TRY(make_map(&s.to_qkv, s.base + NA_QKV, QKV, NA_TOKENS, QKV, 64, 32));
+    TRY(make_map(&s.tm_x32, s.base + NA_X, D, NA_TOKENS, D, 32, 128, true));
+    TRY(make_map(&s.to_y_enc, s.base + NA_Y, FF, NA_TOKENS, FF, 64, 32));
+    TRY(make_map(&s.to_y_head, s.base + NA_Y, HFF, NA_TOKENS, HFF, 64, 32));
+    TRY(make_map(&s.to_qm, s.base + NA_QM, D, NA_MARKERS, D, 64, 32));
+    TRY(make_map(&s.to_ym, s.base + NA_YM, HFF, NA_MARKERS, HFF, 64, 32));
     s.ready = true;
     return JD_OK;
 }
@@ -968,6 +990,8 @@ void noalloc_view(jd_model &v, const jd_model *m, const NoAllocSlot &s) {
     v.status = reinterpret_cast<unsigned *>(b + NA_STATUS);
     v.tm_xn = s.tm_xn; v.tm_o = s.tm_o; v.tm_y_enc = s.tm_y_enc; v.tm_y_head = s.tm_y_head; v.tm_qkv = s.tm_qkv;
     v.tm_xm = s.tm_xm; v.tm_om = s.tm_om; v.tm_xnm = s.tm_xnm; v.tm_ym = s.tm_ym;
+    v.to_qkv = s.to_qkv; v.to_y_enc = s.to_y_enc; v.to_y_head = s.to_y_head; v.to_qm = s.to_qm; v.to_ym = s.to_ym;
+    v.tm_x32 = s.tm_x32;
     v.prof = false;
     v.graph_mode = false;
 }

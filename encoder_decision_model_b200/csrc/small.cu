@@ -235,10 +235,12 @@ __global__ void __launch_bounds__(256) k_scorer(ScorerArgs a) {
 }
 
 cudaError_t gemm_init_attributes();
+cudaError_t attn_init_attributes();
 
 cudaError_t init_kernel_attributes() {
     cudaError_t e = cudaFuncSetAttribute(k_scorer, cudaFuncAttributeMaxDynamicSharedMemorySize, SC_M * D * 4);
     if (e != cudaSuccess) return e;
+    if ((e = attn_init_attributes()) != cudaSuccess) return e;
     return gemm_init_attributes();
 }
 
