@@ -136,6 +136,45 @@ def recorded_traffic(kernel, workload_tag):
     return None
 
 
+# ----------------------------------------------------------------------------- ranks
+
+
+class Ranks:
+    """The timing protocol's process-group steps: barrier, max and sum over
+    ranks (NCCL on the GPU machine, gloo in the CPU tests; single process: no-ops)."""
+
+    def __init__(self, world, device):
+        self.world = world
+        self.device = device
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def _reduce(self, x, op):
+        if self.world == 1:
+            return float(x)
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=op)
+        return float(t.item())
+
+    def max(self, x):
+        import torch.distributed as dist
+        return self._reduce(x, dist.ReduceOp.MAX)
+
+    def sum(self, x):
+        import torch.distributed as dist
+        return self._reduce(x, dist.ReduceOp.SUM)
+
+
+def whole_job_rate(units_this_rank, seconds_this_rank, ranks):
+    """Units processed by all ranks / the slowest rank's time."""
+    return ranks.sum(units_this_rank) / ranks.max(seconds_this_rank)
+
+
 # ----------------------------------------------------------------------------- clocks
 
 
@@ -265,23 +304,8 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def sum_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
+    ranks = Ranks(world, dev)
+    barrier, max_over_ranks, sum_over_ranks = ranks.barrier, ranks.max, ranks.sum
 
     from encoder_decision_model_b200.build import build
     if rank == 0:

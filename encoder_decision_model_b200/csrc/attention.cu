@@ -437,8 +437,13 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+cudaError_t attn_tc_init_attributes();
+
 cudaError_t attn_init_attributes() {
-    return cudaFuncSetAttribute(k_attn_local_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, 7 * 8192 + 64 + 1024);
+    cudaError_t e = cudaFuncSetAttribute(k_attn_local_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         7 * 8192 + 64 + 1024);
+    if (e != cudaSuccess) return e;
+    return attn_tc_init_attributes();
 }
 
 cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st) {
@@ -453,6 +458,8 @@ cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st) {
         else
             k_attn_f32<false><<<grid, 256, 0, st>>>((const float *)a.qkv, (float *)a.o, a.cu_seqlens, a.qb_off,
                                                     a.n_rows, a.window);
+    } else if (!local && a.tm_qkv128) {
+        return launch_attention_tc(a, a.tm_qkv128, num_sms(), st);
     } else {
         const int smem = 5 * 8192 + 64 + 1024;
         if (local && a.window == 64)

@@ -789,6 +789,7 @@ static cudaError_t set_attrs() {
 }
 
 static int g_num_sms = 148;
+int num_sms() { return g_num_sms; }
 
 cudaError_t gemm_init_attributes() {
     cudaError_t e;

@@ -30,7 +30,8 @@ struct GemmOp {
 };
 cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st);
 
-// Per-token row index / position and per-row attention tile offsets.
+// Per-token row index / position and per-row attention work-unit offsets
+// (qb_off holds 2 * (n_rows + 1) ints: 64-query then 128-query block offsets).
 cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
                         cudaStream_t st);
 
@@ -49,9 +50,12 @@ struct AttnArgs {
     int n_rows, n_tokens;
     int window;
     const CUtensorMap *tm_qkv; // BF16 path: box 64 x 64 over [T_cap, 1152]
+    const CUtensorMap *tm_qkv128; // BF16 global layers on tcgen05: box 64 x 128 (null: mma.sync kernel)
     unsigned *status;
 };
 cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st);
+cudaError_t launch_attention_tc(const AttnArgs &a, const CUtensorMap *tm128, int num_sms, cudaStream_t st);
+int num_sms();
 
 // Gather the marker rows: hm[m] = h[mask_pos[m]] (FP32), xm[m] = xn[mask_pos[m]].
 cudaError_t launch_gather_markers(const int *mask_pos, int n_markers, int n_tokens, const float *h, const void *xn,

@@ -185,6 +185,7 @@ struct jd_model {
     // output maps of the column-split epilogues (box 64 x 32)
     CUtensorMap to_qkv{}, to_y_enc{}, to_y_head{}, to_qm{}, to_ym{};
     CUtensorMap tm_x32{};  // FP32 residual stream, box 32 x 128
+    CUtensorMap tm_qkv128{};  // q|k|v, box 64 x 128 (tensor-core attention)
 
     // internal outputs (jd_forward, host entry points) and device batch staging
     float *i_logits = nullptr, *i_probs = nullptr, *i_score = nullptr, *i_noul = nullptr, *i_maxp = nullptr;
@@ -369,7 +370,7 @@ jd_status alloc_workspace(jd_model *m) {
     TRY(m->dalloc(&p, T * HFF * es)); m->y = p;
     TRY(m->dalloc(&m->tok_row, T));
     TRY(m->dalloc(&m->pos, T));
-    TRY(m->dalloc(&m->qb_off, B + 1));
+    TRY(m->dalloc(&m->qb_off, 2 * (B + 1)));
     TRY(m->dalloc(&m->hm, M * D));
     TRY(m->dalloc(&p, M * D * es)); m->xm = p;
     TRY(m->dalloc(&p, M * D * es)); m->qm = p;
@@ -411,6 +412,7 @@ jd_status alloc_workspace(jd_model *m) {
         TRY(make_map(&m->tm_ym, m->ym, HFF, M, HFF, 64, 128));
         TRY(make_map(&m->to_qkv, m->qkv, QKV, T, QKV, 64, 32));
         TRY(make_map(&m->tm_x32, m->x, D, T, D, 32, 128, true));
+        TRY(make_map(&m->tm_qkv128, m->qkv, QKV, T, QKV, 64, 128));
         TRY(make_map(&m->to_y_enc, m->y, FF, T, FF, 64, 32));
         TRY(make_map(&m->to_y_head, m->y, HFF, T, HFF, 64, 32));
         TRY(make_map(&m->to_qm, m->qm, D, M, D, 64, 32));
@@ -489,6 +491,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
     aa.n_rows = B;
     aa.n_tokens = T;
     aa.tm_qkv = &m->tm_qkv;
+    aa.tm_qkv128 = &m->tm_qkv128;
     aa.status = m->status;
 
     for (int l = 0; l < NL; ++l) {
@@ -903,7 +906,7 @@ constexpr size_t NA_Y = NA_O + na_up((size_t)NA_TOKENS * D * 2);
 constexpr size_t NA_TOKROW = NA_Y + na_up((size_t)NA_TOKENS * HFF * 2);
 constexpr size_t NA_POS = NA_TOKROW + na_up((size_t)NA_TOKENS * 4);
 constexpr size_t NA_QBOFF = NA_POS + na_up((size_t)NA_TOKENS * 4);
-constexpr size_t NA_HM = NA_QBOFF + na_up((size_t)(NA_ROWS + 1) * 4);
+constexpr size_t NA_HM = NA_QBOFF + na_up((size_t)2 * (NA_ROWS + 1) * 4);
 constexpr size_t NA_XM = NA_HM + na_up((size_t)NA_MARKERS * D * 4);
 constexpr size_t NA_QM = NA_XM + na_up((size_t)NA_MARKERS * D * 2);
 constexpr size_t NA_OM = NA_QM + na_up((size_t)NA_MARKERS * D * 2);
@@ -926,6 +929,7 @@ struct NoAllocSlot {
     CUtensorMap tm_xn{}, tm_o{}, tm_y_enc{}, tm_y_head{}, tm_qkv{}, tm_xm{}, tm_om{}, tm_xnm{}, tm_ym{};
     CUtensorMap to_qkv{}, to_y_enc{}, to_y_head{}, to_qm{}, to_ym{};
     CUtensorMap tm_x32{};  // FP32 residual stream, box 32 x 128
+    CUtensorMap tm_qkv128{};
 };
 NoAllocSlot g_na_slot[NA_MAX_DEVICES];
 std::mutex g_na_mutex;
@@ -952,6 +956,7 @@ jd_status noalloc_setup(int dev) {
     TRY(make_map(&s.tm_ym, s.base + NA_YM, HFF, NA_MARKERS, HFF, 64, 128));
     TRY(make_map(&s.to_qkv, s.base + NA_QKV, QKV, NA_TOKENS, QKV, 64, 32));
     TRY(make_map(&s.tm_x32, s.base + NA_X, D, NA_TOKENS, D, 32, 128, true));
+    TRY(make_map(&s.tm_qkv128, s.base + NA_QKV, QKV, NA_TOKENS, QKV, 64, 128));
     TRY(make_map(&s.to_y_enc, s.base + NA_Y, FF, NA_TOKENS, FF, 64, 32));
     TRY(make_map(&s.to_y_head, s.base + NA_Y, HFF, NA_TOKENS, HFF, 64, 32));
     TRY(make_map(&s.to_qm, s.base + NA_QM, D, NA_MARKERS, D, 64, 32));
@@ -992,6 +997,7 @@ void noalloc_view(jd_model &v, const jd_model *m, const NoAllocSlot &s) {
     v.tm_xm = s.tm_xm; v.tm_om = s.tm_om; v.tm_xnm = s.tm_xnm; v.tm_ym = s.tm_ym;
     v.to_qkv = s.to_qkv; v.to_y_enc = s.to_y_enc; v.to_y_head = s.to_y_head; v.to_qm = s.to_qm; v.to_ym = s.to_ym;
     v.tm_x32 = s.tm_x32;
+    v.tm_qkv128 = s.tm_qkv128;
     v.prof = false;
     v.graph_mode = false;
 }

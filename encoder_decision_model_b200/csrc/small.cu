@@ -19,28 +19,44 @@ __global__ void k_token_meta(const int *__restrict__ cu, int n_rows, int *__rest
     }
 }
 
-// qb_off[r] = sum over rows < r of ceil(len / 64); one CTA of 1024 threads.
+// Attention work-unit offsets, one CTA of 1024 threads:
+//   qb_off[r]             = sum over rows < r of ceil(len / 64)   (64-query blocks)
+//   qb_off[n_rows + 1 + r] = sum over rows < r of ceil(len / 128)  (128-query blocks)
 __global__ void __launch_bounds__(1024) k_qblock_offsets(const int *__restrict__ cu, int n_rows, int *__restrict__ qb_off) {
-    __shared__ int part[1024];
+    __shared__ int part[2][1024];
     const int tid = threadIdx.x;
     const int per = (n_rows + 1023) / 1024;
     const int r0 = tid * per, r1 = min(n_rows, r0 + per);
-    int s = 0;
-    for (int r = r0; r < r1; ++r) s += (cu[r + 1] - cu[r] + 63) / 64;
-    part[tid] = s;
-    __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {  // inclusive scan
-        const int v = tid >= off ? part[tid - off] : 0;
-        __syncthreads();
-        part[tid] += v;
-        __syncthreads();
-    }
-    int run = tid ? part[tid - 1] : 0;
+    int s64 = 0, s128 = 0;
     for (int r = r0; r < r1; ++r) {
-        qb_off[r] = run;
-        run += (cu[r + 1] - cu[r] + 63) / 64;
+        const int len = cu[r + 1] - cu[r];
+        s64 += (len + 63) / 64;
+        s128 += (len + 127) / 128;
     }
-    if (tid == 1023) qb_off[n_rows] = part[1023];
+    part[0][tid] = s64;
+    part[1][tid] = s128;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {  // inclusive scans
+        const int v0 = tid >= off ? part[0][tid - off] : 0;
+        const int v1 = tid >= off ? part[1][tid - off] : 0;
+        __syncthreads();
+        part[0][tid] += v0;
+        part[1][tid] += v1;
+        __syncthreads();
+    }
+    int run64 = tid ? part[0][tid - 1] : 0, run128 = tid ? part[1][tid - 1] : 0;
+    int *q128 = qb_off + n_rows + 1;
+    for (int r = r0; r < r1; ++r) {
+        const int len = cu[r + 1] - cu[r];
+        qb_off[r] = run64;
+        q128[r] = run128;
+        run64 += (len + 63) / 64;
+        run128 += (len + 127) / 128;
+    }
+    if (tid == 1023) {
+        qb_off[n_rows] = part[0][1023];
+        q128[n_rows] = part[1][1023];
+    }
 }
 
 cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
