@@ -372,6 +372,7 @@ __global__ void __launch_bounds__(128)
     }
 }
 
+
 // ------------------------------------------------------------------ FP32 validation attention
 
 template <bool LOCAL>
@@ -458,7 +459,9 @@ cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st) {
         else
             k_attn_f32<false><<<grid, 256, 0, st>>>((const float *)a.qkv, (float *)a.o, a.cu_seqlens, a.qb_off,
                                                     a.n_rows, a.window);
-    } else if (!local && a.tm_qkv128) {
+    } else if (a.tm_qkv128 && !local) {
+        // tcgen05 for global layers; the +-64 band stays on the mma.sync kernel below,
+        // which measured faster than the band variant of the tcgen05 kernel (2 tiles per item)
         return launch_attention_tc(a, a.tm_qkv128, num_sms(), st);
     } else {
         const int smem = 5 * 8192 + 64 + 1024;

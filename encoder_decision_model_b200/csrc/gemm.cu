@@ -171,8 +171,9 @@ __global__ void __launch_bounds__(256, 1)
 // warp fills the other buffer with tile i + 1.
 //   warp 0 lane 0  TMA producer (A 128 x 64, W BN x 64 per stage)
 //   warp 1         TMEM allocation; lane 0 issues tcgen05.mma
-//   warps 2..5     epilogue, one accumulator row per thread (TMEM lane
-//                  quarter = warp % 4); QKV and bias+activation outputs are
+//   warps 2..      epilogue, one accumulator row per thread (TMEM lane
+//                  quarter = warp % 4; GEGLU runs two warps per quarter, each
+//                  on half of the output columns); QKV and bias+activation outputs are
 //                  staged per warp as 32 rows x 64 columns (bf16, 128-byte
 //                  swizzle) in shared memory and written by one TMA bulk
 //                  store each (double-buffered); GEGLU outputs go straight
@@ -222,18 +223,20 @@ __device__ __forceinline__ void stage_row32(uint8_t *box, int r, int c0, const u
             make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
 }
 
-template <int EPI, int BN>
+template <int EPI, int BN, int NPART>
 __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0, int n0, const EpiParams &ep,
                                                  const CUtensorMap *tmO, OutStage &os, int lane,
-                                                 const float2 (&cs)[32], bool have_cs) {
+                                                 const float2 (&cs)[32], bool have_cs, int part) {
     if constexpr (EPI == EPI_GEGLU) {
         // stored straight from registers: a shared-memory staging pass here
-        // competes with the 256-wide MMAs for shared-memory bandwidth
+        // competes with the 256-wide MMAs for shared-memory bandwidth; with
+        // NPART warps per TMEM lane quarter each takes G / NPART output columns
         constexpr int G = BN / 2;
+        constexpr int GP = G / NPART;
         const int row = row0 + r;
         __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(ep.out) + (size_t)row * ep.ldo + n0 / 2;
 #pragma unroll 1
-        for (int c = 0; c < G; c += 32) {
+        for (int c = part * GP; c < (part + 1) * GP; c += 32) {
             uint32_t u[32], g[32];
             tmem_ld32(tacc + c, u);
             tmem_ld32(tacc + G + c, g);
@@ -324,8 +327,8 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
     }
 }
 
-template <int EPI, int BN>
-__global__ void __launch_bounds__(192, 1)
+template <int EPI, int BN, int EW>
+__global__ void __launch_bounds__(64 + 32 * EW, 1)
     k_gemm_pc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmO, int K, int n_tiles, int nblk, EpiParams ep) {
     using C = PcCfg<BN>;
@@ -348,8 +351,8 @@ __global__ void __launch_bounds__(192, 1)
         }
         mbar_init(&accf[0], 1);
         mbar_init(&accf[1], 1);
-        mbar_init(&acce[0], 4);
-        mbar_init(&acce[1], 4);
+        mbar_init(&acce[0], EW);
+        mbar_init(&acce[1], EW);
         fence_barrier_init();
         fence_proxy_async_smem();
         prefetch_tmap(&tmA);
@@ -410,8 +413,9 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
     } else {
-        const int q = warp & 3;  // TMEM lane quarter of this warp
-        OutStage os{smem + C::RING + (warp - 2) * 2 * C::OUT_BOX, 0u};
+        const int q = warp & 3;           // TMEM lane quarter of this warp
+        const int part = (warp - 2) >> 2;  // which share of the tile's columns (EW / 4 shares)
+        OutStage os{smem + C::RING + ((warp - 2) & 3) * 2 * C::OUT_BOX, 0u};
         uint32_t tc = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tc) {
             const int m0 = (t / nblk) * 128, n0 = (t % nblk) * BN;
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
             tc_fence_after();
             const uint32_t tacc = tmem + buf * C::BUF_COLS + ((uint32_t)(q * 32) << 16);
-            pc_epilogue_rows<EPI, BN>(tacc, lane, row0, n0, ep, &tmO, os, lane, cs, have_cs);
+            pc_epilogue_rows<EPI, BN, EW / 4>(tacc, lane, row0, n0, ep, &tmO, os, lane, cs, have_cs, part);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acce[buf]);
@@ -457,26 +461,25 @@ __global__ void __launch_bounds__(192, 1)
 // looping over 128-row tiles; the 384 accumulator columns stay in one TMEM
 // buffer, so the overlap comes from the producer running ahead (the next
 // tile's A / W stages load while this tile's epilogue streams the residual).
-//   warp 0 lane 0  TMA producer: A box 128 x 64, W as two 192 x 64 boxes
+//   warp 0 lane 0  TMA producer: A box 128 x 64, W as two 192 x 64 boxes (3 stages)
 //   warp 1         TMEM allocation; lane 0 issues the N = 2 x 192 MMAs
 //   warps 2..5     epilogue, one row per thread:
 //     pass 1  per 32-column chunk: the residual chunk (128 x 32 FP32, 128-byte
-//             swizzle) arrives by TMA (three buffers, prefetched across
+//             swizzle) arrives by TMA (two buffers, prefetched across
 //             tiles); v = x + acc (+ bias) is written back in place, stored to
 //             x by TMA and parked in TMEM; row mean and M2 are merged chunk by
 //             chunk (Chan's pairwise update), so one pass yields the moments;
-//     pass 2  xn = LN(v) from TMEM into 128 x 64 bf16 boxes, TMA-stored.
+//     pass 2  xn = LN(v) from TMEM, stored from registers (the shared memory
+//             goes to a three-stage operand ring instead of output staging).
 struct RlCfg {
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = 384 * 128;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int STAGES = 2;
+    static constexpr int STAGES = 3;
     static constexpr int RING = STAGES * STAGE;
     static constexpr int XCH = 128 * 32 * 4;   // residual chunk: 128 rows x 32 FP32
-    static constexpr int NXB = 3;
-    static constexpr int XNB = 128 * 64 * 2;   // output box: 128 rows x 64 bf16
-    static constexpr int NXN = 2;
-    static constexpr int DATA = RING + NXB * XCH + NXN * XNB;
+    static constexpr int NXB = 2;
+    static constexpr int DATA = RING + NXB * XCH;
     static constexpr int BAR_BYTES = (2 * STAGES + 2 + NXB) * 8 + 8;
     static constexpr int SMEM = DATA + BAR_BYTES + 1024;
 };
@@ -489,7 +492,6 @@ __global__ void __launch_bounds__(192, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *xbuf = smem + C::RING;
-    uint8_t *xnbuf = xbuf + C::NXB * C::XCH;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::DATA);
     uint64_t *empty = full + C::STAGES;
     uint64_t *accf = empty + C::STAGES;
@@ -656,15 +658,11 @@ __global__ void __launch_bounds__(192, 1)
             }
             tmem_st_wait();
             const float rstd = 1.0f / sqrtf(m2 * (1.0f / D) + ep.eps);
-            // ---- pass 2
+            // ---- pass 2: xn = LN(v) from TMEM, written straight from registers
+            const int row = m0 + r;
+            __nv_bfloat16 *xo = reinterpret_cast<__nv_bfloat16 *>(ep.out) + (size_t)row * ep.ldo;
 #pragma unroll 1
             for (int j = 0; j < 6; ++j) {
-                const uint32_t g2 = tc * 6 + j;
-                uint8_t *ob = xnbuf + (g2 & 1) * C::XNB;
-                if (g2 >= 2) {
-                    if (leader) bulk_wait_read<0>();
-                    named_bar_sync(1, 128);
-                }
                 uint32_t a[32], b2[32];
                 tmem_ld32(tl + j * 64, a);
                 tmem_ld32(tl + j * 64 + 32, b2);
@@ -687,15 +685,10 @@ __global__ void __launch_bounds__(192, 1)
                         w[h * 16 + 2 * j4 + 1] = pack_bf16x2(y2, y3);
                     }
                 }
+                if (row < ep.rows) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(xo + j * 64);
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc)
-                    *reinterpret_cast<uint4 *>(ob + r * 128 + ((cc ^ (r & 7)) << 4)) =
-                        make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
-                fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                if (leader) {
-                    tma_store_2d(&tmXN, ob, j * 64, m0);
-                    bulk_commit();
+                    for (int cc = 0; cc < 8; ++cc) dst[cc] = make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
                 }
             }
             tc_fence_before();
@@ -798,13 +791,13 @@ cudaError_t gemm_init_attributes() {
     if ((e = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(k_gemm_rl, cudaFuncAttributeMaxDynamicSharedMemorySize, RlCfg::SMEM)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 192, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<192>::SMEM)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_GEGLU, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_GEGLU, 256, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<256>::SMEM)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_BIAS_ACT, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_BIAS_ACT, 256, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<256>::SMEM)) != cudaSuccess)
         return e;
     if ((e = set_attrs<EPI_QKV, 384>()) != cudaSuccess) return e;
@@ -836,17 +829,16 @@ static cudaError_t launch_pc(const GemmOp &op, cudaStream_t st) {
     const int n_tiles = nblk * ((op.ep.rows + 127) / 128);
     const int grid = n_tiles < g_num_sms ? n_tiles : g_num_sms;
     if (!op.tmO) return cudaErrorInvalidValue;
-    k_gemm_pc<EPI, BN><<<grid, 192, PcCfg<BN>::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmO, op.K, n_tiles, nblk, op.ep);
+    constexpr int EW = EPI == EPI_GEGLU ? 8 : 4;  // epilogue warps
+    k_gemm_pc<EPI, BN, EW><<<grid, 64 + 32 * EW, PcCfg<BN>::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmO, op.K, n_tiles,
+                                                                         nblk, op.ep);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st) {
     if (op.ep.rows <= 0) return cudaSuccess;
     if (op.N % op.bn != 0 || op.K % 64 != 0) return cudaErrorInvalidValue;
-    // the streaming residual kernel keeps a 2-stage operand ring; for K > 384 the
-    // 3-stage single-tile kernel (weights streamed per tile) measured faster
-    if (!fp32 && op.epi == EPI_RESID_LN && op.tmX && op.tmXN && op.ep.ln_g && !op.ep.fin_g && op.N == D &&
-        op.K <= 384) {
+    if (!fp32 && op.epi == EPI_RESID_LN && op.tmX && op.tmXN && op.ep.ln_g && !op.ep.fin_g && op.N == D) {
         const int n_tiles = (op.ep.rows + 127) / 128;
         const int grid = n_tiles < g_num_sms ? n_tiles : g_num_sms;
         k_gemm_rl<<<grid, 192, RlCfg::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmX, *op.tmXN, op.K, n_tiles, op.ep);

@@ -31,7 +31,8 @@ struct GemmOp {
 cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st);
 
 // Per-token row index / position and per-row attention work-unit offsets
-// (qb_off holds 2 * (n_rows + 1) ints: 64-query then 128-query block offsets).
+// (qb_off holds 2 * (n_rows + 1) ints: 64-query then 128-query block offsets,
+// followed by the row of every 128-query block: n_tokens / 128 + n_rows ints).
 cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
                         cudaStream_t st);
 

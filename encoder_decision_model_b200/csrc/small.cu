@@ -59,12 +59,20 @@ __global__ void __launch_bounds__(1024) k_qblock_offsets(const int *__restrict__
     }
 }
 
+// row of every 128-query block: qb_row[q128[r] .. q128[r + 1]) = r
+__global__ void k_qblock_rows(const int *__restrict__ qb_off, int n_rows, int *__restrict__ qb_row) {
+    const int *q128 = qb_off + n_rows + 1;
+    for (int r = blockIdx.x * blockDim.y + threadIdx.y; r < n_rows; r += gridDim.x * blockDim.y)
+        for (int qb = q128[r] + threadIdx.x; qb < q128[r + 1]; qb += blockDim.x) qb_row[qb] = r;
+}
+
 cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
                         cudaStream_t st) {
     if (n_rows <= 0) return cudaSuccess;
     (void)n_tokens;
     k_token_meta<<<min(n_rows, 4096), 256, 0, st>>>(cu_seqlens, n_rows, tok_row, pos);
     k_qblock_offsets<<<1, 1024, 0, st>>>(cu_seqlens, n_rows, qb_off);
+    k_qblock_rows<<<min((n_rows + 7) / 8, 1024), dim3(32, 8), 0, st>>>(qb_off, n_rows, qb_off + 2 * (n_rows + 1));
     return cudaGetLastError();
 }
 
