@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--workload", default="throughput", choices=["throughput", "long"],
                     help="throughput: 1024 rows of 64..1024 tokens; long: 16 rows of 8192 tokens")
     ap.add_argument("--latency-calls", type=int, default=1000)
+    ap.add_argument("--router-reps", type=int, default=5, help="timed jd_route_host calls (0: skip)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=3)
@@ -69,10 +70,12 @@ def workload(args, rank):
     return rows, opts, desc
 
 
-def algorithmic_cost(name, lens, n_markers):
-    """(bytes, flops) per launch of kernel `name` for rows of lengths `lens`."""
+def algorithmic_cost(name, lens, n_markers, kper=None):
+    """(bytes, flops) per launch of kernel `name` for rows of lengths `lens`
+    (`kper`: options per row, needed for the marker attention)."""
     lens = np.asarray(lens, dtype=np.float64)
     T = lens.sum()
+    M = float(n_markers)
     if name == "embed_ln":
         return T * (4 + 1536 + 1536 + 768), T * 3 * D
     if name in ("gemm_qkv_rope", "head0_gemm_in"):
@@ -97,6 +100,15 @@ def algorithmic_cost(name, lens, n_markers):
         return T * (3 * 768 + 768), 4.0 * 64 * NH * vis
     if name == "head1_gemm_kv":
         return T * (768 + 1536), T * 2 * D * 2 * D
+    if name == "head1_gather":  # mask_pos, FP32 state row and BF16 normed row in, both out
+        return M * (4 + 2 * (1536 + 768)), 0.0
+    if name == "head1_marker_attn" and kper is not None:  # K,V of every row once; q in, o out
+        return T * 1536 + M * (768 + 768), 4.0 * 64 * NH * float((np.asarray(kper, np.float64) * lens).sum())
+    if name == "scorer":  # FP32 marker states, the scorer weights, one logit per marker
+        return M * (1536 + 4) + 4 * (D * D + 4 * D + 1), M * (2 * D * D + 2 * D + 8 * D)
+    if name == "readout":  # logits in, probs out, four values per row
+        lens_b = len(lens)
+        return M * 8 + lens_b * (4 + 1 + 16), M * 4.0
     return None
 
 
@@ -291,6 +303,73 @@ def run_reference(args):
 # ----------------------------------------------------------------------------- our arm
 
 
+ROUTER_KERNELS = ("embed_ln", "attn_local", "attn_global", "head0_attn", "head1_gather", "head1_marker_attn",
+                  "scorer", "readout")
+
+
+def measure_router(jl, wpath, local, rank, ranks, reps, peaks):
+    """Router workload: 512 independent requests, each a 256-id state, a question
+    and 72 labels; round 1 scores groups of <=20 labels (4 rows per request), the
+    survivors go to one final row per request.  decisions/s = requests / wall time
+    of jd_route_host (serialisation, both forward rounds, survivor rule, copies).
+    Round 1 is also run alone with per-kernel events to give the HBM fraction of
+    the attention, norm and gather kernels at this shape."""
+    import torch
+    from workloads import Row, requests_config4
+    reqs = requests_config4(512, seed=104 + 1000 * rank)
+    opts = jl.encode_opts(1024, 512, True)
+    m = jl.Model(wpath, 1 << 20, 2048, 2048 * 20, precision=jl.JD_PREC_BF16, device=local)
+    for _ in range(2):
+        out = m.jd_route_host(reqs, opts)
+    ranks.barrier()
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        out = m.jd_route_host(reqs, opts)
+    el = ranks.max(time.perf_counter() - t0)
+    total = ranks.sum(float(len(reqs) * reps))
+
+    rows = [Row(state=q.state, question=q.question, options=q.labels[g:g + 20], qtype=0)
+            for q in reqs for g in range(0, len(q.labels), 20)]
+    hb = jl.jd_serialize(rows, opts)
+    dev = torch.device("cuda", local)
+    up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    keep = [up(hb.tokens), up(hb.cu_seqlens), up(hb.mask_pos), up(hb.opt_off), up(hb.row_type)]
+    B, M, T = hb.n_rows, hb.n_markers, hb.n_tokens
+    batch = jl.Model.device_batch(B, T, M, hb.max_row_len, *keep)
+    outs = dict(logits=torch.empty(M, device=dev), probs=torch.empty(M, device=dev),
+                choice=torch.empty(B, dtype=torch.int32, device=dev), score=torch.empty(B, device=dev),
+                noul=torch.empty(B, device=dev), max_p=torch.empty(B, device=dev))
+    st = torch.cuda.Stream(device=dev)
+    m.jd_decide(batch, **outs, stream=st)
+    torch.cuda.synchronize()
+    m.jd_set_profiling(True)
+    for _ in range(3):
+        m.jd_decide(batch, **outs, stream=st)
+    prof = m.jd_profile_report()
+    m.jd_set_profiling(False)
+    torch.cuda.synchronize()
+    m.jd_check_status()
+    m.close()
+    lens = np.diff(hb.cu_seqlens)
+    r1 = {}
+    for name, (n, tot) in prof.items():
+        d = dict(launches=n // 3, ms=tot / 3)
+        c = algorithmic_cost(name, lens, M, np.diff(hb.opt_off))
+        if c is not None and n:
+            a = tot / n / 1000.0
+            d["hbm_frac"] = c[0] / a / 1e9 / peaks["hbm"]
+            d["tensor_frac"] = c[1] / a / 1e12 / peaks["tc_sust"]
+        r1[name] = d
+    return {"workload": "512 requests x 72 labels of 3..12 ids on a 256-id state; groups of <=20, then one "
+                        "final row of the survivors; head budget 512, max_length 1024, strict",
+            "value": total / el, "unit": "requests/s", "ms_per_call": 1000 * el / reps,
+            "rows_per_round": [int(x) for x in out["rows_per_round"]],
+            "round1": {"rows": int(B), "tokens": int(T), "markers": int(M),
+                       "ms_forward": sum(v["ms"] for v in r1.values()),
+                       "hbm_bound_kernels": {k: r1[k] for k in ROUTER_KERNELS if k in r1},
+                       "per_kernel": r1}}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -409,8 +488,13 @@ def run_ours(args):
                                     "jd_decide_host with CUDA-graph replay, host serialisation and copies included")
         lm.close()
 
-    # ---- roofline of the dominant kernel
+    # ---- router: 512 requests x 72 labels, both rounds and the host work between them
     peaks = read_peaks()
+    router = None
+    if args.router_reps > 0:
+        router = measure_router(jl, weights_path(0), local, rank, ranks, args.router_reps, peaks)
+
+    # ---- roofline of the dominant kernel
     roof = None
     per_kernel = {}
     for name, (n, tot) in prof.items():
@@ -419,7 +503,7 @@ def run_ours(args):
         top = max(prof, key=lambda k: prof[k][1])
         n, tot = prof[top]
         avg_s = tot / n / 1000.0
-        cost = algorithmic_cost(top, lens, M)
+        cost = algorithmic_cost(top, lens, M, np.diff(hb.opt_off))
         if cost is not None:
             byt, fl = cost
             t_hbm = byt / (peaks["hbm"] * 1e9)
@@ -440,7 +524,7 @@ def run_ours(args):
             roof["avg_launch_ms"] = avg_s * 1000.0
             roof["kernel_source_sha"] = kernel_source_sha()
         for name, d in per_kernel.items():
-            c = algorithmic_cost(name, lens, M)
+            c = algorithmic_cost(name, lens, M, np.diff(hb.opt_off))
             if c is None or d["launches_per_step"] == 0:
                 continue
             a = d["ms_per_step"] / d["launches_per_step"] / 1000.0
@@ -462,7 +546,7 @@ def run_ours(args):
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "call": "jd_decide_host (serialise + H2D from pinned staging + forward + D2H + sync)"},
             "gpu_launches": int(launches_per_step * args.steps),
-            "clocks": ck, "per_kernel": per_kernel}
+            "clocks": ck, "per_kernel": per_kernel, "router": router}
     if rank == 0:
         s = json.dumps(line)
         print(s, flush=True)

@@ -1,30 +1,32 @@
-// Bidirectional attention inside each packed row on the 5th-generation tensor
-// cores, global and +-64-window variants.
+// Bidirectional global attention inside each packed row on the 5th-generation
+// tensor cores.
 //
-// "Julia-1 MLX", "Performance": every third encoder layer attends globally,
-// the others within +-64 tokens; the two head layers attend over the whole row
-// ("Julia-1: one score per mask token", "The decision head", step 2).  Rows
-// are packed back to back ("julia1 -- Rust runtime for Julia-1", "Why it is
-// faster"); a work item is one 128-query block of one row and one head, and a
-// persistent CTA per SM walks the item list.  Keys come in 128-key tiles: all
-// of the row's tiles (global), or the two tiles of the band [q0 - 64, q0 + 192)
-// (window); keys outside the row or the window get probability zero.
+// "Julia-1 MLX", "Performance": every third encoder layer attends over the whole
+// row; so do the two head layers ("Julia-1: one score per mask token", "The
+// decision head", step 2).  Rows are packed back to back ("julia1 -- Rust
+// runtime for Julia-1", "Why it is faster").  A work item is one 256-query
+// block of one row and one head: two 128-query tiles (the second is absent
+// when the row ends inside the first) that share every K and V tile, so the
+// keys and values of a row cross from L2 once per 256 queries.  With one
+// 128-query tile per CTA the kernel ran at the L2-to-SM bandwidth; two tiles
+// halve that traffic per query.  A persistent CTA per SM walks the item list.
 //
-//   warp 0 lane 0  TMA producer: Q (128 x 64) once per item into one of two
-//                  buffers; K and V tiles (128 keys x 64, 128-byte swizzle) into
-//                  a three-stage ring
-//   warp 1         TMEM allocation; lane 0 issues tcgen05.mma:
-//                    S_j = Q K_j^T      (M 128, N 128, K 64) into one of two S buffers
-//                    O  += P_j V_j      (M 128, N 64,  K 128; V read MN-major)
-//   warps 2..9     softmax: two warps per TMEM lane quarter, each owning one
-//                  query row per thread and one half (64 keys) of every tile;
-//                  the halves combine row maxima (and, at the end, row sums)
-//                  through shared memory.  The running max is kept lazily: O
-//                  and the sums are rescaled only when the max grows by more
-//                  than 2^8, so P stays below 256.  P is written as bf16 into
-//                  shared memory (K-major, 128-byte swizzle; each half writes
-//                  its own 64-key block).
-// TMEM columns: S buffers 0 and 128, O at 256.
+//   warp 0 lane 0   TMA producer: both Q tiles (128 x 64, 128-byte swizzle)
+//                   once per item into one of two buffers; K tiles (128 keys x
+//                   64) into a four-stage ring, each stage released when its
+//                   S products complete
+//   warp 10 lane 0  TMA producer of the V tiles: a four-stage ring, each stage
+//                   released when its PV products complete
+//   warp 1          TMEM allocation; lane 0 issues tcgen05.mma:
+//                     S_x = Q_x K_j^T  (M 128, N 128, K 64; A, B from shared memory)
+//                     O_x += P_x V_j   (M 128, N 64, K 128; P from TMEM, V read MN-major)
+//   warps 2..5      softmax of Q tile 0, warps 6..9 of Q tile 1: one query
+//                   row per thread (warp w reads TMEM lane quarter w % 4), all
+//                   128 keys of every tile.  The running max is kept lazily: O
+//                   and the row sum are rescaled only when the max grows by
+//                   more than 2^8, so P stays below 256.  P is stored as bf16
+//                   pairs into TMEM, where the PV product reads it.
+// TMEM columns: S_x at 128 x, O_x at 256 + 64 x, P_x at 384 + 64 x.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -35,21 +37,21 @@ namespace {
 constexpr int TQ = 128, TK = 128;
 constexpr int Q_BYTES = TQ * 128;          // 128 rows x 64 bf16
 constexpr int KT_BYTES = TK * 128;         // 128 keys x 64 bf16
-constexpr int KV_STAGE = 2 * KT_BYTES;     // K tile then V tile
-constexpr int P_BYTES = TQ * TK * 2;       // two 64-key blocks of 128 x 128 B
-constexpr int NKV = 3;                     // K/V ring depth
-constexpr int OFF_Q = 0;                   // two Q buffers (work items alternate)
-constexpr int OFF_KV = OFF_Q + 2 * Q_BYTES;
-constexpr int OFF_P = OFF_KV + NKV * KV_STAGE;
-constexpr int OFF_X = OFF_P + 2 * P_BYTES;           // row exchange: max [2][2][128], sum [2][128]
-constexpr int X_BYTES = (2 * 2 * 128 + 2 * 128) * 4;
-constexpr int OFF_BAR = OFF_X + X_BYTES;
-// qfull[2], qfree[2], kvfull[3], kvempty[3], sfull[2], pready[2], pvdone[2], ofree
-constexpr int NBAR = 17;
+constexpr int NK = 4;                      // K ring depth
+constexpr int NV = 4;                      // V ring depth
+constexpr int OFF_Q = 0;                   // [item buffer][q tile]
+constexpr int OFF_K = OFF_Q + 4 * Q_BYTES;
+constexpr int OFF_V = OFF_K + NK * KT_BYTES;
+constexpr int OFF_BAR = OFF_V + NV * KT_BYTES;
+// qfull[2], qfree[2], kfull[NK], kfree[NK], vfull[NV], vfree[NV],
+// sfull[2], sfree[2], pready[2], pvdone[2], ofree[2] (the last five per Q tile)
+constexpr int NBAR = 2 + 2 + 2 * NK + 2 * NV + 5 * 2;
 constexpr int ATC_SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-constexpr uint32_t T_O = 256;
+static_assert(ATC_SMEM <= 227 * 1024, "attention shared memory");
+constexpr uint32_t T_S = 0, T_O = 256, T_P = 384;
 constexpr float kLazy = 8.0f;    // log2 headroom before the running max is moved
-constexpr int SM_THREADS = 256;  // softmax warps 2..9
+constexpr int V_WARP = 10;
+constexpr int ATC_THREADS = 11 * 32;
 }  // namespace
 
 // 2^x with the hardware approximation (ex2.approx.ftz; 2^-inf = 0)
@@ -59,60 +61,68 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]: A is M x K in TMEM (lane = row, two bf16 per column)
+__device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 struct AtcItem {
-    int h, cs, ce, q0, ks0, nt;
+    int h, cs, ce, q0, nt, nx;  // nx: Q tiles in this item (1 or 2)
 };
 
-template <bool LOCAL>
-__device__ __forceinline__ AtcItem atc_item(const int *q128, const int *qb_row, const int *cu, int w) {
+__device__ __forceinline__ AtcItem atc_item(const int *q256, const int *pb_row, const int *cu, int w) {
     AtcItem t;
-    const int qb = w / NH;
+    const int pb = w / NH;
     t.h = w % NH;
-    const int row = qb_row[qb];
+    const int row = pb_row[pb];
     t.cs = cu[row];
     t.ce = cu[row + 1];
-    t.q0 = t.cs + (qb - q128[row]) * TQ;
-    if (LOCAL) {
-        t.ks0 = t.q0 - 64;
-        t.nt = 2;
-    } else {
-        t.ks0 = t.cs;
-        t.nt = (t.ce - t.cs + TK - 1) / TK;
-    }
+    t.q0 = t.cs + (pb - q256[row]) * (2 * TQ);
+    t.nt = (t.ce - t.cs + TK - 1) / TK;
+    t.nx = t.q0 + TQ < t.ce ? 2 : 1;
     return t;
 }
 
-template <bool LOCAL>
-__global__ void __launch_bounds__(64 + SM_THREADS, 1)
+__global__ void __launch_bounds__(ATC_THREADS, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tm, __nv_bfloat16 *__restrict__ out, const int *__restrict__ cu,
               const int *__restrict__ qb_off, int n_rows, unsigned *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *xmax = reinterpret_cast<float *>(smem + OFF_X);  // [S buffer][half][row]
-    float *xsum = xmax + 2 * 2 * 128;                        // [half][row]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *qfull = bars + 0, *qfree = bars + 2, *kvfull = bars + 4, *kvempty = bars + 7, *sfull = bars + 10,
-             *pready = bars + 12, *pvdone = bars + 14, *ofree = bars + 16;
+    uint64_t *qfull = bars + 0, *qfree = bars + 2, *kfull = bars + 4, *kfree = kfull + NK, *vfull = kfree + NK,
+             *vfree = vfull + NV, *sfull = vfree + NV, *sfree = sfull + 2, *pready = sfree + 2, *pvdone = pready + 2,
+             *ofree = pvdone + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBAR);
 
-    const int *q128 = qb_off + n_rows + 1;
-    const int *qb_row = q128 + n_rows + 1;
-    const int n_items = q128[n_rows] * NH;
+    const int *q256 = qb_off + n_rows + 1;
+    const int *pb_row = q256 + n_rows + 1;
+    const int n_items = q256[n_rows] * NH;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NKV; ++i) {
-            mbar_init(&kvfull[i], 1);
-            mbar_init(&kvempty[i], 1);
+        for (int i = 0; i < NK; ++i) {
+            mbar_init(&kfull[i], 1);
+            mbar_init(&kfree[i], 1);
+        }
+        for (int i = 0; i < NV; ++i) {
+            mbar_init(&vfull[i], 1);
+            mbar_init(&vfree[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&qfull[i], 1);
             mbar_init(&qfree[i], 1);
             mbar_init(&sfull[i], 1);
-            mbar_init(&pready[i], SM_THREADS / 32);
+            mbar_init(&sfree[i], 4);
+            mbar_init(&pready[i], 4);
             mbar_init(&pvdone[i], 1);
+            mbar_init(&ofree[i], 4);
         }
-        mbar_init(ofree, SM_THREADS / 32);
         fence_barrier_init();
         fence_proxy_async_smem();
         prefetch_tmap(&tm);
@@ -130,18 +140,30 @@ __global__ void __launch_bounds__(64 + SM_THREADS, 1)
         if (lane == 0) {
             uint32_t J = 0, it = 0;
             for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++it) {
-                const AtcItem t = atc_item<LOCAL>(q128, qb_row, cu, w);
+                const AtcItem t = atc_item(q256, pb_row, cu, w);
                 const uint32_t qbuf = it & 1;
                 if (it >= 2) mbar_wait(&qfree[qbuf], ((it - 2) >> 1) & 1, status);
-                mbar_arrive_expect_tx(&qfull[qbuf], Q_BYTES);
-                tma_load_2d(smem + OFF_Q + qbuf * Q_BYTES, &tm, &qfull[qbuf], t.h * DH, t.q0);
+                mbar_arrive_expect_tx(&qfull[qbuf], t.nx * Q_BYTES);
+                for (int x = 0; x < t.nx; ++x)
+                    tma_load_2d(smem + OFF_Q + (qbuf * 2 + x) * Q_BYTES, &tm, &qfull[qbuf], t.h * DH, t.q0 + x * TQ);
                 for (int j = 0; j < t.nt; ++j, ++J) {
-                    const uint32_t s = J % NKV;
-                    if (J >= NKV) mbar_wait(&kvempty[s], ((J - NKV) / NKV) & 1, status);
-                    uint8_t *st = smem + OFF_KV + s * KV_STAGE;
-                    mbar_arrive_expect_tx(&kvfull[s], KV_STAGE);
-                    tma_load_2d(st, &tm, &kvfull[s], D + t.h * DH, t.ks0 + j * TK);
-                    tma_load_2d(st + KT_BYTES, &tm, &kvfull[s], 2 * D + t.h * DH, t.ks0 + j * TK);
+                    const uint32_t s = J % NK;
+                    if (J >= NK) mbar_wait(&kfree[s], ((J - NK) / NK) & 1, status);
+                    mbar_arrive_expect_tx(&kfull[s], KT_BYTES);
+                    tma_load_2d(smem + OFF_K + s * KT_BYTES, &tm, &kfull[s], D + t.h * DH, t.cs + j * TK);
+                }
+            }
+        }
+    } else if (warp == V_WARP) {
+        if (lane == 0) {
+            uint32_t J = 0;
+            for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
+                const AtcItem t = atc_item(q256, pb_row, cu, w);
+                for (int j = 0; j < t.nt; ++j, ++J) {
+                    const uint32_t s = J % NV;
+                    if (J >= NV) mbar_wait(&vfree[s], ((J - NV) / NV) & 1, status);
+                    mbar_arrive_expect_tx(&vfull[s], KT_BYTES);
+                    tma_load_2d(smem + OFF_V + s * KT_BYTES, &tm, &vfull[s], 2 * D + t.h * DH, t.cs + j * TK);
                 }
             }
         }
@@ -150,148 +172,144 @@ __global__ void __launch_bounds__(64 + SM_THREADS, 1)
             constexpr uint32_t idesc_s = idesc_bf16_f32(TK);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(DH) | (1u << 16);  // B (V) is MN-major
             uint32_t J = 0, it = 0;
+            uint32_t cnt[2] = {0, 0};   // S tiles issued per Q tile, over all items
+            uint32_t uses[2] = {0, 0};  // items that used each Q tile
             for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++it) {
-                const AtcItem t = atc_item<LOCAL>(q128, qb_row, cu, w);
+                const AtcItem t = atc_item(q256, pb_row, cu, w);
                 const uint32_t qbuf = it & 1;
-                const uint32_t q_base = smem_u32(smem + OFF_Q + qbuf * Q_BYTES);
                 mbar_wait(&qfull[qbuf], (it >> 1) & 1, status);
                 tc_fence_after();
-                const uint32_t J0 = J;
-                auto issue_pv = [&](uint32_t Jp) {
-                    const uint32_t b = Jp & 1;
-                    mbar_wait(&pready[b], (Jp >> 1) & 1, status);
-                    if (Jp == J0 && it >= 1) mbar_wait(ofree, (it - 1) & 1, status);
-                    tc_fence_after();
-                    const uint32_t p_base = smem_u32(smem + OFF_P + b * P_BYTES);
-                    const uint32_t v_base = smem_u32(smem + OFF_KV + (Jp % NKV) * KV_STAGE + KT_BYTES);
+                const uint32_t J0 = J, c0[2] = {cnt[0], cnt[1]};
+                auto issue_pv = [&](int j) {
+                    const uint32_t Jp = J0 + j, s = Jp % NV;
+                    mbar_wait(&vfull[s], (Jp / NV) & 1, status);
+                    const uint32_t v_base = smem_u32(smem + OFF_V + s * KT_BYTES);
+                    for (int x = 0; x < t.nx; ++x) {
+                        const uint32_t c = c0[x] + j;
+                        mbar_wait(&pready[x], c & 1, status);
+                        if (j == 0 && uses[x] >= 1) mbar_wait(&ofree[x], (uses[x] - 1) & 1, status);
+                        tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < TK / 16; ++ks) {
-                        const uint64_t ad = sdesc_sw128(p_base + (ks >> 2) * (TQ * 128) + (ks & 3) * 32);
-                        const uint64_t bd = sdesc_sw128(v_base + ks * 16 * 128);
-                        tc_mma_bf16(tmem + T_O, ad, bd, idesc_pv, (Jp != J0 || ks != 0) ? 1u : 0u);
+                        for (int ks = 0; ks < TK / 16; ++ks)
+                            tc_mma_bf16_ts(tmem + T_O + 64 * x, tmem + T_P + 64 * x + 8 * ks,
+                                           sdesc_sw128(v_base + ks * 16 * 128), idesc_pv, (j != 0 || ks != 0) ? 1u : 0u);
+                        tc_commit(&pvdone[x]);
                     }
-                    tc_commit(&pvdone[b]);
-                    tc_commit(&kvempty[Jp % NKV]);
+                    tc_commit(&vfree[s]);
                 };
                 for (int j = 0; j < t.nt; ++j, ++J) {
-                    const uint32_t b = J & 1, s = J % NKV;
-                    mbar_wait(&kvfull[s], (J / NKV) & 1, status);
-                    if (J >= 2) mbar_wait(&pready[b], ((J - 2) >> 1) & 1, status);  // S buffer b read out
-                    tc_fence_after();
-                    const uint32_t k_base = smem_u32(smem + OFF_KV + s * KV_STAGE);
+                    const uint32_t s = J % NK;
+                    mbar_wait(&kfull[s], (J / NK) & 1, status);
+                    const uint32_t k_base = smem_u32(smem + OFF_K + s * KT_BYTES);
+                    for (int x = 0; x < t.nx; ++x) {
+                        const uint32_t c = cnt[x]++;
+                        if (c >= 1) mbar_wait(&sfree[x], (c - 1) & 1, status);  // S_x read out
+                        tc_fence_after();
+                        const uint32_t q_base = smem_u32(smem + OFF_Q + (qbuf * 2 + x) * Q_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc_mma_bf16(tmem + b * TK, sdesc_sw128(q_base + kk * 32), sdesc_sw128(k_base + kk * 32),
-                                    idesc_s, kk != 0);
-                    tc_commit(&sfull[b]);
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma_bf16(tmem + T_S + TK * x, sdesc_sw128(q_base + kk * 32),
+                                        sdesc_sw128(k_base + kk * 32), idesc_s, kk != 0);
+                        tc_commit(&sfull[x]);
+                    }
+                    tc_commit(&kfree[s]);
                     if (j == t.nt - 1) tc_commit(&qfree[qbuf]);
-                    if (j >= 1) issue_pv(J - 1);
+                    if (j >= 1) issue_pv(j - 1);
                 }
-                issue_pv(J - 1);
+                issue_pv(t.nt - 1);
+                for (int x = 0; x < t.nx; ++x) ++uses[x];
             }
         }
     } else {
-        const int q = warp & 3;            // TMEM lane quarter
-        const int hf = (warp - 2) >> 2;    // which 64-key half of each tile
-        const int r = q * 32 + lane;       // query row inside the item
-        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+        const int x = (warp - 2) >> 2;         // Q tile of this warp group
+        const int r = (warp & 3) * 32 + lane;  // query row inside the tile = TMEM lane
+        const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float sl2 = 0.125f * 1.4426950408889634f;
-        uint32_t J = 0, it = 0;
-        for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++it) {
-            const AtcItem t = atc_item<LOCAL>(q128, qb_row, cu, w);
-            const int qi = t.q0 + r;
+        uint32_t c = 0;
+        for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
+            const AtcItem t = atc_item(q256, pb_row, cu, w);
+            if (x >= t.nx) continue;
+            const int qi = t.q0 + x * TQ + r;
             float m = -INFINITY, l = 0.f;
-            for (int j = 0; j < t.nt; ++j, ++J) {
-                const uint32_t b = J & 1;
-                const int k0 = t.ks0 + j * TK + hf * 64;  // first key of this thread's half tile
-                mbar_wait(&sfull[b], (J >> 1) & 1, status);
+            for (int j = 0; j < t.nt; ++j, ++c) {
+                const int k0 = t.cs + j * TK;
+                mbar_wait(&sfull[x], c & 1, status);
                 __syncwarp();
                 tc_fence_after();
-                uint32_t sv[64];
-                tmem_ld32(tl + b * TK + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                tmem_ld32(tl + b * TK + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-                tmem_ld_wait();
-                // keys outside the row (and, windowed, outside |i - j| <= 64) do not take part
-                const bool full = LOCAL ? false : (k0 + 64 <= t.ce);
-                if (!full) {
+                uint32_t sv[128];
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) {
-                        const int key = k0 + e;
-                        bool ok = key >= t.cs && key < t.ce;
-                        if (LOCAL) ok = ok && abs(qi - key) <= 64;
-                        if (!ok) sv[e] = __float_as_uint(-INFINITY);
-                    }
+                for (int q = 0; q < 4; ++q)
+                    tmem_ld32(tl + T_S + TK * x + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * q]));
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfree[x]);
+                // keys past the end of the row do not take part
+                if (k0 + TK > t.ce) {
+#pragma unroll
+                    for (int e = 0; e < TK; ++e)
+                        if (k0 + e >= t.ce) sv[e] = __float_as_uint(-INFINITY);
                 }
                 float m8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(sv[e]);
 #pragma unroll
-                for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(sv[e]));
-                const float mh = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-                // combine with the other half of the row (per S buffer, so the
-                // next tile's write cannot overtake the partner's read)
-                xmax[((b * 2) + hf) * 128 + r] = mh;
-                named_bar_sync(1, SM_THREADS);
-                const float mx = fmaxf(mh, xmax[((b * 2) + (hf ^ 1)) * 128 + r]) * sl2;
+                for (int e = 8; e < TK; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(sv[e]));
+                const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
                 if (mx > m + kLazy) {
                     if (m != -INFINITY) {
                         const float alpha = ex2_approx(m - mx);
                         l *= alpha;
-                        mbar_wait(&pvdone[(J - 1) & 1], ((J - 1) >> 1) & 1, status);
+                        mbar_wait(&pvdone[x], (c - 1) & 1, status);  // every PV product on O_x has landed
                         __syncwarp();
                         tc_fence_after();
-                        uint32_t o[32];  // this half rescales O columns [32 hf, 32 hf + 32)
-                        tmem_ld32(tl + T_O + hf * 32, o);
-                        tmem_ld_wait();
+#pragma unroll 1
+                        for (int hc = 0; hc < 64; hc += 32) {  // 32 columns at a time: S stays in registers
+                            uint32_t o[32];
+                            tmem_ld32(tl + T_O + 64 * x + hc, o);
+                            tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tl + T_O + hf * 32, o);
+                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            tmem_st32(tl + T_O + 64 * x + hc, o);
+                        }
                         tmem_st_wait();
                     }
                     m = mx;
                 }
-                if (J >= 2) mbar_wait(&pvdone[b], ((J - 2) >> 1) & 1, status);  // P buffer b read by the MMA
-                uint8_t *blk = smem + OFF_P + b * P_BYTES + hf * (TQ * 128);
+                uint32_t pk[64];
                 float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < 64; c += 32) {
-                    uint32_t w16[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c + e]), sl2, -m));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + e + 1]), sl2, -m));
-                        ls[(e >> 1) & 3] += p0 + p1;
-                        w16[e >> 1] = pack_bf16x2(p0, p1);
-                    }
-                    const int ch0 = c >> 3;
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4)
-                        *reinterpret_cast<uint4 *>(blk + r * 128 + (((ch0 + k4) ^ (r & 7)) << 4)) =
-                            make_uint4(w16[4 * k4], w16[4 * k4 + 1], w16[4 * k4 + 2], w16[4 * k4 + 3]);
+                for (int e = 0; e < TK; e += 2) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -m));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -m));
+                    ls[(e >> 1) & 3] += p0 + p1;
+                    pk[e >> 1] = pack_bf16x2(p0, p1);
                 }
                 l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-                fence_proxy_async_smem();
+                if (j != 0) mbar_wait(&pvdone[x], (c - 1) & 1, status);  // P_x consumed by the last product
+                __syncwarp();
+                tc_fence_after();
+                tmem_st32(tl + T_P + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+                tmem_st32(tl + T_P + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&pready[b]);
+                if (lane == 0) mbar_arrive(&pready[x]);
             }
-            // O / (l_half0 + l_half1) for this item; this half stores O columns [32 hf, 32 hf + 32)
-            xsum[hf * 128 + r] = l;
-            named_bar_sync(1, SM_THREADS);
-            const float ltot = l + xsum[(hf ^ 1) * 128 + r];
-            mbar_wait(&pvdone[(J - 1) & 1], ((J - 1) >> 1) & 1, status);
+            // O / l for this item's query rows
+            mbar_wait(&pvdone[x], (c - 1) & 1, status);
             __syncwarp();
             tc_fence_after();
-            uint32_t o[32];
-            tmem_ld32(tl + T_O + hf * 32, o);
+            uint32_t o[64];
+            tmem_ld32(tl + T_O + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+            tmem_ld32(tl + T_O + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
             tmem_ld_wait();
-            named_bar_sync(1, SM_THREADS);  // both halves have read xsum before the next item writes it
             if (qi < t.ce) {
-                const float inv = 1.0f / ltot;
-                uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)qi * D + t.h * DH + hf * 32);
+                const float inv = 1.0f / l;
+                uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)qi * D + t.h * DH);
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
+                for (int k4 = 0; k4 < 8; ++k4) {
                     uint32_t wv[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
@@ -302,7 +320,7 @@ __global__ void __launch_bounds__(64 + SM_THREADS, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(ofree);
+            if (lane == 0) mbar_arrive(&ofree[x]);
         }
     }
     __syncthreads();
@@ -313,22 +331,17 @@ __global__ void __launch_bounds__(64 + SM_THREADS, 1)
 }
 
 cudaError_t attn_tc_init_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(k_attn_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATC_SMEM);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_attn_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATC_SMEM);
+    return cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, ATC_SMEM);
 }
 
 cudaError_t launch_attention_tc(const AttnArgs &a, const CUtensorMap *tm128, int num_sms, cudaStream_t st) {
     if (a.n_rows <= 0 || a.n_tokens <= 0) return cudaSuccess;
+    if (a.window >= 0) return cudaErrorInvalidValue;  // global attention only
     // an upper bound of the work items; CTAs beyond the real count exit at once
-    const long items = ((long)a.n_tokens / TQ + a.n_rows) * NH;
+    const long items = ((long)a.n_tokens / (2 * TQ) + a.n_rows) * NH;
     const int grid = (int)(items < num_sms ? items : num_sms);
-    if (a.window >= 0)
-        k_attn_tc<true><<<grid, 64 + SM_THREADS, ATC_SMEM, st>>>(*tm128, (__nv_bfloat16 *)a.o, a.cu_seqlens,
-                                                                   a.qb_off, a.n_rows, a.status);
-    else
-        k_attn_tc<false><<<grid, 64 + SM_THREADS, ATC_SMEM, st>>>(*tm128, (__nv_bfloat16 *)a.o, a.cu_seqlens,
-                                                                    a.qb_off, a.n_rows, a.status);
+    k_attn_tc<<<grid, ATC_THREADS, ATC_SMEM, st>>>(*tm128, (__nv_bfloat16 *)a.o, a.cu_seqlens, a.qb_off, a.n_rows,
+                                                   a.status);
     return cudaGetLastError();
 }
 

@@ -31,8 +31,8 @@ struct GemmOp {
 cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st);
 
 // Per-token row index / position and per-row attention work-unit offsets
-// (qb_off holds 2 * (n_rows + 1) ints: 64-query then 128-query block offsets,
-// followed by the row of every 128-query block: n_tokens / 128 + n_rows ints).
+// (qb_off holds 2 * (n_rows + 1) ints: 64-query then 256-query block offsets,
+// followed by the row of every 256-query block: n_tokens / 256 + n_rows ints).
 cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
                         cudaStream_t st);
 
@@ -47,7 +47,7 @@ struct AttnArgs {
     const void *qkv;
     void *o;
     const int *cu_seqlens;
-    const int *qb_off;        // [B + 1] prefix sums of ceil(len / 64)
+    const int *qb_off;        // the prep kernel's block offsets and 256-query block rows
     int n_rows, n_tokens;
     int window;
     const CUtensorMap *tm_qkv; // BF16 path: box 64 x 64 over [T_cap, 1152]

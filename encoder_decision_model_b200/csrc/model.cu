@@ -370,7 +370,7 @@ jd_status alloc_workspace(jd_model *m) {
     TRY(m->dalloc(&p, T * HFF * es)); m->y = p;
     TRY(m->dalloc(&m->tok_row, T));
     TRY(m->dalloc(&m->pos, T));
-    TRY(m->dalloc(&m->qb_off, 2 * (B + 1) + T / 128 + B));
+    TRY(m->dalloc(&m->qb_off, 2 * (B + 1) + T / 256 + B));
     TRY(m->dalloc(&m->hm, M * D));
     TRY(m->dalloc(&p, M * D * es)); m->xm = p;
     TRY(m->dalloc(&p, M * D * es)); m->qm = p;
@@ -906,7 +906,7 @@ constexpr size_t NA_Y = NA_O + na_up((size_t)NA_TOKENS * D * 2);
 constexpr size_t NA_TOKROW = NA_Y + na_up((size_t)NA_TOKENS * HFF * 2);
 constexpr size_t NA_POS = NA_TOKROW + na_up((size_t)NA_TOKENS * 4);
 constexpr size_t NA_QBOFF = NA_POS + na_up((size_t)NA_TOKENS * 4);
-constexpr size_t NA_HM = NA_QBOFF + na_up((size_t)(2 * (NA_ROWS + 1) + NA_TOKENS / 128 + NA_ROWS) * 4);
+constexpr size_t NA_HM = NA_QBOFF + na_up((size_t)(2 * (NA_ROWS + 1) + NA_TOKENS / 256 + NA_ROWS) * 4);
 constexpr size_t NA_XM = NA_HM + na_up((size_t)NA_MARKERS * D * 4);
 constexpr size_t NA_QM = NA_XM + na_up((size_t)NA_MARKERS * D * 2);
 constexpr size_t NA_OM = NA_QM + na_up((size_t)NA_MARKERS * D * 2);

@@ -21,20 +21,20 @@ __global__ void k_token_meta(const int *__restrict__ cu, int n_rows, int *__rest
 
 // Attention work-unit offsets, one CTA of 1024 threads:
 //   qb_off[r]             = sum over rows < r of ceil(len / 64)   (64-query blocks)
-//   qb_off[n_rows + 1 + r] = sum over rows < r of ceil(len / 128)  (128-query blocks)
+//   qb_off[n_rows + 1 + r] = sum over rows < r of ceil(len / 256)  (256-query blocks)
 __global__ void __launch_bounds__(1024) k_qblock_offsets(const int *__restrict__ cu, int n_rows, int *__restrict__ qb_off) {
     __shared__ int part[2][1024];
     const int tid = threadIdx.x;
     const int per = (n_rows + 1023) / 1024;
     const int r0 = tid * per, r1 = min(n_rows, r0 + per);
-    int s64 = 0, s128 = 0;
+    int s64 = 0, s256 = 0;
     for (int r = r0; r < r1; ++r) {
         const int len = cu[r + 1] - cu[r];
         s64 += (len + 63) / 64;
-        s128 += (len + 127) / 128;
+        s256 += (len + 255) / 256;
     }
     part[0][tid] = s64;
-    part[1][tid] = s128;
+    part[1][tid] = s256;
     __syncthreads();
     for (int off = 1; off < 1024; off <<= 1) {  // inclusive scans
         const int v0 = tid >= off ? part[0][tid - off] : 0;
@@ -44,26 +44,26 @@ __global__ void __launch_bounds__(1024) k_qblock_offsets(const int *__restrict__
         part[1][tid] += v1;
         __syncthreads();
     }
-    int run64 = tid ? part[0][tid - 1] : 0, run128 = tid ? part[1][tid - 1] : 0;
-    int *q128 = qb_off + n_rows + 1;
+    int run64 = tid ? part[0][tid - 1] : 0, run256 = tid ? part[1][tid - 1] : 0;
+    int *q256 = qb_off + n_rows + 1;
     for (int r = r0; r < r1; ++r) {
         const int len = cu[r + 1] - cu[r];
         qb_off[r] = run64;
-        q128[r] = run128;
+        q256[r] = run256;
         run64 += (len + 63) / 64;
-        run128 += (len + 127) / 128;
+        run256 += (len + 255) / 256;
     }
     if (tid == 1023) {
         qb_off[n_rows] = part[0][1023];
-        q128[n_rows] = part[1][1023];
+        q256[n_rows] = part[1][1023];
     }
 }
 
-// row of every 128-query block: qb_row[q128[r] .. q128[r + 1]) = r
-__global__ void k_qblock_rows(const int *__restrict__ qb_off, int n_rows, int *__restrict__ qb_row) {
-    const int *q128 = qb_off + n_rows + 1;
+// row of every 256-query block: pb_row[q256[r] .. q256[r + 1]) = r
+__global__ void k_qblock_rows(const int *__restrict__ qb_off, int n_rows, int *__restrict__ pb_row) {
+    const int *q256 = qb_off + n_rows + 1;
     for (int r = blockIdx.x * blockDim.y + threadIdx.y; r < n_rows; r += gridDim.x * blockDim.y)
-        for (int qb = q128[r] + threadIdx.x; qb < q128[r + 1]; qb += blockDim.x) qb_row[qb] = r;
+        for (int pb = q256[r] + threadIdx.x; pb < q256[r + 1]; pb += blockDim.x) pb_row[pb] = r;
 }
 
 cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
