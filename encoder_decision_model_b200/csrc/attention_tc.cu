@@ -25,7 +25,11 @@
 //                   128 keys of every tile.  The running max is kept lazily: O
 //                   and the row sum are rescaled only when the max grows by
 //                   more than 2^8, so P stays below 256.  P is stored as bf16
-//                   pairs into TMEM, where the PV product reads it.
+//                   pairs into TMEM, where the PV product reads it.  The two
+//                   groups take turns at the exponentials (named barriers 1 and
+//                   2), so that the special-function unit, which bounds that
+//                   phase, is busy with one group while the other loads S,
+//                   takes the row max and hands P over.
 // TMEM columns: S_x at 128 x, O_x at 256 + 64 x, P_x at 384 + 64 x.
 
 #include "common.cuh"
@@ -52,7 +56,15 @@ constexpr uint32_t T_S = 0, T_O = 256, T_P = 384;
 constexpr float kLazy = 8.0f;    // log2 headroom before the running max is moved
 constexpr int V_WARP = 10;
 constexpr int ATC_THREADS = 11 * 32;
+constexpr int BAR_G0_DONE = 1, BAR_G1_DONE = 2, BAR_ITEM = 3;  // named barriers of the softmax groups
 }  // namespace
+
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
 
 // 2^x with the hardware approximation (ex2.approx.ftz; 2^-inf = 0)
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -230,6 +242,8 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             const AtcItem t = atc_item(q256, pb_row, cu, w);
             if (x >= t.nx) continue;
             const int qi = t.q0 + x * TQ + r;
+            const bool pp = t.nx == 2;  // both groups busy: alternate the exponential phases
+            if (pp) named_bar_sync(BAR_ITEM, 256);
             float m = -INFINITY, l = 0.f;
             for (int j = 0; j < t.nt; ++j, ++c) {
                 const int k0 = t.cs + j * TK;
@@ -250,13 +264,15 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     for (int e = 0; e < TK; ++e)
                         if (k0 + e >= t.ce) sv[e] = __float_as_uint(-INFINITY);
                 }
-                float m8[8];
+                float m4[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(sv[e]);
+                for (int e = 0; e < 4; ++e) m4[e] = __uint_as_float(sv[e]);
 #pragma unroll
-                for (int e = 8; e < TK; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(sv[e]));
-                const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * sl2;
+                for (int e = 4; e < TK; e += 8)
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+                        m4[a] = fmax3(m4[a], __uint_as_float(sv[e + 2 * a]), __uint_as_float(sv[e + 2 * a + 1]));
+                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
                 if (mx > m + kLazy) {
                     if (m != -INFINITY) {
                         const float alpha = ex2_approx(m - mx);
@@ -277,21 +293,36 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     }
                     m = mx;
                 }
-                uint32_t pk[64];
+                if (pp) {
+                    if (x == 0) {
+                        if (j != 0) named_bar_sync(BAR_G1_DONE, 256);
+                    } else {
+                        named_bar_sync(BAR_G0_DONE, 256);
+                    }
+                }
                 float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int e = 0; e < TK; e += 2) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -m));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -m));
-                    ls[(e >> 1) & 3] += p0 + p1;
-                    pk[e >> 1] = pack_bf16x2(p0, p1);
+                for (int hk = 0; hk < 2; ++hk) {  // 64 keys at a time; the first half's store overlaps the second
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int e = 0; e < 64; e += 2) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[64 * hk + e]), sl2, -m));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[64 * hk + e + 1]), sl2, -m));
+                        ls[(e >> 1) & 3] += p0 + p1;
+                        pk[e >> 1] = pack_bf16x2(p0, p1);
+                    }
+                    if (hk == 0) {
+                        if (j != 0) mbar_wait(&pvdone[x], (c - 1) & 1, status);  // P_x consumed by the last product
+                        __syncwarp();
+                        tc_fence_after();
+                    }
+                    tmem_st32(tl + T_P + 64 * x + 32 * hk, pk);
+                }
+                if (pp) {
+                    if (x == 0) named_bar_arrive(BAR_G0_DONE, 256);
+                    else if (j != t.nt - 1) named_bar_arrive(BAR_G1_DONE, 256);
                 }
                 l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-                if (j != 0) mbar_wait(&pvdone[x], (c - 1) & 1, status);  // P_x consumed by the last product
-                __syncwarp();
-                tc_fence_after();
-                tmem_st32(tl + T_P + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-                tmem_st32(tl + T_P + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();

@@ -461,34 +461,49 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
 // looping over 128-row tiles; the 384 accumulator columns stay in one TMEM
 // buffer, so the overlap comes from the producer running ahead (the next
 // tile's A / W stages load while this tile's epilogue streams the residual).
-//   warp 0 lane 0  TMA producer: A box 128 x 64, W as two 192 x 64 boxes (3 stages)
+//   warp 0 lane 0  TMA producer: A box 128 x 64, W as two 192 x 64 boxes (STAGES-deep ring)
 //   warp 1         TMEM allocation; lane 0 issues the N = 2 x 192 MMAs
 //   warps 2..5     epilogue, one row per thread:
 //     pass 1  per 32-column chunk: the residual chunk (128 x 32 FP32, 128-byte
-//             swizzle) arrives by TMA (two buffers, prefetched across
-//             tiles); v = x + acc (+ bias) is written back in place, stored to
-//             x by TMA and parked in TMEM; row mean and M2 are merged chunk by
+//             swizzle) arrives by TMA (NXB buffers, prefetched across tiles,
+//             so NXB - 1 chunk loads are in flight while one is processed);
+//             v = x + acc (+ bias) is written back in place, stored to x by
+//             TMA and parked in TMEM; row mean and M2 are merged chunk by
 //             chunk (Chan's pairwise update), so one pass yields the moments;
 //     pass 2  xn = LN(v) from TMEM, stored from registers (the shared memory
-//             goes to a three-stage operand ring instead of output staging).
+//             goes to the operand ring and the residual buffers instead of
+//             output staging).
+// The residual stream is the HBM traffic of this kernel; with two buffers the
+// loads in flight per SM covered about half of the memory latency.
+template <int STAGES_, int NXB_>
 struct RlCfg {
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = 384 * 128;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int STAGES = 3;
+    static constexpr int STAGES = STAGES_;
     static constexpr int RING = STAGES * STAGE;
     static constexpr int XCH = 128 * 32 * 4;   // residual chunk: 128 rows x 32 FP32
-    static constexpr int NXB = 2;
+    static constexpr int NXB = NXB_;
     static constexpr int DATA = RING + NXB * XCH;
     static constexpr int BAR_BYTES = (2 * STAGES + 2 + NXB) * 8 + 8;
     static constexpr int SMEM = DATA + BAR_BYTES + 1024;
+    static_assert(NXB >= 2 && NXB <= 12 && SMEM <= 227 * 1024, "residual GEMM shared memory");
 };
+#ifndef JD_RL_STAGES
+#define JD_RL_STAGES 2
+#endif
+#ifndef JD_RL_NXB
+#define JD_RL_NXB 6
+#endif
+constexpr int RL_STAGES = JD_RL_STAGES, RL_NXB = JD_RL_NXB;
+using RlCur = RlCfg<RL_STAGES, RL_NXB>;
 
+template <int STAGES_, int NXB_>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_rl(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXN, int K, int n_tiles,
               EpiParams ep) {
-    using C = RlCfg;
+    using C = RlCfg<STAGES_, NXB_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *xbuf = smem + C::RING;
@@ -578,7 +593,7 @@ __global__ void __launch_bounds__(192, 1)
         const bool leader = threadIdx.x == 64;
         const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
         const int first = blockIdx.x;
-        // residual chunk loads: chunk index g = (local tile) * 12 + c into buffer g % 3
+        // residual chunk loads: chunk index g = (local tile) * 12 + c into buffer g % NXB
         if (leader && first < n_tiles) {
             for (int c = 0; c < C::NXB; ++c) {
                 mbar_arrive_expect_tx(&xfull[c], C::XCH);
@@ -590,7 +605,6 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t tc = 0;
         for (int t = first; t < n_tiles; t += gridDim.x, ++tc) {
             const int m0 = t * 128;
-            const int tnext = t + gridDim.x;
             mbar_wait(accf, tc & 1, ep.status);
             __syncwarp();
             tc_fence_after();
@@ -646,13 +660,17 @@ __global__ void __launch_bounds__(192, 1)
                 if (leader) {
                     tma_store_2d(&tmX, xb, c * 32, m0);
                     bulk_commit();
-                    // refill this buffer with the chunk three ahead (this tile, else the next one)
-                    const int cn = c + C::NXB;
-                    const int tt = cn < 12 ? t : tnext;
-                    if (tt < n_tiles) {
-                        bulk_wait_read<0>();
-                        mbar_arrive_expect_tx(&xfull[b], C::XCH);
-                        tma_load_2d(xb, &tmX, &xfull[b], (cn % 12) * 32, tt * 128);
+                    // refill the previous chunk's buffer (its store has read it once at most
+                    // this chunk's store is pending) with chunk g - 1 + NXB
+                    if (g >= 1) {
+                        const uint32_t h = g - 1 + C::NXB;
+                        const int th = first + (int)(h / 12) * (int)gridDim.x;
+                        if (th < n_tiles) {
+                            const uint32_t bp = (g - 1) % C::NXB;
+                            bulk_wait_read<1>();
+                            mbar_arrive_expect_tx(&xfull[bp], C::XCH);
+                            tma_load_2d(xbuf + bp * C::XCH, &tmX, &xfull[bp], (int)(h % 12) * 32, th * 128);
+                        }
                     }
                 }
             }
@@ -789,7 +807,8 @@ cudaError_t gemm_init_attributes() {
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(k_gemm_rl, cudaFuncAttributeMaxDynamicSharedMemorySize, RlCfg::SMEM)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(k_gemm_rl<RL_STAGES, RL_NXB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  RlCur::SMEM)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 192, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<192>::SMEM)) != cudaSuccess)
@@ -841,7 +860,8 @@ cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st) {
     if (!fp32 && op.epi == EPI_RESID_LN && op.tmX && op.tmXN && op.ep.ln_g && !op.ep.fin_g && op.N == D) {
         const int n_tiles = (op.ep.rows + 127) / 128;
         const int grid = n_tiles < g_num_sms ? n_tiles : g_num_sms;
-        k_gemm_rl<<<grid, 192, RlCfg::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmX, *op.tmXN, op.K, n_tiles, op.ep);
+        k_gemm_rl<RL_STAGES, RL_NXB><<<grid, 192, RlCur::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmX, *op.tmXN, op.K,
+                                                                     n_tiles, op.ep);
         return cudaGetLastError();
     }
     if (!fp32) {  // persistent tcgen05 kernels for the column-split epilogues
