@@ -178,6 +178,8 @@ __global__ void __launch_bounds__(256, 1)
 //                  swizzle) in shared memory and written by one TMA bulk
 //                  store each (double-buffered); GEGLU outputs go straight
 //                  from registers to global memory.
+constexpr int GEGLU_EW = 8;  // GEGLU epilogue warps (16 measured no faster)
+
 template <int BN>
 struct PcCfg {
     static constexpr int A_BYTES = 128 * 128;
@@ -230,7 +232,9 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
     if constexpr (EPI == EPI_GEGLU) {
         // stored straight from registers: a shared-memory staging pass here
         // competes with the 256-wide MMAs for shared-memory bandwidth; with
-        // NPART warps per TMEM lane quarter each takes G / NPART output columns
+        // NPART warps per TMEM lane quarter each takes G / NPART output columns.
+        // GELU uses the rational erf approximation (gelu_as, |error| < 5e-7):
+        // with erff this epilogue was slower than the tile's MMAs.
         constexpr int G = BN / 2;
         constexpr int GP = G / NPART;
         const int row = row0 + r;
@@ -249,8 +253,8 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int j = q * 8 + e * 2;
-                        w[e] = pack_bf16x2(gelu_erf(__uint_as_float(u[j])) * __uint_as_float(g[j]),
-                                           gelu_erf(__uint_as_float(u[j + 1])) * __uint_as_float(g[j + 1]));
+                        w[e] = pack_bf16x2(gelu_as(__uint_as_float(u[j])) * __uint_as_float(g[j]),
+                                           gelu_as(__uint_as_float(u[j + 1])) * __uint_as_float(g[j + 1]));
                     }
                     dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
@@ -813,7 +817,7 @@ cudaError_t gemm_init_attributes() {
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 192, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<192>::SMEM)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_GEGLU, 256, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_GEGLU, 256, GEGLU_EW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<256>::SMEM)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_BIAS_ACT, 256, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -848,7 +852,7 @@ static cudaError_t launch_pc(const GemmOp &op, cudaStream_t st) {
     const int n_tiles = nblk * ((op.ep.rows + 127) / 128);
     const int grid = n_tiles < g_num_sms ? n_tiles : g_num_sms;
     if (!op.tmO) return cudaErrorInvalidValue;
-    constexpr int EW = EPI == EPI_GEGLU ? 8 : 4;  // epilogue warps
+    constexpr int EW = EPI == EPI_GEGLU ? GEGLU_EW : 4;  // epilogue warps
     k_gemm_pc<EPI, BN, EW><<<grid, 64 + 32 * EW, PcCfg<BN>::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmO, op.K, n_tiles,
                                                                          nblk, op.ep);
     return cudaGetLastError();
