@@ -38,6 +38,15 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // Exact GELU x * Phi(x), Phi written with erff.
+// 32-byte store (8 x 32 bits) to global memory; p must be 32-byte aligned.  A warp
+// writing one row per thread then fills whole 32-byte sectors per instruction.
+__device__ __forceinline__ void st_global_v8(void *p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
+                                             uint32_t a5, uint32_t a6, uint32_t a7) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2),
+                 "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+                 : "memory");
+}
+
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
 // GELU(x) = x Phi(x), Phi(x) = (1 + erf(x / sqrt 2)) / 2, with erf from the rational

@@ -245,18 +245,18 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
             tmem_ld32(tacc + c, u);
             tmem_ld32(tacc + G + c, g);
             tmem_ld_wait();
-            if (row < ep.rows) {
-                uint4 *dst = reinterpret_cast<uint4 *>(o + c);
+            if (row < ep.rows) {  // 32-byte stores: a warp instruction fills whole sectors
+                uint8_t *dst = reinterpret_cast<uint8_t *>(o + c);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t w[4];
+                for (int q = 0; q < 2; ++q) {
+                    uint32_t w[8];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = q * 8 + e * 2;
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = q * 16 + e * 2;
                         w[e] = pack_bf16x2(gelu_as(__uint_as_float(u[j])) * __uint_as_float(g[j]),
                                            gelu_as(__uint_as_float(u[j + 1])) * __uint_as_float(g[j + 1]));
                     }
-                    dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
+                    st_global_v8(dst + 32 * q, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
                 }
             }
         }
@@ -707,10 +707,12 @@ __global__ void __launch_bounds__(192, 1)
                         w[h * 16 + 2 * j4 + 1] = pack_bf16x2(y2, y3);
                     }
                 }
-                if (row < ep.rows) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(xo + j * 64);
+                if (row < ep.rows) {  // 32-byte stores: a warp instruction fills whole sectors
+                    uint8_t *dst = reinterpret_cast<uint8_t *>(xo + j * 64);
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) dst[cc] = make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
+                    for (int cc = 0; cc < 4; ++cc)
+                        st_global_v8(dst + 32 * cc, w[8 * cc], w[8 * cc + 1], w[8 * cc + 2], w[8 * cc + 3], w[8 * cc + 4],
+                                     w[8 * cc + 5], w[8 * cc + 6], w[8 * cc + 7]);
                 }
             }
             tc_fence_before();
