@@ -336,17 +336,17 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             tmem_ld32(tl + T_O + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
             tmem_ld32(tl + T_O + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
             tmem_ld_wait();
-            if (qi < t.ce) {
+            if (qi < t.ce) {  // 32-byte stores: a warp instruction fills whole sectors
                 const float inv = 1.0f / l;
-                uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)qi * D + t.h * DH);
+                uint8_t *dst = reinterpret_cast<uint8_t *>(out + (size_t)qi * D + t.h * DH);
 #pragma unroll
-                for (int k4 = 0; k4 < 8; ++k4) {
-                    uint32_t wv[4];
+                for (int k8 = 0; k8 < 4; ++k8) {
+                    uint32_t wv[8];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        wv[e] = pack_bf16x2(__uint_as_float(o[8 * k4 + 2 * e]) * inv,
-                                            __uint_as_float(o[8 * k4 + 2 * e + 1]) * inv);
-                    dst[k4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    for (int e = 0; e < 8; ++e)
+                        wv[e] = pack_bf16x2(__uint_as_float(o[16 * k8 + 2 * e]) * inv,
+                                            __uint_as_float(o[16 * k8 + 2 * e + 1]) * inv);
+                    st_global_v8(dst + 32 * k8, wv[0], wv[1], wv[2], wv[3], wv[4], wv[5], wv[6], wv[7]);
                 }
             }
             tc_fence_before();
