@@ -30,7 +30,7 @@ struct EpiParams {
     void *out;               // [rows, ldo] of OutT (unused by a RESID_LN without ln_g)
     int ldo;
     const float *bias;       // [N] by weight row, or null
-    const float2 *rope;      // [MAX_POS][32] (cos, sin), or null
+    const float4 *rope;      // [16][MAX_POS]: plane k holds (cos, sin) of pairs 2k, 2k + 1 per position, or null
     int out_col0;            // column offset of this launch's output inside the tensor map (BF16 path)
     const int *pos;          // [rows] position within the request row
     int rope_cols;           // output columns [0, rope_cols) are rotated
@@ -190,7 +190,7 @@ __device__ __forceinline__ void epi_qkv_row(const float *acc, int row, int n0, c
             b1 += ep.bias[n + 33 + i];
         }
         if (ep.rope && n < ep.rope_cols) {
-            const float4 cs = *reinterpret_cast<const float4 *>(ep.rope + (size_t)pos * 32 + i);
+            const float4 cs = ep.rope[(size_t)(i >> 1) * MAX_POS + pos];
             const float r0 = a0 * cs.x - b0 * cs.y, s0 = b0 * cs.x + a0 * cs.y;
             const float r1 = a1 * cs.z - b1 * cs.w, s1 = b1 * cs.z + a1 * cs.w;
             a0 = r0; b0 = s0; a1 = r1; b1 = s1;

@@ -237,14 +237,10 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
         // with erff this epilogue was slower than the tile's MMAs.
         constexpr int G = BN / 2;
         constexpr int GP = G / NPART;
+        static_assert(GP == 64, "two 32-column chunks per warp");
         const int row = row0 + r;
         __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(ep.out) + (size_t)row * ep.ldo + n0 / 2;
-#pragma unroll 1
-        for (int c = part * GP; c < (part + 1) * GP; c += 32) {
-            uint32_t u[32], g[32];
-            tmem_ld32(tacc + c, u);
-            tmem_ld32(tacc + G + c, g);
-            tmem_ld_wait();
+        auto emit = [&](const uint32_t (&u)[32], const uint32_t (&g)[32], int c) {
             if (row < ep.rows) {  // 32-byte stores: a warp instruction fills whole sectors
                 uint8_t *dst = reinterpret_cast<uint8_t *>(o + c);
 #pragma unroll
@@ -259,7 +255,18 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
                     st_global_v8(dst + 32 * q, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
                 }
             }
-        }
+        };
+        // the second chunk's TMEM loads are in flight while the first chunk computes
+        const int c0 = part * GP;
+        uint32_t u0[32], g0[32], u1[32], g1[32];
+        tmem_ld32(tacc + c0, u0);
+        tmem_ld32(tacc + G + c0, g0);
+        tmem_ld_wait();
+        tmem_ld32(tacc + c0 + 32, u1);
+        tmem_ld32(tacc + G + c0 + 32, g1);
+        emit(u0, g0, c0);
+        tmem_ld_wait();
+        emit(u1, g1, c0 + 32);
     } else if constexpr (EPI == EPI_BIAS_ACT) {
 #pragma unroll 1
         for (int c = 0; c < BN; c += 64) {
@@ -429,10 +436,11 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
             if constexpr (EPI == EPI_QKV) {
                 if (ep.rope && n0 < ep.rope_cols) {
                     const int row = row0 + lane;
-                    const float4 *src = reinterpret_cast<const float4 *>(ep.rope + (size_t)(row < ep.rows ? ep.pos[row] : 0) * 32);
+                    // position-minor planes: consecutive rows (positions) of a warp read one contiguous span
+                    const float4 *src = ep.rope + (row < ep.rows ? ep.pos[row] : 0);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float4 v = src[i];
+                        const float4 v = src[(size_t)i * MAX_POS];
                         cs[2 * i] = make_float2(v.x, v.y);
                         cs[2 * i + 1] = make_float2(v.z, v.w);
                     }

@@ -172,7 +172,7 @@ struct jd_model {
     float *in_b[2] = {}, *out_b[2] = {}, *l1_b[2] = {}, *l2_b[2] = {};
     float *sc_g = nullptr, *sc_b = nullptr, *sc_w1t = nullptr, *sc_b1 = nullptr, *sc_w2 = nullptr, *sc_b2 = nullptr;
     float *lin_w = nullptr, *lin_b = nullptr;
-    float2 *rope_g = nullptr, *rope_l = nullptr;
+    float4 *rope_g = nullptr, *rope_l = nullptr;  // [16][MAX_POS] (cos, sin) of pairs 2k, 2k + 1
 
     // workspace
     float *x = nullptr;
@@ -282,15 +282,19 @@ jd_status load_proj(jd_model *m, WeightFile &wf, const std::string &name, int N,
     return upload_proj(m, h, 0, N, K, bn, p);
 }
 
-jd_status make_rope_table(jd_model *m, double theta, float2 **dst) {
-    std::vector<float2> h((size_t)MAX_POS * 32);
-    for (int p = 0; p < MAX_POS; ++p)
-        for (int i = 0; i < 32; ++i) {
-            const double ang = (double)p * std::pow(theta, -2.0 * i / 64.0);
-            h[(size_t)p * 32 + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+// RoPE angles p * theta^(-2i/64) in double, stored as 16 position-minor planes:
+// plane k, position p = (cos, sin) of frequency 2k, then of 2k + 1.
+jd_status make_rope_table(jd_model *m, double theta, float4 **dst) {
+    std::vector<float4> h((size_t)16 * MAX_POS);
+    for (int k = 0; k < 16; ++k)
+        for (int p = 0; p < MAX_POS; ++p) {
+            const double a0 = (double)p * std::pow(theta, -2.0 * (2 * k) / 64.0);
+            const double a1 = (double)p * std::pow(theta, -2.0 * (2 * k + 1) / 64.0);
+            h[(size_t)k * MAX_POS + p] =
+                make_float4((float)std::cos(a0), (float)std::sin(a0), (float)std::cos(a1), (float)std::sin(a1));
         }
     TRY(m->dalloc(dst, h.size()));
-    CK(cudaMemcpy(*dst, h.data(), h.size() * sizeof(float2), cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(*dst, h.data(), h.size() * sizeof(float4), cudaMemcpyHostToDevice));
     return JD_OK;
 }
 
