@@ -253,6 +253,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory matrix descriptor: K-major tile with 64-byte swizzle, rows of 64
+// bytes (32 bf16), 8-row atoms 512 bytes apart (tile base 512-byte aligned).
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
+    d |= (uint64_t)1 << 16;                     // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(512 >> 4) << 32;            // stride byte offset: 8 rows x 64 B
+    d |= (uint64_t)1 << 46;                     // descriptor version (sm_100)
+    d |= (uint64_t)4 << 61;                     // 64-byte swizzle
+    return d;
+}
+
 // Instruction descriptor for kind::f16: bf16 A/B, f32 D, K-major A and B, M = 128.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);

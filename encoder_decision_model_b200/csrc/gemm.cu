@@ -473,7 +473,10 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
 // looping over 128-row tiles; the 384 accumulator columns stay in one TMEM
 // buffer, so the overlap comes from the producer running ahead (the next
 // tile's A / W stages load while this tile's epilogue streams the residual).
-//   warp 0 lane 0  TMA producer: A box 128 x 64, W as two 192 x 64 boxes (STAGES-deep ring)
+//   warp 0 lane 0  TMA producer: per 32-wide k-block, A box 128 x 32 and W as two 192 x 32
+//                  boxes (64-byte swizzle) into a STAGES-deep ring; 32-wide k-blocks give
+//                  twice the stages of 64-wide ones in the same memory, so more of the
+//                  operand loads are in flight (the K = 1152 mainloop waited on them)
 //   warp 1         TMEM allocation; lane 0 issues the N = 2 x 192 MMAs
 //   warps 2..5     epilogue, one row per thread:
 //     pass 1  per 32-column chunk: the residual chunk (128 x 32 FP32, 128-byte
@@ -489,8 +492,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
 // loads in flight per SM covered about half of the memory latency.
 template <int STAGES_, int NXB_>
 struct RlCfg {
-    static constexpr int A_BYTES = 128 * 128;
-    static constexpr int B_BYTES = 384 * 128;
+    static constexpr int A_BYTES = 128 * 64;   // 128 rows x 32 bf16
+    static constexpr int B_BYTES = 384 * 64;   // 384 rows x 32 bf16
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int STAGES = STAGES_;
     static constexpr int RING = STAGES * STAGE;
@@ -502,7 +505,7 @@ struct RlCfg {
     static_assert(NXB >= 2 && NXB <= 12 && SMEM <= 227 * 1024, "residual GEMM shared memory");
 };
 #ifndef JD_RL_STAGES
-#define JD_RL_STAGES 2
+#define JD_RL_STAGES 4
 #endif
 #ifndef JD_RL_NXB
 #define JD_RL_NXB 6
@@ -527,7 +530,7 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xfull + C::NXB);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int KB = K / 64;
+    const int KB = K / 32;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -567,9 +570,9 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     uint8_t *sa = smem + s * C::STAGE;
                     mbar_arrive_expect_tx(&full[s], C::STAGE);
-                    tma_load_2d(sa, &tmA, &full[s], kb * 64, m0);
-                    tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * 64, 0);
-                    tma_load_2d(sa + C::A_BYTES + 192 * 128, &tmB, &full[s], kb * 64, 192);
+                    tma_load_2d(sa, &tmA, &full[s], kb * 32, m0);
+                    tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * 32, 0);
+                    tma_load_2d(sa + C::A_BYTES + 192 * 64, &tmB, &full[s], kb * 32, 192);
                 }
             }
         }
@@ -588,11 +591,11 @@ __global__ void __launch_bounds__(192, 1)
                     const uint32_t a_base = smem_u32(smem + s * C::STAGE);
                     const uint32_t b_base = a_base + C::A_BYTES;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        tc_mma_bf16(tmem, sdesc_sw128(a_base + k * 32), sdesc_sw128(b_base + k * 32), idesc,
+                    for (int k = 0; k < 2; ++k) {
+                        tc_mma_bf16(tmem, sdesc_sw64(a_base + k * 32), sdesc_sw64(b_base + k * 32), idesc,
                                     (kb | k) != 0);
-                        tc_mma_bf16(tmem + 192, sdesc_sw128(a_base + k * 32),
-                                    sdesc_sw128(b_base + 192 * 128 + k * 32), idesc, (kb | k) != 0);
+                        tc_mma_bf16(tmem + 192, sdesc_sw64(a_base + k * 32),
+                                    sdesc_sw64(b_base + 192 * 64 + k * 32), idesc, (kb | k) != 0);
                     }
                     tc_commit(&empty[s]);
                 }
@@ -871,10 +874,11 @@ static cudaError_t launch_pc(const GemmOp &op, cudaStream_t st) {
 cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st) {
     if (op.ep.rows <= 0) return cudaSuccess;
     if (op.N % op.bn != 0 || op.K % 64 != 0) return cudaErrorInvalidValue;
-    if (!fp32 && op.epi == EPI_RESID_LN && op.tmX && op.tmXN && op.ep.ln_g && !op.ep.fin_g && op.N == D) {
+    if (!fp32 && op.epi == EPI_RESID_LN && op.tmX && op.tmXN && op.tmA64 && op.tmB64 && op.ep.ln_g && !op.ep.fin_g &&
+        op.N == D && op.K % 32 == 0) {
         const int n_tiles = (op.ep.rows + 127) / 128;
         const int grid = n_tiles < g_num_sms ? n_tiles : g_num_sms;
-        k_gemm_rl<RL_STAGES, RL_NXB><<<grid, 192, RlCur::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmX, *op.tmXN, op.K,
+        k_gemm_rl<RL_STAGES, RL_NXB><<<grid, 192, RlCur::SMEM, st>>>(*op.tmA64, *op.tmB64, *op.tmX, *op.tmXN, op.K,
                                                                      n_tiles, op.ep);
         return cudaGetLastError();
     }

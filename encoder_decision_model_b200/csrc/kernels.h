@@ -23,6 +23,8 @@ struct GemmOp {
     const CUtensorMap *tmO;   // BF16 column-split epilogues: output, box 64 x 32, 128-byte swizzle
     const CUtensorMap *tmX;   // BF16 residual epilogue: FP32 residual, box 32 x 128, 128-byte swizzle
     const CUtensorMap *tmXN;  // BF16 residual epilogue: LayerNorm output, box 64 x 128, 128-byte swizzle
+    const CUtensorMap *tmA64; // BF16 residual GEMM: A box 32 x 128, 64-byte swizzle
+    const CUtensorMap *tmB64; // BF16 residual GEMM: W box 32 x 192, 64-byte swizzle
     const float *A32;         // FP32 path: A [rows, lda]
     int lda;
     const float *W32;         // FP32 path: W [N, K]

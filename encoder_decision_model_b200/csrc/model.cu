@@ -131,9 +131,10 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D map over [rows, cols] with row stride ld (elements); box = box_cols x box_rows, 128-byte swizzle.
+// 2-D map over [rows, cols] with row stride ld (elements); box = box_cols x box_rows, 128-byte
+// swizzle unless sw64 (64-byte swizzle, for boxes of 32 bf16 columns).
 jd_status make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_cols,
-                   uint32_t box_rows, bool fp32 = false) {
+                   uint32_t box_rows, bool fp32 = false, bool sw64 = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(JD_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     cuuint64_t dims[2] = {cols, rows};
@@ -141,7 +142,8 @@ jd_status make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t row
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t es[2] = {1, 1};
     CUresult r = fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(JD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return JD_OK;
@@ -150,6 +152,7 @@ jd_status make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t row
 struct ProjW {            // one projection weight [N, K]
     void *w = nullptr;    // bf16 or f32 on device
     CUtensorMap tm{};     // BF16 mode only
+    CUtensorMap tm64{};   // BF16 mode, 384-wide tiles: box 32 x 192, 64-byte swizzle (residual GEMM)
     int N = 0, K = 0;
 };
 
@@ -182,6 +185,7 @@ struct jd_model {
     void *xm = nullptr, *qm = nullptr, *om = nullptr, *xnm = nullptr, *ym = nullptr;
     unsigned *status = nullptr;
     CUtensorMap tm_xn{}, tm_o{}, tm_y_enc{}, tm_y_head{}, tm_qkv{}, tm_xm{}, tm_om{}, tm_xnm{}, tm_ym{};
+    CUtensorMap tm_o64{}, tm_y_enc64{}, tm_y_head64{};  // residual GEMM A operands: box 32 x 128, 64-byte swizzle
     // output maps of the column-split epilogues (box 64 x 32)
     CUtensorMap to_qkv{}, to_y_enc{}, to_y_head{}, to_qm{}, to_ym{};
     CUtensorMap tm_x32{};  // FP32 residual stream, box 32 x 128
@@ -272,6 +276,7 @@ jd_status upload_proj(jd_model *m, const std::vector<float> &h, int r0, int N, i
         // one TMA box per MMA: 192 rows for 384-wide tiles (two N=192 MMAs), else the tile width
         const uint32_t box_rows = bn == 384 ? 192 : (uint32_t)bn;
         TRY(make_map(&p.tm, d, K, N, K, 64, box_rows));
+        if (bn == 384) TRY(make_map(&p.tm64, d, K, N, K, 32, 192, false, true));
     }
     return JD_OK;
 }
@@ -409,6 +414,9 @@ jd_status alloc_workspace(jd_model *m) {
         TRY(make_map(&m->tm_o, m->o, D, T, D, 64, 128));
         TRY(make_map(&m->tm_y_enc, m->y, FF, T, FF, 64, 128));
         TRY(make_map(&m->tm_y_head, m->y, HFF, T, HFF, 64, 128));
+        TRY(make_map(&m->tm_o64, m->o, D, T, D, 32, 128, false, true));
+        TRY(make_map(&m->tm_y_enc64, m->y, FF, T, FF, 32, 128, false, true));
+        TRY(make_map(&m->tm_y_head64, m->y, HFF, T, HFF, 32, 128, false, true));
         TRY(make_map(&m->tm_qkv, m->qkv, QKV, T, QKV, 64, 64));
         TRY(make_map(&m->tm_xm, m->xm, D, M, D, 64, 128));
         TRY(make_map(&m->tm_om, m->om, D, M, D, 64, 128));
@@ -436,11 +444,14 @@ EpiParams base_ep(jd_model *m, int rows) {
 }
 
 GemmOp make_op(int epi, int bn, const ProjW &w, const CUtensorMap *tmA, const void *A, int lda, const EpiParams &ep,
-               const CUtensorMap *tmO = nullptr, const CUtensorMap *tmX = nullptr, const CUtensorMap *tmXN = nullptr) {
+               const CUtensorMap *tmO = nullptr, const CUtensorMap *tmX = nullptr, const CUtensorMap *tmXN = nullptr,
+               const CUtensorMap *tmA64 = nullptr) {
     GemmOp op;
     op.tmO = tmO;
     op.tmX = tmX;
     op.tmXN = tmXN;
+    op.tmA64 = tmA64;
+    op.tmB64 = tmA64 ? &w.tm64 : nullptr;
     op.epi = epi;
     op.bn = bn;
     op.K = w.K;
@@ -516,7 +527,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.ldo = D;
         e.resid = m->x;
         e.ln_g = m->mlp_g[l];
-        KL("gemm_wo_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo[l], &m->tm_o, m->o, D, e, nullptr, &m->tm_x32, &m->tm_xn), f32, st));
+        KL("gemm_wo_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo[l], &m->tm_o, m->o, D, e, nullptr, &m->tm_x32, &m->tm_xn, &m->tm_o64), f32, st));
 
         e = base_ep(m, T);
         e.out = m->y;
@@ -538,7 +549,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
             e.ln_g = m->n1g[0];
             e.ln_b = m->n1b[0];
         }
-        KL("gemm_wo2_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo2[l], &m->tm_y_enc, m->y, FF, e, nullptr, &m->tm_x32, &m->tm_xn), f32, st));
+        KL("gemm_wo2_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo2[l], &m->tm_y_enc, m->y, FF, e, nullptr, &m->tm_x32, &m->tm_xn, &m->tm_y_enc64), f32, st));
     }
 
     // ---- head layer 0 (all tokens)
@@ -557,7 +568,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.resid = m->x;
         e.ln_g = m->n2g[0];
         e.ln_b = m->n2b[0];
-        KL("head0_gemm_out", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->out_p[0], &m->tm_o, m->o, D, e, nullptr, &m->tm_x32, &m->tm_xn), f32, st));
+        KL("head0_gemm_out", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->out_p[0], &m->tm_o, m->o, D, e, nullptr, &m->tm_x32, &m->tm_xn, &m->tm_o64), f32, st));
         e = base_ep(m, T);
         e.out = m->y;
         e.ldo = HFF;
@@ -570,7 +581,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.resid = m->x;
         e.ln_g = m->n1g[1];
         e.ln_b = m->n1b[1];
-        KL("head0_gemm_ffn2", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[0], &m->tm_y_head, m->y, HFF, e, nullptr, &m->tm_x32, &m->tm_xn), f32, st));
+        KL("head0_gemm_ffn2", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[0], &m->tm_y_head, m->y, HFF, e, nullptr, &m->tm_x32, &m->tm_xn, &m->tm_y_head64), f32, st));
     }
     // ---- head layer 1: keys / values for every token, the rest at the markers only
     {
@@ -931,6 +942,7 @@ struct NoAllocSlot {
     bool ready = false;
     uint8_t *base = nullptr;  // device address of g_noalloc_scratch on this device
     CUtensorMap tm_xn{}, tm_o{}, tm_y_enc{}, tm_y_head{}, tm_qkv{}, tm_xm{}, tm_om{}, tm_xnm{}, tm_ym{};
+    CUtensorMap tm_o64{}, tm_y_enc64{}, tm_y_head64{};  // residual GEMM A operands: box 32 x 128, 64-byte swizzle
     CUtensorMap to_qkv{}, to_y_enc{}, to_y_head{}, to_qm{}, to_ym{};
     CUtensorMap tm_x32{};  // FP32 residual stream, box 32 x 128
     CUtensorMap tm_qkv128{};
@@ -953,6 +965,9 @@ jd_status noalloc_setup(int dev) {
     TRY(make_map(&s.tm_o, s.base + NA_O, D, NA_TOKENS, D, 64, 128));
     TRY(make_map(&s.tm_y_enc, s.base + NA_Y, FF, NA_TOKENS, FF, 64, 128));
     TRY(make_map(&s.tm_y_head, s.base + NA_Y, HFF, NA_TOKENS, HFF, 64, 128));
+    TRY(make_map(&s.tm_o64, s.base + NA_O, D, NA_TOKENS, D, 32, 128, false, true));
+    TRY(make_map(&s.tm_y_enc64, s.base + NA_Y, FF, NA_TOKENS, FF, 32, 128, false, true));
+    TRY(make_map(&s.tm_y_head64, s.base + NA_Y, HFF, NA_TOKENS, HFF, 32, 128, false, true));
     TRY(make_map(&s.tm_qkv, s.base + NA_QKV, QKV, NA_TOKENS, QKV, 64, 64));
     TRY(make_map(&s.tm_xm, s.base + NA_XM, D, NA_MARKERS, D, 64, 128));
     TRY(make_map(&s.tm_om, s.base + NA_OM, D, NA_MARKERS, D, 64, 128));
@@ -998,6 +1013,7 @@ void noalloc_view(jd_model &v, const jd_model *m, const NoAllocSlot &s) {
     v.xm = b + NA_XM; v.qm = b + NA_QM; v.om = b + NA_OM; v.xnm = b + NA_XNM; v.ym = b + NA_YM;
     v.status = reinterpret_cast<unsigned *>(b + NA_STATUS);
     v.tm_xn = s.tm_xn; v.tm_o = s.tm_o; v.tm_y_enc = s.tm_y_enc; v.tm_y_head = s.tm_y_head; v.tm_qkv = s.tm_qkv;
+    v.tm_o64 = s.tm_o64; v.tm_y_enc64 = s.tm_y_enc64; v.tm_y_head64 = s.tm_y_head64;
     v.tm_xm = s.tm_xm; v.tm_om = s.tm_om; v.tm_xnm = s.tm_xnm; v.tm_ym = s.tm_ym;
     v.to_qkv = s.to_qkv; v.to_y_enc = s.to_y_enc; v.to_y_head = s.to_y_head; v.to_qm = s.to_qm; v.to_ym = s.to_ym;
     v.tm_x32 = s.tm_x32;
