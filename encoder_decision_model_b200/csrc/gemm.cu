@@ -505,10 +505,10 @@ struct RlCfg {
     static_assert(NXB >= 2 && NXB <= 12 && SMEM <= 227 * 1024, "residual GEMM shared memory");
 };
 #ifndef JD_RL_STAGES
-#define JD_RL_STAGES 4
+#define JD_RL_STAGES 5
 #endif
 #ifndef JD_RL_NXB
-#define JD_RL_NXB 6
+#define JD_RL_NXB 4
 #endif
 constexpr int RL_STAGES = JD_RL_STAGES, RL_NXB = JD_RL_NXB;
 using RlCur = RlCfg<RL_STAGES, RL_NXB>;
