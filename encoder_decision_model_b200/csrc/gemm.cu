@@ -485,11 +485,12 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
 //             v = x + acc (+ bias) is written back in place, stored to x by
 //             TMA and parked in TMEM; row mean and M2 are merged chunk by
 //             chunk (Chan's pairwise update), so one pass yields the moments;
-//     pass 2  xn = LN(v) from TMEM, stored from registers (the shared memory
-//             goes to the operand ring and the residual buffers instead of
-//             output staging).
-// The residual stream is the HBM traffic of this kernel; with two buffers the
-// loads in flight per SM covered about half of the memory latency.
+//     pass 2  xn = LN(v) from TMEM, stored from registers with 32-byte stores
+//             (the shared memory goes to the operand ring and the residual
+//             buffers instead of output staging).
+// The residual stream is the HBM traffic of this kernel.  Measured splits of the
+// 224 KB between operand stages and residual buffers (32 KB / 16 KB each): five
+// stages and four buffers beat 4 + 6, 3 + 8 and 6 + 2.
 template <int STAGES_, int NXB_>
 struct RlCfg {
     static constexpr int A_BYTES = 128 * 64;   // 128 rows x 32 bf16
