@@ -40,7 +40,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--rows", type=int, default=1024, help="rows per rank and step")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="rows per rank and step (default 1024 for throughput, 16 for long)")
     ap.add_argument("--workload", default="throughput", choices=["throughput", "long"],
                     help="throughput: 1024 rows of 64..1024 tokens; long: 16 rows of 8192 tokens")
     ap.add_argument("--latency-calls", type=int, default=1000)
@@ -58,14 +59,15 @@ def parse():
 def workload(args, rank):
     from workloads import rows_config2, rows_config3
     if args.workload == "long":
-        rows = rows_config3(16, seed=103 + 1000 * rank)
+        n = args.rows or 16
+        rows = rows_config3(n, seed=103 + 1000 * rank)
         opts = dict(max_length=8192, head_budget=256, strict=False)
-        desc = ("long context: 16 rows x 8192 tokens, 20 options (capped to the 256-token head budget, "
+        desc = (f"long context: {n} rows x 8192 tokens, 20 options (capped to the 256-token head budget, "
                 "non-strict), choice/score")
     else:
-        rows = rows_config2(args.rows, seed=102 + 1000 * rank)
+        rows = rows_config2(args.rows or 1024, seed=102 + 1000 * rank)
         opts = dict(max_length=1024, head_budget=512, strict=True)
-        desc = (f"batched throughput: {args.rows} packed rows, lengths U[64,1024], 2..20 options of 1..48 ids, "
+        desc = (f"batched throughput: {args.rows or 1024} packed rows, lengths U[64,1024], 2..20 options of 1..48 ids, "
                 "types uniform, head budget 512, strict")
     return rows, opts, desc
 
