@@ -46,6 +46,8 @@ def parse():
                     help="throughput: 1024 rows of 64..1024 tokens; long: 16 rows of 8192 tokens")
     ap.add_argument("--latency-calls", type=int, default=1000)
     ap.add_argument("--router-reps", type=int, default=5, help="timed jd_route_host calls (0: skip)")
+    ap.add_argument("--serve-seconds", type=float, default=2.0,
+                    help="seconds per thread count of the concurrent-serving measurement (0: skip)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=3)
@@ -309,6 +311,58 @@ ROUTER_KERNELS = ("embed_ln", "attn_local", "attn_global", "head0_attn", "head1_
                   "scorer", "readout")
 
 
+def measure_serving(jl, wpath, local, seconds, thread_counts=(1, 2, 4)):
+    """Single 3-question requests (one 200-token state) served from 1, 2, 4 host
+    threads, each with its own handle (jd_model_create_shared: one copy of the
+    weights) and its own stream, CUDA-graph replay on; requests/s and latency."""
+    import threading
+    import torch
+    from workloads import rows_config1
+    r1 = rows_config1()
+    o1 = jl.encode_opts(1024, 512, True)
+    base = jl.Model(wpath, 2048, 8, 64, precision=jl.JD_PREC_BF16, device=local)
+    out = []
+    for n in thread_counts:
+        handles = [jl.Model.shared(base, 2048, 8, 64) for _ in range(n)]
+        lat = [[] for _ in range(n)]
+        start = threading.Barrier(n + 1)
+
+        def serve(k):
+            torch.cuda.set_device(local)
+            st = torch.cuda.Stream(device=local)
+            h = handles[k]
+            h.jd_set_graph_mode(True)
+            for _ in range(10):
+                h.jd_decide_host(r1, o1, stream=st)
+            start.wait()
+            t_end = time.perf_counter() + seconds
+            while True:
+                t = time.perf_counter()
+                if t >= t_end:
+                    break
+                h.jd_decide_host(r1, o1, stream=st)
+                lat[k].append(1000 * (time.perf_counter() - t))
+
+        ths = [threading.Thread(target=serve, args=(k,)) for k in range(n)]
+        for t in ths:
+            t.start()
+        start.wait()
+        t0 = time.perf_counter()
+        for t in ths:
+            t.join()
+        el = time.perf_counter() - t0
+        allv = np.concatenate([np.asarray(v) for v in lat])
+        out.append({"threads": n, "requests_per_s": float(len(allv) / el),
+                    "p50_ms_per_call": float(np.percentile(allv, 50)), "p99_ms_per_call": float(np.percentile(allv, 99))})
+        for h in handles:
+            h.jd_check_status()
+            h.close()
+    base.close()
+    return {"workload": "3 questions (choice/4, score/3, noul/2) on one 200-token state per request, "
+                        "each thread its own shared handle and stream, CUDA-graph replay, host work included",
+            "results": out}
+
+
 def measure_router(jl, wpath, local, rank, ranks, reps, peaks):
     """Router workload: 512 independent requests, each a 256-id state, a question
     and 72 labels; round 1 scores groups of <=20 labels (4 rows per request), the
@@ -490,6 +544,10 @@ def run_ours(args):
                                     "jd_decide_host with CUDA-graph replay, host serialisation and copies included")
         lm.close()
 
+    serving = None
+    if rank == 0 and args.serve_seconds > 0:
+        serving = measure_serving(jl, weights_path(0), local, args.serve_seconds)
+
     # ---- router: 512 requests x 72 labels, both rounds and the host work between them
     peaks = read_peaks()
     router = None
@@ -548,7 +606,7 @@ def run_ours(args):
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "call": "jd_decide_host (serialise + H2D from pinned staging + forward + D2H + sync)"},
             "gpu_launches": int(launches_per_step * args.steps),
-            "clocks": ck, "per_kernel": per_kernel, "router": router}
+            "clocks": ck, "per_kernel": per_kernel, "router": router, "concurrent_serving": serving}
     if rank == 0:
         s = json.dumps(line)
         print(s, flush=True)

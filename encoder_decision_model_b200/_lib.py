@@ -96,6 +96,7 @@ def lib():
     L.jd_batch_free.argtypes = [C.POINTER(jd_batch)]
     L.jd_batch_free.restype = None
     L.jd_model_create.argtypes = [C.POINTER(jd_model_config), C.c_char_p, C.c_int, C.POINTER(C.c_void_p)]
+    L.jd_model_create_shared.argtypes = [C.c_void_p, C.POINTER(jd_model_config), C.POINTER(C.c_void_p)]
     L.jd_model_destroy.argtypes = [C.c_void_p]
     L.jd_model_destroy.restype = None
     L.jd_model_device_bytes.argtypes = [C.c_void_p]
@@ -116,7 +117,7 @@ def lib():
     L.jd_last_launch_count.restype = C.c_int32
     L.jd_set_profiling.argtypes = [C.c_void_p, C.c_int]
     L.jd_profile_report.argtypes = [C.c_void_p, C.c_char_p, C.c_size_t]
-    for name in ("jd_serialize", "jd_model_create", "jd_decide", "jd_forward", "jd_decide_host",
+    for name in ("jd_serialize", "jd_model_create", "jd_model_create_shared", "jd_decide", "jd_forward", "jd_decide_host",
                  "jd_decide_packed_host", "jd_check_status", "jd_set_graph_mode", "jd_set_profiling",
                  "jd_profile_report"):
         getattr(L, name).restype = C.c_int
@@ -230,6 +231,19 @@ class Model:
         _check(L.jd_model_create(C.byref(cfg), str(weights_path).encode(), int(device), C.byref(h)))
         self.h = h
         self.cfg = cfg
+
+    @classmethod
+    def shared(cls, base, max_tokens, max_rows, max_markers, scorer=JD_SCORER_MLP, head_act=JD_ACT_RELU):
+        """jd_model_create_shared: a handle on base's weights with its own workspace
+        (for another stream / host thread); keeps base alive."""
+        self = cls.__new__(cls)
+        cfg = jd_model_config(int(max_tokens), int(max_rows), int(max_markers), base.cfg.precision, scorer, head_act)
+        h = C.c_void_p()
+        _check(lib().jd_model_create_shared(base.h, C.byref(cfg), C.byref(h)))
+        self.h = h
+        self.cfg = cfg
+        self.base = base
+        return self
 
     def close(self):
         if getattr(self, "h", None):

@@ -303,6 +303,23 @@ jd_status make_rope_table(jd_model *m, double theta, float4 **dst) {
     return JD_OK;
 }
 
+// Copy the weight pointers and their tensor maps of m into v (no device memory is allocated).
+void share_weights(jd_model &v, const jd_model *m) {
+    v.E = m->E; v.emb_g = m->emb_g; v.fin_g = m->fin_g; v.type_tab = m->type_tab;
+    for (int l = 0; l < NL; ++l) {
+        v.attn_g[l] = m->attn_g[l]; v.mlp_g[l] = m->mlp_g[l];
+        v.Wqkv[l] = m->Wqkv[l]; v.Wo[l] = m->Wo[l]; v.Wi[l] = m->Wi[l]; v.Wo2[l] = m->Wo2[l];
+    }
+    for (int i = 0; i < 2; ++i) {
+        v.n1g[i] = m->n1g[i]; v.n1b[i] = m->n1b[i]; v.n2g[i] = m->n2g[i]; v.n2b[i] = m->n2b[i];
+        v.in_full[i] = m->in_full[i]; v.in_q[i] = m->in_q[i]; v.in_kv[i] = m->in_kv[i];
+        v.out_p[i] = m->out_p[i]; v.lin1[i] = m->lin1[i]; v.lin2[i] = m->lin2[i];
+        v.in_b[i] = m->in_b[i]; v.out_b[i] = m->out_b[i]; v.l1_b[i] = m->l1_b[i]; v.l2_b[i] = m->l2_b[i];
+    }
+    v.sc_g = m->sc_g; v.sc_b = m->sc_b; v.sc_w1t = m->sc_w1t; v.sc_b1 = m->sc_b1; v.sc_w2 = m->sc_w2;
+    v.sc_b2 = m->sc_b2; v.lin_w = m->lin_w; v.lin_b = m->lin_b; v.rope_g = m->rope_g; v.rope_l = m->rope_l;
+}
+
 jd_status load_weights(jd_model *m, const char *path) {
     WeightFile wf;
     TRY(open_weights(path, wf));
@@ -714,6 +731,38 @@ extern "C" jd_status jd_model_create(const jd_model_config *cfg, const char *wei
     return JD_OK;
 }
 
+// A second handle on the weights of `base` (their device memory stays owned by base) with a
+// workspace, staging buffers and graph cache of its own ("Julia-1 MLX", "Performance": single
+// requests served from several threads, each on its own stream).
+extern "C" jd_status jd_model_create_shared(const jd_model *base, const jd_model_config *cfg, jd_model **out) {
+    clear_error();
+    if (!out || !cfg || !base) return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    *out = nullptr;
+    if (cfg->max_tokens < 1 || cfg->max_rows < 1 || cfg->max_markers < 1)
+        return fail(JD_ERR_INVALID_ARG, "capacities must be positive");
+    if (cfg->precision != base->cfg.precision) return fail(JD_ERR_INVALID_ARG, "precision differs from the base model's");
+    CK(cudaSetDevice(base->device));
+    jd_model *m = new jd_model();
+    m->cfg = *cfg;
+    m->device = base->device;
+    m->fp32 = base->fp32;
+    m->T_cap = (cfg->max_tokens + 127) / 128 * 128;
+    m->B_cap = cfg->max_rows;
+    m->M_cap = (cfg->max_markers + 127) / 128 * 128;
+    share_weights(*m, base);
+    jd_status s = alloc_workspace(m);
+    if (s == JD_OK) {
+        cudaError_t e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) s = fail(JD_ERR_CUDA, "setup: %s", cudaGetErrorString(e));
+    }
+    if (s != JD_OK) {
+        jd_model_destroy(m);
+        return s;
+    }
+    *out = m;
+    return JD_OK;
+}
+
 extern "C" void jd_model_destroy(jd_model *m) {
     if (!m) return;
     cudaSetDevice(m->device);
@@ -990,19 +1039,7 @@ void noalloc_view(jd_model &v, const jd_model *m, const NoAllocSlot &s) {
     v.cfg = m->cfg;
     v.device = m->device;
     v.fp32 = false;
-    v.E = m->E; v.emb_g = m->emb_g; v.fin_g = m->fin_g; v.type_tab = m->type_tab;
-    for (int l = 0; l < NL; ++l) {
-        v.attn_g[l] = m->attn_g[l]; v.mlp_g[l] = m->mlp_g[l];
-        v.Wqkv[l] = m->Wqkv[l]; v.Wo[l] = m->Wo[l]; v.Wi[l] = m->Wi[l]; v.Wo2[l] = m->Wo2[l];
-    }
-    for (int i = 0; i < 2; ++i) {
-        v.n1g[i] = m->n1g[i]; v.n1b[i] = m->n1b[i]; v.n2g[i] = m->n2g[i]; v.n2b[i] = m->n2b[i];
-        v.in_full[i] = m->in_full[i]; v.in_q[i] = m->in_q[i]; v.in_kv[i] = m->in_kv[i];
-        v.out_p[i] = m->out_p[i]; v.lin1[i] = m->lin1[i]; v.lin2[i] = m->lin2[i];
-        v.in_b[i] = m->in_b[i]; v.out_b[i] = m->out_b[i]; v.l1_b[i] = m->l1_b[i]; v.l2_b[i] = m->l2_b[i];
-    }
-    v.sc_g = m->sc_g; v.sc_b = m->sc_b; v.sc_w1t = m->sc_w1t; v.sc_b1 = m->sc_b1; v.sc_w2 = m->sc_w2;
-    v.sc_b2 = m->sc_b2; v.lin_w = m->lin_w; v.lin_b = m->lin_b; v.rope_g = m->rope_g; v.rope_l = m->rope_l;
+    share_weights(v, m);
     uint8_t *b = s.base;
     v.x = reinterpret_cast<float *>(b + NA_X);
     v.xn = b + NA_XN; v.qkv = b + NA_QKV; v.o = b + NA_O; v.y = b + NA_Y;

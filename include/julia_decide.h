@@ -164,7 +164,19 @@ jd_status jd_model_create(const jd_model_config *cfg, const char *weights_path, 
                           jd_model **out);
 void jd_model_destroy(jd_model *model);
 
-/* Device bytes held by the model (weights + workspace). */
+/* A second handle on the weights of `base` with a workspace, staging buffers and
+ * CUDA-graph cache of its own, sized by cfg (precision must equal base's; scorer
+ * and head_act are this handle's).  "Julia-1 MLX", "Performance": a server taking
+ * single requests scores them from several threads, each on its own stream; one
+ * handle per thread / stream gives that on one copy of the weights.  Calls on one
+ * handle must not overlap (they share its workspace); calls on different handles
+ * may run concurrently on different streams.  `base` owns the weights' device
+ * memory and must outlive every shared handle; jd_model_destroy(shared) frees only
+ * the handle's own memory.  Errors: JD_ERR_INVALID_ARG (NULL, capacities < 1,
+ * precision differs), JD_ERR_CUDA (allocation). */
+jd_status jd_model_create_shared(const jd_model *base, const jd_model_config *cfg, jd_model **out);
+
+/* Device bytes held by the model (weights + workspace; a shared handle counts its own memory only). */
 size_t jd_model_device_bytes(const jd_model *model);
 
 /* Full forward pass and read-outs on a packed batch in device memory.

@@ -143,3 +143,10 @@ def test_model_create_fails_loudly_without_gpu(L, weights_file):
 
 def test_version(L):
     assert "sm_100a" in jl.jd_version()
+
+
+def test_shared_handle_argument_checks(L):
+    cfg = jl.jd_model_config(1024, 8, 64, jl.JD_PREC_BF16, jl.JD_SCORER_MLP, jl.JD_ACT_RELU)
+    h = ctypes.c_void_p()
+    assert L.jd_model_create_shared(None, ctypes.byref(cfg), ctypes.byref(h)) == 1  # JD_ERR_INVALID_ARG
+    assert not h.value
