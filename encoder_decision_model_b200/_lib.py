@@ -158,21 +158,54 @@ def encode_opts(max_length=8192, head_budget=256, strict=True, bos=2, eos=1, mas
     return jd_encode_opts(max_length, head_budget, int(bool(strict)), bos, eos, mask, vocab)
 
 
+def _struct_dtype(ct):
+    """numpy dtype with the byte layout of ctypes structure `ct` (pointers as uint64)."""
+    names, formats, offsets = [], [], []
+    for name, typ in ct._fields_:
+        names.append(name)
+        formats.append(np.int32 if typ is C.c_int32 else np.uint64)
+        offsets.append(getattr(ct, name).offset)
+    return np.dtype({"names": names, "formats": formats, "offsets": offsets, "itemsize": C.sizeof(ct)})
+
+
+def _pack_lists(seqs):
+    """One int32 buffer for a list of id sequences: (flat, offsets, lengths)."""
+    lens = np.fromiter((len(x) for x in seqs), dtype=np.int64, count=len(seqs))
+    flat = np.concatenate([np.asarray(x, dtype=np.int32).ravel() for x in seqs]) if seqs else np.zeros(0, np.int32)
+    flat = np.ascontiguousarray(flat, dtype=np.int32)
+    offs = np.zeros(len(seqs), dtype=np.int64)
+    if len(seqs) > 1:
+        np.cumsum(lens[:-1], out=offs[1:])
+    return flat, offs, lens
+
+
 class _RowKeep:
-    """Holds the ctypes row array and the numpy buffers it points into."""
+    """The jd_row array of `rows` and the buffers it points into, built with
+    vectorised numpy (one buffer per field kind, not one object per option)."""
 
     def __init__(self, rows):
-        self.keep = []
-        self.arr = (jd_row * max(1, len(rows)))()
-        for i, r in enumerate(rows):
-            st = np.ascontiguousarray(r.state, dtype=np.int32)
-            q = np.ascontiguousarray(r.question, dtype=np.int32)
-            opts = [np.ascontiguousarray(o, dtype=np.int32) for o in r.options]
-            optp = (i32p * max(1, len(opts)))(*[o.ctypes.data_as(i32p) for o in opts])
-            lens = np.asarray([len(o) for o in opts] or [0], dtype=np.int32)
-            self.keep += [st, q, opts, optp, lens]
-            self.arr[i] = jd_row(st.ctypes.data_as(i32p), len(st), q.ctypes.data_as(i32p), len(q), optp,
-                                 lens.ctypes.data_as(i32p), len(opts), int(r.qtype))
+        n = len(rows)
+        st, st_off, st_len = _pack_lists([r.state for r in rows])
+        q, q_off, q_len = _pack_lists([r.question for r in rows])
+        k = np.fromiter((len(r.options) for r in rows), dtype=np.int64, count=n)
+        opt, o_off, o_len = _pack_lists([o for r in rows for o in r.options])
+        optp = (opt.ctypes.data + 4 * o_off).astype(np.uint64) if len(o_off) else np.zeros(1, np.uint64)
+        olen = o_len.astype(np.int32) if len(o_len) else np.zeros(1, np.int32)
+        first = np.zeros(n, dtype=np.int64)
+        if n > 1:
+            np.cumsum(k[:-1], out=first[1:])
+        arr = np.zeros(max(1, n), dtype=_struct_dtype(jd_row))
+        if n:
+            arr["state"][:n] = st.ctypes.data + 4 * st_off
+            arr["n_state"][:n] = st_len
+            arr["question"][:n] = q.ctypes.data + 4 * q_off
+            arr["n_question"][:n] = q_len
+            arr["options"][:n] = optp.ctypes.data + 8 * first
+            arr["n_option_ids"][:n] = olen.ctypes.data + 4 * first
+            arr["k"][:n] = k
+            arr["type"][:n] = np.fromiter((int(r.qtype) for r in rows), dtype=np.int32, count=n)
+        self.keep = (st, q, opt, optp, olen, arr)
+        self.arr = arr.ctypes.data_as(C.POINTER(jd_row))
 
 
 class HostBatch:
@@ -278,18 +311,27 @@ class Model:
                       stream=None):
         """Route requests (objects with state/question/labels); returns dict of
         winner, winner_p, final_candidates [n, 20], final_probs [n, 20], rows_per_round."""
-        keep = []
-        arr = (jd_route_request * max(1, len(requests)))()
-        for i, r in enumerate(requests):
-            st = np.ascontiguousarray(r.state, dtype=np.int32)
-            q = np.ascontiguousarray(r.question, dtype=np.int32)
-            labs = [np.ascontiguousarray(x, dtype=np.int32) for x in r.labels]
-            lp = (i32p * len(labs))(*[x.ctypes.data_as(i32p) for x in labs])
-            ln = np.asarray([len(x) for x in labs], dtype=np.int32)
-            keep += [st, q, labs, lp, ln]
-            arr[i] = jd_route_request(st.ctypes.data_as(i32p), len(st), q.ctypes.data_as(i32p), len(q), lp,
-                                      ln.ctypes.data_as(i32p), len(labs))
         n = len(requests)
+        st, st_off, st_len = _pack_lists([r.state for r in requests])
+        q, q_off, q_len = _pack_lists([r.question for r in requests])
+        nl = np.fromiter((len(r.labels) for r in requests), dtype=np.int64, count=n)
+        lab, l_off, l_len = _pack_lists([x for r in requests for x in r.labels])
+        labp = (lab.ctypes.data + 4 * l_off).astype(np.uint64) if len(l_off) else np.zeros(1, np.uint64)
+        llen = l_len.astype(np.int32) if len(l_len) else np.zeros(1, np.int32)
+        first = np.zeros(n, dtype=np.int64)
+        if n > 1:
+            np.cumsum(nl[:-1], out=first[1:])
+        req = np.zeros(max(1, n), dtype=_struct_dtype(jd_route_request))
+        if n:
+            req["state"][:n] = st.ctypes.data + 4 * st_off
+            req["n_state"][:n] = st_len
+            req["question"][:n] = q.ctypes.data + 4 * q_off
+            req["n_question"][:n] = q_len
+            req["labels"][:n] = labp.ctypes.data + 8 * first
+            req["n_label_ids"][:n] = llen.ctypes.data + 4 * first
+            req["n_labels"][:n] = nl
+        keep = (st, q, lab, labp, llen, req)
+        arr = req.ctypes.data_as(C.POINTER(jd_route_request))
         o = dict(winner=np.zeros(n, np.int32), winner_p=np.zeros(n, np.float32),
                  final_candidates=np.zeros((n, 20), np.int32), final_probs=np.zeros((n, 20), np.float32),
                  rows_per_round=np.zeros(16, np.int32))
