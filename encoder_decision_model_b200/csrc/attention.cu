@@ -486,15 +486,18 @@ cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st) {
 template <typename T>
 __global__ void __launch_bounds__(128)
     k_marker_attn(const T *__restrict__ qm, const T *__restrict__ qkv, T *__restrict__ om, const int *__restrict__ cu,
-                  const int *__restrict__ opt_off) {
+                  const int *__restrict__ opt_off, int nsplit, float *__restrict__ part) {
     __shared__ float Qs[32][DH];
     __shared__ float Ks[32][DH + 1];
     __shared__ float Vs[32][DH];
     __shared__ float S[32][32];
     __shared__ float Ms[32], Ls[32], Cs[32];
-    const int row = blockIdx.x, h = blockIdx.y;
+    const int row = blockIdx.x, h = blockIdx.y, sp = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int cs = cu[row], ce = cu[row + 1];
+    const int rs = cu[row], re = cu[row + 1];
+    // this CTA's share of the row's keys (split sp of nsplit, 32-key aligned)
+    const int chunk = ((re - rs + nsplit - 1) / nsplit + 31) / 32 * 32;
+    const int cs = min(re, rs + sp * chunk), ce = min(re, cs + chunk);
     const int mb = opt_off[row], me = opt_off[row + 1];
     const float sl2 = 0.125f * 1.4426950408889634f;
     for (int qc = mb; qc < me; qc += 32) {
@@ -563,24 +566,67 @@ __global__ void __launch_bounds__(128)
             const int e = tid + 128 * r;
             const int qi = e >> 6, d = e & 63;
             if (qi < nq) {
-                const float v = oacc[r] / Ls[qi];
-                om[(size_t)(qc + qi) * D + h * DH + d] = (T)v;
+                if (nsplit == 1) {
+                    om[(size_t)(qc + qi) * D + h * DH + d] = (T)(oacc[r] / Ls[qi]);
+                } else {  // partial result of this key split: running max (log2), sum, unnormalised o
+                    float *pe = part + ((size_t)((qc + qi) * NH + h) * nsplit + sp) * (DH + 2);
+                    if (d == 0) {
+                        pe[0] = Ms[qi];
+                        pe[1] = Ls[qi];
+                    }
+                    pe[2 + d] = oacc[r];
+                }
             }
         }
     }
 }
 
+// Merge the key splits of every (marker, head): o = sum_s 2^(m_s - m) o_s / sum_s 2^(m_s - m) l_s.
+template <typename T>
+__global__ void __launch_bounds__(64)
+    k_marker_combine(const float *__restrict__ part, int nsplit, T *__restrict__ om) {
+    const int mk = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+    const float *pe = part + (size_t)(mk * NH + h) * nsplit * (DH + 2);
+    float m = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) m = fmaxf(m, pe[s * (DH + 2)]);
+    float l = 0.f, o = 0.f;
+    for (int s = 0; s < nsplit; ++s) {
+        const float ms = pe[s * (DH + 2)];
+        const float w = ms == -INFINITY ? 0.f : exp2f(ms - m);
+        l = fmaf(pe[s * (DH + 2) + 1], w, l);
+        o = fmaf(pe[s * (DH + 2) + 2 + d], w, o);
+    }
+    om[(size_t)mk * D + h * DH + d] = (T)(o / l);
+}
+
+// One CTA per (row, head) leaves most SMs idle on long rows: split the keys, one
+// split per 1024 keys of the longest row (at most 8), within the scratch capacity.
+int marker_attention_splits(int n_markers, int max_row_len, const float *part, int part_entries) {
+    int nsplit = max_row_len > 1024 ? min(8, (max_row_len + 1023) / 1024) : 1;
+    if (!part || n_markers <= 0) return 1;
+    if (nsplit > 1 && (long)n_markers * nsplit > part_entries) nsplit = max(1, part_entries / n_markers);
+    return nsplit;
+}
+
 cudaError_t launch_marker_attention(const void *qm, const void *qkv, void *om, const int *cu_seqlens,
-                                    const int *opt_off, const int *mask_pos, int n_rows, bool fp32, cudaStream_t st) {
-    (void)mask_pos;
-    if (n_rows <= 0) return cudaSuccess;
-    dim3 grid(n_rows, NH);
+                                    const int *opt_off, int n_rows, int n_markers, int max_row_len, float *part,
+                                    int part_entries, bool fp32, cudaStream_t st) {
+    if (n_rows <= 0 || n_markers <= 0) return cudaSuccess;
+    const int nsplit = marker_attention_splits(n_markers, max_row_len, part, part_entries);
+    dim3 grid(n_rows, NH, nsplit);
     if (fp32)
         k_marker_attn<float><<<grid, 128, 0, st>>>((const float *)qm, (const float *)qkv, (float *)om, cu_seqlens,
-                                                   opt_off);
+                                                   opt_off, nsplit, part);
     else
         k_marker_attn<__nv_bfloat16><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)qm, (const __nv_bfloat16 *)qkv,
-                                                           (__nv_bfloat16 *)om, cu_seqlens, opt_off);
+                                                           (__nv_bfloat16 *)om, cu_seqlens, opt_off, nsplit, part);
+    if (nsplit > 1) {
+        dim3 g2(n_markers, NH);
+        if (fp32)
+            k_marker_combine<float><<<g2, DH, 0, st>>>(part, nsplit, (float *)om);
+        else
+            k_marker_combine<__nv_bfloat16><<<g2, DH, 0, st>>>(part, nsplit, (__nv_bfloat16 *)om);
+    }
     return cudaGetLastError();
 }
 

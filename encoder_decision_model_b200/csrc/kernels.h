@@ -66,8 +66,14 @@ cudaError_t launch_gather_markers(const int *mask_pos, int n_markers, int n_toke
 
 // Marker-only attention of the last head layer: the queries of each row's
 // markers qm [M, 384] against all keys / values of that row (qkv columns 384..).
+// Rows longer than 1024 keys split their keys over up to 8 CTAs per (row, head),
+// with partial results in `part` (part_entries x 6 heads x 66 floats; null: no split)
+// merged by a second kernel.
 cudaError_t launch_marker_attention(const void *qm, const void *qkv, void *om, const int *cu_seqlens,
-                                    const int *opt_off, const int *mask_pos, int n_rows, bool fp32, cudaStream_t st);
+                                    const int *opt_off, int n_rows, int n_markers, int max_row_len, float *part,
+                                    int part_entries, bool fp32, cudaStream_t st);
+constexpr int MARKER_PART_ENTRIES_MIN = 4096;  // scratch entries: max(marker capacity, this)
+int marker_attention_splits(int n_markers, int max_row_len, const float *part, int part_entries);
 
 // Scorer: logits[m] from the marker states hm [M, 384].
 struct ScorerArgs {

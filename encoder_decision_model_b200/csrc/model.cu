@@ -182,6 +182,8 @@ struct jd_model {
     void *xn = nullptr, *qkv = nullptr, *o = nullptr, *y = nullptr;
     int *tok_row = nullptr, *pos = nullptr, *qb_off = nullptr;
     float *hm = nullptr;
+    float *mk_part = nullptr;  // key-split partials of the marker attention
+    int mk_part_entries = 0;
     void *xm = nullptr, *qm = nullptr, *om = nullptr, *xnm = nullptr, *ym = nullptr;
     unsigned *status = nullptr;
     CUtensorMap tm_xn{}, tm_o{}, tm_y_enc{}, tm_y_head{}, tm_qkv{}, tm_xm{}, tm_om{}, tm_xnm{}, tm_ym{};
@@ -398,6 +400,8 @@ jd_status alloc_workspace(jd_model *m) {
     TRY(m->dalloc(&m->pos, T));
     TRY(m->dalloc(&m->qb_off, 2 * (B + 1) + T / 256 + B));
     TRY(m->dalloc(&m->hm, M * D));
+    m->mk_part_entries = std::max((int)M, MARKER_PART_ENTRIES_MIN);
+    TRY(m->dalloc(&m->mk_part, (size_t)m->mk_part_entries * NH * (DH + 2)));
     TRY(m->dalloc(&p, M * D * es)); m->xm = p;
     TRY(m->dalloc(&p, M * D * es)); m->qm = p;
     TRY(m->dalloc(&p, M * D * es)); m->om = p;
@@ -614,7 +618,9 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.ldo = D;
         e.bias = m->in_b[1];
         KL("head1_gemm_q", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_q[1], &m->tm_xm, m->xm, D, e, &m->to_qm), f32, st));
-        KL("head1_marker_attn", 1, launch_marker_attention(m->qm, m->qkv, m->om, b->cu_seqlens, b->opt_off, b->mask_pos, B, f32, st));
+        KL("head1_marker_attn", marker_attention_splits(M, b->max_row_len, m->mk_part, m->mk_part_entries) > 1 ? 2 : 1,
+           launch_marker_attention(m->qm, m->qkv, m->om, b->cu_seqlens, b->opt_off, B, M, b->max_row_len, m->mk_part,
+                                   m->mk_part_entries, f32, st));
         e = base_ep(m, M);
         e.out = m->xnm;
         e.ldo = D;
