@@ -581,6 +581,178 @@ __global__ void __launch_bounds__(128)
     }
 }
 
+// BF16 marker attention on the tensor cores (mma.sync m16n8k16): one CTA per (row, head,
+// key split), two warps of 16 marker queries each (a row has at most 20 markers, so one
+// 32-query pass; longer lists loop), Q by TMA from the marker-query buffer, 64-key K / V
+// tiles in a two-stage TMA ring, online softmax in registers.  The SIMT kernel above
+// spent two shared-memory loads per FMA on the dot products.
+constexpr int MQ = 32;  // marker queries per pass
+__global__ void __launch_bounds__(64)
+    k_marker_attn_mma(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tm,
+                      __nv_bfloat16 *__restrict__ om, const int *__restrict__ cu, const int *__restrict__ opt_off,
+                      int nsplit, float *__restrict__ part, unsigned *status) {
+    extern __shared__ uint8_t sm_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = sm;                                   // 32 x 64
+    uint8_t *sK[2] = {sm + 4096, sm + 4096 + 8192};     // 64 x 64 each
+    uint8_t *sV[2] = {sm + 4096 + 2 * 8192, sm + 4096 + 3 * 8192};
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + 4096 + 4 * 8192);  // 0: Q, 1..2: K/V stages
+
+    const int row = blockIdx.x, h = blockIdx.y, sp = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rs = cu[row], re = cu[row + 1];
+    const int chunk = ((re - rs + nsplit - 1) / nsplit + 31) / 32 * 32;
+    const int cs = min(re, rs + sp * chunk), ce = min(re, cs + chunk);
+    const int mb = opt_off[row], me = opt_off[row + 1];
+    const int ntiles = (ce - cs + BK - 1) / BK;
+    const float sl2 = 0.125f * 1.4426950408889634f;
+    const int g = lane >> 2, tq = lane & 3;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+    uint32_t qphase = 0, kvuse[2] = {0, 0};
+    for (int qc = mb; qc < me; qc += MQ) {
+        if (threadIdx.x == 0) {
+            mbar_arrive_expect_tx(&bars[0], MQ * 128);
+            tma_load_2d(sQ, &tmq, &bars[0], h * DH, qc);
+            for (int t = 0; t < 2 && t < ntiles; ++t) {
+                mbar_arrive_expect_tx(&bars[1 + t], 16384);
+                tma_load_2d(sK[t], &tm, &bars[1 + t], D + h * DH, cs + t * BK);
+                tma_load_2d(sV[t], &tm, &bars[1 + t], 2 * D + h * DH, cs + t * BK);
+            }
+        }
+        bool ok = mbar_wait(&bars[0], qphase & 1, status);
+        ++qphase;
+        uint32_t qf[4][4];
+        {
+            const uint32_t base = smem_u32(sQ);
+            const int r = warp * 16 + (lane & 15);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                ldsm_x4(base + sw128(r, kk * 2 + (lane >> 4)), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+        }
+        float o[8][4];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        for (int t = 0; t < ntiles; ++t) {
+            const int s = t & 1;
+            if (ok && !mbar_wait(&bars[1 + s], kvuse[s] & 1, status)) ok = false;
+            ++kvuse[s];
+            if (ok) {
+                const uint32_t kb = smem_u32(sK[s]), vb = smem_u32(sV[s]);
+                const int kt0 = cs + t * BK;
+                float sc[8][4];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+#pragma unroll
+                for (int np = 0; np < 4; ++np) {
+                    const int kr = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(kb + sw128(kr, kk * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
+                        mma_bf16(sc[2 * np], qf[kk], b0, b1);
+                        mma_bf16(sc[2 * np + 1], qf[kk], b2, b3);
+                    }
+                }
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const bool in = kt0 + j * 8 + 2 * tq + e < ce;  // keys of this split only
+                        sc[j][e] = in ? sc[j][e] * sl2 : -INFINITY;
+                        sc[j][2 + e] = in ? sc[j][2 + e] * sl2 : -INFINITY;
+                        mx0 = fmaxf(mx0, sc[j][e]);
+                        mx1 = fmaxf(mx1, sc[j][2 + e]);
+                    }
+                }
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0, mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
+                const float c0 = exp2f(m0 - mu0), c1 = exp2f(m1 - mu1);
+                m0 = mn0;
+                m1 = mn1;
+                float rs0 = 0.f, rs1 = 0.f;
+                uint32_t pa[4][4];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float p0 = exp2f(sc[j][0] - mu0), p1 = exp2f(sc[j][1] - mu0);
+                    const float p2 = exp2f(sc[j][2] - mu1), p3 = exp2f(sc[j][3] - mu1);
+                    rs0 += p0 + p1;
+                    rs1 += p2 + p3;
+                    pa[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p0, p1);
+                    pa[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+                }
+                l0 = l0 * c0 + rs0;
+                l1 = l1 * c1 + rs1;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    o[j][0] *= c0; o[j][1] *= c0;
+                    o[j][2] *= c1; o[j][3] *= c1;
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int vr = kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+                    for (int dp = 0; dp < 4; ++dp) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_t(vb + sw128(vr, dp * 2 + (lane >> 4)), b0, b1, b2, b3);
+                        mma_bf16(o[2 * dp], pa[kk], b0, b1);
+                        mma_bf16(o[2 * dp + 1], pa[kk], b2, b3);
+                    }
+                }
+            }
+            __syncthreads();  // both warps are done with stage s
+            if (threadIdx.x == 0 && t + 2 < ntiles) {
+                mbar_arrive_expect_tx(&bars[1 + s], 16384);
+                tma_load_2d(sK[s], &tm, &bars[1 + s], D + h * DH, cs + (t + 2) * BK);
+                tma_load_2d(sV[s], &tm, &bars[1 + s], 2 * D + h * DH, cs + (t + 2) * BK);
+            }
+        }
+        // kvuse[s] counts the completed phases of stage s across passes
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+        const int r0 = qc + warp * 16 + g, r1 = r0 + 8;  // marker indices of this thread's two rows
+        if (ok) {
+            if (nsplit == 1) {
+                const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int col = h * DH + j * 8 + 2 * tq;
+                    if (r0 < me)
+                        *reinterpret_cast<uint32_t *>(om + (size_t)r0 * D + col) = pack_bf16x2(o[j][0] * i0, o[j][1] * i0);
+                    if (r1 < me)
+                        *reinterpret_cast<uint32_t *>(om + (size_t)r1 * D + col) = pack_bf16x2(o[j][2] * i1, o[j][3] * i1);
+                }
+            } else {  // partials of this key split: running max (log2), sum, unnormalised o
+                float *p0 = part + ((size_t)(r0 * NH + h) * nsplit + sp) * (DH + 2);
+                float *p1 = part + ((size_t)(r1 * NH + h) * nsplit + sp) * (DH + 2);
+                if (r0 < me && tq == 0) { p0[0] = m0; p0[1] = l0; }
+                if (r1 < me && tq == 0) { p1[0] = m1; p1[1] = l1; }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int d = j * 8 + 2 * tq;
+                    if (r0 < me) { p0[2 + d] = o[j][0]; p0[3 + d] = o[j][1]; }
+                    if (r1 < me) { p1[2 + d] = o[j][2]; p1[3 + d] = o[j][3]; }
+                }
+            }
+        }
+        __syncthreads();  // sQ and the K / V stages are free for the next pass
+    }
+}
+constexpr int MARKER_MMA_SMEM = 4096 + 4 * 8192 + 64 + 1024;
+
 // Merge the key splits of every (marker, head): o = sum_s 2^(m_s - m) o_s / sum_s 2^(m_s - m) l_s.
 template <typename T>
 __global__ void __launch_bounds__(64)
@@ -610,13 +782,17 @@ int marker_attention_splits(int n_markers, int max_row_len, const float *part, i
 
 cudaError_t launch_marker_attention(const void *qm, const void *qkv, void *om, const int *cu_seqlens,
                                     const int *opt_off, int n_rows, int n_markers, int max_row_len, float *part,
-                                    int part_entries, bool fp32, cudaStream_t st) {
+                                    int part_entries, bool fp32, const CUtensorMap *tm_q, const CUtensorMap *tm_kv,
+                                    unsigned *status, cudaStream_t st) {
     if (n_rows <= 0 || n_markers <= 0) return cudaSuccess;
     const int nsplit = marker_attention_splits(n_markers, max_row_len, part, part_entries);
     dim3 grid(n_rows, NH, nsplit);
     if (fp32)
         k_marker_attn<float><<<grid, 128, 0, st>>>((const float *)qm, (const float *)qkv, (float *)om, cu_seqlens,
                                                    opt_off, nsplit, part);
+    else if (tm_q && tm_kv)
+        k_marker_attn_mma<<<grid, 64, MARKER_MMA_SMEM, st>>>(*tm_q, *tm_kv, (__nv_bfloat16 *)om, cu_seqlens, opt_off,
+                                                             nsplit, part, status);
     else
         k_marker_attn<__nv_bfloat16><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)qm, (const __nv_bfloat16 *)qkv,
                                                            (__nv_bfloat16 *)om, cu_seqlens, opt_off, nsplit, part);

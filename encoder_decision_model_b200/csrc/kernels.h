@@ -69,9 +69,12 @@ cudaError_t launch_gather_markers(const int *mask_pos, int n_markers, int n_toke
 // Rows longer than 1024 keys split their keys over up to 8 CTAs per (row, head),
 // with partial results in `part` (part_entries x 6 heads x 66 floats; null: no split)
 // merged by a second kernel.
+// BF16 with both maps (tm_q: marker queries, box 64 x 32; tm_kv: q|k|v, box 64 x 64) runs on
+// the tensor cores (mma.sync); otherwise a SIMT kernel.
 cudaError_t launch_marker_attention(const void *qm, const void *qkv, void *om, const int *cu_seqlens,
                                     const int *opt_off, int n_rows, int n_markers, int max_row_len, float *part,
-                                    int part_entries, bool fp32, cudaStream_t st);
+                                    int part_entries, bool fp32, const CUtensorMap *tm_q, const CUtensorMap *tm_kv,
+                                    unsigned *status, cudaStream_t st);
 constexpr int MARKER_PART_ENTRIES_MIN = 4096;  // scratch entries: max(marker capacity, this)
 int marker_attention_splits(int n_markers, int max_row_len, const float *part, int part_entries);
 

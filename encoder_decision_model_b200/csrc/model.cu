@@ -620,7 +620,8 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         KL("head1_gemm_q", 1, launch_gemm(make_op(EPI_QKV, 384, m->in_q[1], &m->tm_xm, m->xm, D, e, &m->to_qm), f32, st));
         KL("head1_marker_attn", marker_attention_splits(M, b->max_row_len, m->mk_part, m->mk_part_entries) > 1 ? 2 : 1,
            launch_marker_attention(m->qm, m->qkv, m->om, b->cu_seqlens, b->opt_off, B, M, b->max_row_len, m->mk_part,
-                                   m->mk_part_entries, f32, st));
+                                   m->mk_part_entries, f32, f32 ? nullptr : &m->to_qm, f32 ? nullptr : &m->tm_qkv,
+                                   m->status, st));
         e = base_ep(m, M);
         e.out = m->xnm;
         e.ldo = D;
