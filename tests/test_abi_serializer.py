@@ -150,3 +150,21 @@ def test_shared_handle_argument_checks(L):
     h = ctypes.c_void_p()
     assert L.jd_model_create_shared(None, ctypes.byref(cfg), ctypes.byref(h)) == 1  # JD_ERR_INVALID_ARG
     assert not h.value
+
+
+def test_marshalled_struct_layouts_match_ctypes():
+    """The vectorised marshalling writes jd_row / jd_route_request records with numpy;
+    their layout must be the C structures' (field offsets and size as ctypes lays them out)."""
+    for ct in (jl.jd_row, jl.jd_route_request):
+        dt = jl._struct_dtype(ct)
+        assert dt.itemsize == ctypes.sizeof(ct)
+        for name, typ in ct._fields_:
+            assert dt.fields[name][1] == getattr(ct, name).offset, (ct.__name__, name)
+            assert dt.fields[name][0].itemsize == ctypes.sizeof(typ), (ct.__name__, name)
+    # a record written through numpy reads back field by field through ctypes
+    rows = [Row(state=np.arange(5, 12), question=np.arange(20, 23), options=[np.arange(30, 34), np.arange(40, 42)], qtype=2)]
+    keep = jl._RowKeep(rows)
+    r = keep.arr[0]
+    assert (r.n_state, r.n_question, r.k, r.type) == (7, 3, 2, 2)
+    assert [r.state[i] for i in range(7)] == list(range(5, 12))
+    assert [r.options[1][i] for i in range(r.n_option_ids[1])] == [40, 41]
