@@ -239,26 +239,34 @@ __global__ void __launch_bounds__(128)
 // i.e. nine 16-key chunks, so each warp visits just those and runs an exact
 // two-pass softmax over them in registers (no running rescale).
 constexpr int LW_CHUNKS = 9;  // (16 + 2 * 64) / 16
+// Two heads per CTA (8 warps, 2 CTAs per SM): 16 resident warps per SM instead of 12.
+constexpr int LOC_HEADS = 2;
+constexpr int LOC_HEAD_BYTES = 7 * 8192;  // Q tile, 3 K tiles, 3 V tiles
+// The barriers sit in front of the 1024-byte aligned tiles, inside the alignment slack, so two
+// CTAs fit one SM's 228 KB with the 1 KB each CTA reserves.
+constexpr int LOC_SMEM = LOC_HEADS * LOC_HEAD_BYTES + 1024;
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128 * LOC_HEADS, 2)
     k_attn_local_bf16(const __grid_constant__ CUtensorMap tm, __nv_bfloat16 *__restrict__ out,
                       const int *__restrict__ cu, const int *__restrict__ qb_off, int n_rows, unsigned *status) {
-    extern __shared__ uint8_t sm_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQ = sm;                  // 64 x 64
-    uint8_t *sK = sm + 8192;           // 3 tiles of 64 x 64
-    uint8_t *sV = sm + 4 * 8192;       // 3 tiles
-    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 7 * 8192);
+    extern __shared__ __align__(16) uint8_t sm_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 8 * LOC_HEADS + 1023) &
+                                              ~uintptr_t(1023));
+    const int hh = (threadIdx.x >> 5) >> 2;  // head slot of this warp's group of four
+    uint8_t *sQ = sm + hh * LOC_HEAD_BYTES;  // 64 x 64
+    uint8_t *sK = sQ + 8192;                 // 3 tiles of 64 x 64
+    uint8_t *sV = sQ + 4 * 8192;             // 3 tiles
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm_raw) + hh;
 
-    const int tile = blockIdx.x, h = blockIdx.y;
+    const int tile = blockIdx.x, h = blockIdx.y * LOC_HEADS + hh;
     if (tile >= qb_off[n_rows]) return;
     const int row = find_row(qb_off, n_rows, tile);
     const int cs = cu[row], ce = cu[row + 1];
     const int q0 = cs + (tile - qb_off[row]) * BQ;
     const int kbase = q0 - 64;         // band start (may precede the row: masked)
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;  // warp inside the head's group
 
-    if (threadIdx.x == 0) {
+    if ((threadIdx.x & 127) == 0) {
         mbar_init(bar, 1);
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -441,8 +449,10 @@ __global__ void __launch_bounds__(256)
 cudaError_t attn_tc_init_attributes();
 
 cudaError_t attn_init_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(k_attn_local_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         7 * 8192 + 64 + 1024);
+    cudaError_t e = cudaFuncSetAttribute(k_attn_local_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, LOC_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_attn_local_bf16, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     return attn_tc_init_attributes();
 }
@@ -466,8 +476,8 @@ cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st) {
     } else {
         const int smem = 5 * 8192 + 64 + 1024;
         if (local && a.window == 64)
-            k_attn_local_bf16<<<grid, 128, 7 * 8192 + 64 + 1024, st>>>(*a.tm_qkv, (__nv_bfloat16 *)a.o, a.cu_seqlens,
-                                                                       a.qb_off, a.n_rows, a.status);
+            k_attn_local_bf16<<<dim3(max_tiles, NH / LOC_HEADS), 128 * LOC_HEADS, LOC_SMEM, st>>>(
+                *a.tm_qkv, (__nv_bfloat16 *)a.o, a.cu_seqlens, a.qb_off, a.n_rows, a.status);
         else if (local)
             k_attn_bf16<true><<<grid, 128, smem, st>>>(*a.tm_qkv, (__nv_bfloat16 *)a.o, a.cu_seqlens, a.qb_off,
                                                        a.n_rows, a.window, a.status);
