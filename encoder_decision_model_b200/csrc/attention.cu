@@ -37,6 +37,13 @@ __device__ __forceinline__ int find_row(const int *qb_off, int n_rows, int tile)
 
 // ------------------------------------------------------------------ mma.sync helpers
 
+// 2^x by the special-function unit (ex2.approx.ftz: results below 2^-126 flush to 0, 2^-inf = 0)
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
@@ -308,16 +315,21 @@ __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
             mma_bf16(sc[2 * cc + 1], qf[kk], b2, b3);
         }
     }
+    // Masks on the raw scores; the scale goes into the exponent's FMA below.  Key kj of 8-column
+    // block j lies kj - qi = 8j - 64 + (2tq + e) - g (- 8 for qi1) from the query, which is inside
+    // [-63, 63] for 2 <= j < 16: only the two outer chunks at each end need the window test.
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
+        const bool edge = j < 2 || j >= 2 * LW_CHUNKS - 2;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int kj = kbase + (warp * 2 + j) * 8 + 2 * tq + e;
             const bool in_row = kj >= cs && kj < ce;
-            const bool v0 = in_row && abs(qi0 - kj) <= 64, v1 = in_row && abs(qi1 - kj) <= 64;
-            sc[j][e] = v0 ? sc[j][e] * sl2 : -INFINITY;
-            sc[j][2 + e] = v1 ? sc[j][2 + e] * sl2 : -INFINITY;
+            const bool v0 = in_row && (!edge || abs(qi0 - kj) <= 64);
+            const bool v1 = in_row && (!edge || abs(qi1 - kj) <= 64);
+            sc[j][e] = v0 ? sc[j][e] : -INFINITY;
+            sc[j][2 + e] = v1 ? sc[j][2 + e] : -INFINITY;
             mx0 = fmaxf(mx0, sc[j][e]);
             mx1 = fmaxf(mx1, sc[j][2 + e]);
         }
@@ -326,13 +338,13 @@ __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mu0 = mx0 == -INFINITY ? 0.f : mx0, mu1 = mx1 == -INFINITY ? 0.f : mx1;
+    const float mu0 = mx0 == -INFINITY ? 0.f : -mx0 * sl2, mu1 = mx1 == -INFINITY ? 0.f : -mx1 * sl2;
     float l0 = 0.f, l1 = 0.f;
     uint32_t pa[LW_CHUNKS][4];
 #pragma unroll
     for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
-        const float p0 = exp2f(sc[j][0] - mu0), p1 = exp2f(sc[j][1] - mu0);
-        const float p2 = exp2f(sc[j][2] - mu1), p3 = exp2f(sc[j][3] - mu1);
+        const float p0 = ex2_ftz(fmaf(sc[j][0], sl2, mu0)), p1 = ex2_ftz(fmaf(sc[j][1], sl2, mu0));
+        const float p2 = ex2_ftz(fmaf(sc[j][2], sl2, mu1)), p3 = ex2_ftz(fmaf(sc[j][3], sl2, mu1));
         l0 += p0 + p1;
         l1 += p2 + p3;
         pa[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p0, p1);
