@@ -55,7 +55,7 @@ def oracle_run(path, rows, opts, scorer="mlp", head_act="relu", row_ids=None):
 
 
 def compare(hb, res, ref, bf16, check_taps=True, label=""):
-    """Assert the benchmark spec's tolerances row by row; returns summary stats."""
+    """Assert the parity tolerances row by row; returns summary stats."""
     from oracle import readouts
 
     worst = dict(logit=0.0, prob=0.0, enc_rel=0.0, hm_rel=0.0, argmax_checked=0, spread=0.0)
