@@ -262,14 +262,31 @@ def oracle_sample(rows, opts, seconds, min_rows=2):
 
 
 def blas_threads():
+    """Threads of the BLAS that runs NumPy's matmuls (the oracle's); other BLAS
+    copies loaded by other packages do not run the oracle."""
     try:
         from threadpoolctl import threadpool_info
-        th = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if th:
-            return int(max(th))
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        own = [i for i in info if "numpy" in (i.get("filepath") or "")] or info
+        if own:
+            return int(max(i.get("num_threads", 0) for i in own))
     except Exception:
         pass
     return os.cpu_count()
+
+
+def oracle_four_threads(rows, opts, seconds):
+    """The same oracle sample with BLAS held to 4 threads (the CPU runtimes on the
+    pages quote 4-thread figures); None when threadpoolctl is missing."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return None
+    with threadpool_limits(limits=4, user_api="blas"):
+        n, toks, el = oracle_sample(rows, opts, seconds)
+        cores = blas_threads()
+    return {"value": n / el, "unit": UNIT, "cores": cores,
+            "sample": f"first {n} rows ({toks} tokens), {el:.1f} s"}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -462,6 +479,7 @@ def run_ours(args):
         n, toks, el = oracle_sample(rows, opts, args.cpu_seconds)
         cpu = {"value": n / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": f"first {n} rows ({toks} tokens) of this workload, float64 NumPy oracle, {el:.1f} s"}
+        cpu["threads_4"] = oracle_four_threads(rows, opts, args.cpu_seconds)
 
     model = jl.Model(weights_path(0), T, B, M, precision=jl.JD_PREC_BF16, device=local)
     up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
