@@ -126,10 +126,14 @@ def read_peaks():
 
 
 def kernel_source_sha():
+    """SHA-256 (first 16 hex digits) of the sources that decide what the GPU runs:
+    the kernels and their launch code (*.cu, *.cuh) and their shared declarations
+    (kernels.h).  The host-only serializer, router and API files are not part of
+    it: they launch nothing."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "encoder_decision_model_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+        if f.endswith((".cu", ".cuh")) or f == "kernels.h":
             h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 

@@ -87,6 +87,8 @@ extern "C" jd_status jd_route_host(jd_model *m, const jd_route_request *reqs, in
     jd::clear_error();
     if (!m || !opts || !out || (n_requests > 0 && !reqs) || n_requests < 0)
         return jd::fail(JD_ERR_INVALID_ARG, "NULL argument");
+    if (n_requests > 0 && !out->winner) return jd::fail(JD_ERR_INVALID_ARG, "out->winner is NULL");
+    if (out->rows_per_round && out->max_rounds < 0) return jd::fail(JD_ERR_INVALID_ARG, "max_rounds < 0");
     if (max_tokens < 1 || max_rows < 1 || max_markers < kGroup)
         return jd::fail(JD_ERR_INVALID_ARG, "chunk capacities too small");
     for (int r = 0; r < n_requests; ++r)

@@ -140,6 +140,9 @@ extern "C" jd_status jd_serialize(const jd_row *rows, int32_t n_rows, const jd_e
     if (!opts || (n_rows > 0 && !rows) || n_rows < 0) return jd::fail(JD_ERR_INVALID_ARG, "rows/opts invalid");
     if (opts->max_length < 1 || opts->max_length > kMaxLength || opts->head_budget < 1 || opts->vocab < 1)
         return jd::fail(JD_ERR_INVALID_ARG, "max_length must be in [1, 8192] and head_budget >= 1");
+    const int32_t special[3] = {opts->bos, opts->eos, opts->mask};
+    if (!ids_in_range(special, 3, opts->vocab))
+        return jd::fail(JD_ERR_TOKEN_RANGE, "bos/eos/mask id outside [0, %d)", opts->vocab);
 
     std::vector<RowPlan> plans(n_rows);
     long T = 0, M = 0;
@@ -158,6 +161,7 @@ extern "C" jd_status jd_serialize(const jd_row *rows, int32_t n_rows, const jd_e
     if (T > 0x7fffffffL) return jd::fail(JD_ERR_INVALID_ARG, "batch too large");
 
     jd_batch *b = xalloc<jd_batch>(1);
+    if (!b) return jd::fail(JD_ERR_INVALID_ARG, "host allocation failed");
     std::memset(b, 0, sizeof(*b));
     b->n_rows = n_rows;
     b->n_tokens = (int32_t)T;
@@ -184,17 +188,17 @@ extern "C" jd_status jd_serialize(const jd_row *rows, int32_t n_rows, const jd_e
         const RowPlan &pl = plans[r];
         int32_t start = pos;
         t[pos++] = opts->bos;
-        std::memcpy(t + pos, row.question, sizeof(int32_t) * pl.nq);
+        if (pl.nq) std::memcpy(t + pos, row.question, sizeof(int32_t) * pl.nq);
         pos += pl.nq;
         t[pos++] = opts->eos;
         for (int k = 0; k < row.k; ++k) {
             b->mask_pos[m++] = pos;
             t[pos++] = opts->mask;
-            std::memcpy(t + pos, row.options[k], sizeof(int32_t) * pl.olen[k]);
+            if (pl.olen[k]) std::memcpy(t + pos, row.options[k], sizeof(int32_t) * pl.olen[k]);
             pos += pl.olen[k];
         }
         t[pos++] = opts->eos;
-        std::memcpy(t + pos, row.state, sizeof(int32_t) * pl.ns);
+        if (pl.ns) std::memcpy(t + pos, row.state, sizeof(int32_t) * pl.ns);
         pos += pl.ns;
         t[pos++] = opts->eos;
         b->cu_seqlens[r + 1] = pos;

@@ -82,7 +82,7 @@ typedef struct {
     int32_t max_length;   /* 1..8192 */
     int32_t head_budget;  /* >= 1; tokens before the state */
     int32_t strict;       /* nonzero: raise JD_ERR_OVERFLOW instead of truncating */
-    int32_t bos, eos, mask;
+    int32_t bos, eos, mask;  /* special ids, in [0, vocab) like every other id */
     int32_t vocab;        /* ids must lie in [0, vocab) */
 } jd_encode_opts;
 
@@ -146,7 +146,9 @@ const char *jd_version(void);
 /* Serialize rows into a packed host batch ("From a state to one decision").
  * Layout per row: <bos> question <eos> (<mask> option)_k <eos> state <eos>.
  * Always errors: K outside [2,20] or noul with K != 2 (JD_ERR_OPTION_COUNT),
- * an id outside [0, vocab) (JD_ERR_TOKEN_RANGE).  Strict: an option over 48
+ * an id outside [0, vocab), the special ids included (JD_ERR_TOKEN_RANGE).
+ * Invalid opts (max_length, head_budget, vocab) -> JD_ERR_INVALID_ARG; opts
+ * errors leave *bad_row at -1.  Strict: an option over 48
  * ids, head over budget or total over max_length -> JD_ERR_OVERFLOW.
  * Non-strict: clip options to 48 ids; if the head is over budget cap every
  * option at the largest common length that fits (clip the question from its
@@ -220,12 +222,12 @@ typedef struct {
 
 /* Router outputs (host memory, caller-owned; optional arrays may be NULL). */
 typedef struct {
-    int32_t *winner;            /* [n_requests] index of the chosen label */
-    float *winner_p;            /* [n_requests] its probability in the final call (1 if unscored) */
+    int32_t *winner;            /* required [n_requests] index of the chosen label (NULL: JD_ERR_INVALID_ARG) */
+    float *winner_p;            /* optional [n_requests] its probability in the final call (1 if unscored) */
     int32_t *final_candidates;  /* optional [n_requests * 20] label indices of the final call, -1 padded */
     float *final_probs;         /* optional [n_requests * 20] their probabilities */
     int32_t *rows_per_round;    /* optional [max_rounds] rows scored per round, all requests together */
-    int32_t max_rounds;
+    int32_t max_rounds;         /* >= 0 when rows_per_round is set; rounds beyond it are not recorded */
     int32_t n_rounds;           /* written: rounds including the final call */
 } jd_route_outputs;
 

@@ -87,6 +87,7 @@ def _check_ids(arr, vocab, what):
 def serialize_row(row, opt: EncodeOptions) -> Encoded:
     if not (1 <= opt.max_length <= MAX_LENGTH_LIMIT) or opt.head_budget < 1:
         raise EncodingError(ERR_INVALID_ARG, "max_length must be in [1, 8192] and head_budget >= 1")
+    _check_ids([opt.bos, opt.eos, opt.mask], opt.vocab, "bos/eos/mask")
     if row.qtype not in (0, 1, 2):
         raise EncodingError(ERR_INVALID_ARG, "type must be choice (0), score (1) or noul (2)")
     k = len(row.options)

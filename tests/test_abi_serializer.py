@@ -168,3 +168,70 @@ def test_marshalled_struct_layouts_match_ctypes():
     assert (r.n_state, r.n_question, r.k, r.type) == (7, 3, 2, 2)
     assert [r.state[i] for i in range(7)] == list(range(5, 12))
     assert [r.options[1][i] for i in range(r.n_option_ids[1])] == [40, 41]
+
+
+@pytest.mark.parametrize("field", ["bos", "eos", "mask"])
+@pytest.mark.parametrize("value", [-1, 256000])
+def test_special_ids_out_of_range(L, field, value):
+    """A special id outside [0, vocab) is rejected like any other id, by the C
+    serializer and the oracle alike; it is an options error, so no row is blamed."""
+    rows = rows_config1()
+    kw = dict(bos=2, eos=1, mask=4)
+    kw[field] = value
+    with pytest.raises(EncodingError) as eo:
+        serialize_row(rows[0], EncodeOptions(max_length=1024, head_budget=512, strict=True, **kw))
+    with pytest.raises(jl.JDError) as ei:
+        jl.jd_serialize(rows, jl.encode_opts(1024, 512, True, **kw))
+    assert ei.value.code == eo.value.code == jl.JD_ERR_TOKEN_RANGE
+    assert ei.value.bad_row == -1
+
+
+def test_null_arrays_with_zero_lengths(L):
+    """Empty question, state and option arrays may be passed as NULL pointers."""
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    opt0 = np.array([11, 12, 13], np.int32)
+    optp = (i32p * 2)(opt0.ctypes.data_as(i32p), i32p())
+    optn = (ctypes.c_int32 * 2)(3, 0)
+    row = jl.jd_row()
+    row.state, row.n_state = None, 0
+    row.question, row.n_question = None, 0
+    row.options = ctypes.cast(optp, type(row.options))
+    row.n_option_ids = ctypes.cast(optn, type(row.n_option_ids))
+    row.k, row.type = 2, 0
+    out = ctypes.POINTER(jl.jd_batch)()
+    bad = ctypes.c_int32(-1)
+    opts = jl.encode_opts(64, 64, True)
+    assert L.jd_serialize(ctypes.byref(row), 1, ctypes.byref(opts), ctypes.byref(out), ctypes.byref(bad)) == 0
+    b = out.contents
+    toks = np.ctypeslib.as_array(ctypes.cast(b.tokens, i32p), shape=(b.n_tokens,)).copy()
+    mp = np.ctypeslib.as_array(ctypes.cast(b.mask_pos, i32p), shape=(b.n_markers,)).copy()
+    L.jd_batch_free(out)
+    enc = serialize_row(Row(state=np.zeros(0, np.int32), question=np.zeros(0, np.int32),
+                            options=[opt0, np.zeros(0, np.int32)], qtype=0),
+                        EncodeOptions(max_length=64, head_budget=64, strict=True))
+    np.testing.assert_array_equal(toks, enc.ids)
+    np.testing.assert_array_equal(mp, enc.mask_pos)
+
+
+def test_route_requires_winner_output(L):
+    """jd_route_host checks its arguments before it touches the model: a NULL
+    winner array is JD_ERR_INVALID_ARG (the handle here is a dummy host buffer
+    that the call never reaches)."""
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    lab = np.array([10, 11], np.int32)
+    labp = (i32p * 3)(*([lab.ctypes.data_as(i32p)] * 3))
+    labn = (ctypes.c_int32 * 3)(2, 2, 2)
+    st = np.arange(10, 20, dtype=np.int32)
+    req = jl.jd_route_request()
+    req.state, req.n_state = st.ctypes.data_as(i32p), len(st)
+    req.question, req.n_question = None, 0
+    req.labels = ctypes.cast(labp, type(req.labels))
+    req.n_label_ids = ctypes.cast(labn, type(req.n_label_ids))
+    req.n_labels = 3
+    out = jl.jd_route_outputs()
+    dummy = ctypes.create_string_buffer(64)
+    opts = jl.encode_opts(1024, 512, True)
+    code = L.jd_route_host(ctypes.cast(dummy, ctypes.c_void_p), ctypes.byref(req), 1, ctypes.byref(opts),
+                           4096, 16, 64, ctypes.byref(out), None)
+    assert code == jl.JD_ERR_INVALID_ARG
+    assert "winner" in L.jd_last_error().decode()
