@@ -160,8 +160,17 @@ jd_status jd_serialize(const jd_row *rows, int32_t n_rows, const jd_encode_opts 
 void jd_batch_free(jd_batch *batch);
 
 /* Load the .jdw weights file and allocate the device workspace for the given
- * capacity on `device`.  BF16 copies of the projection weights are made here;
- * the embedding table, norms, biases and head stay FP32. */
+ * capacity on `device` (the architecture of "The decision head" and "Julia-1
+ * MLX", "Performance": 22 encoder layers of width 384, a 3 x 384 type table,
+ * two head layers, the scorer).  BF16 copies of the projection weights are
+ * made here; the embedding table, norms, biases and head stay FP32.  On
+ * success *out is a handle the caller owns and releases with
+ * jd_model_destroy (NULL is accepted there); on failure *out is NULL.
+ * Errors: JD_ERR_INVALID_ARG (NULL argument, a capacity < 1, unknown
+ * precision, device index out of range), JD_ERR_CUDA (no CUDA device, a
+ * device other than sm_100, an allocation or copy failed), JD_ERR_IO (the
+ * weights file is missing, truncated, or lacks a tensor of the expected
+ * shape). */
 jd_status jd_model_create(const jd_model_config *cfg, const char *weights_path, int device,
                           jd_model **out);
 void jd_model_destroy(jd_model *model);
@@ -181,15 +190,25 @@ jd_status jd_model_create_shared(const jd_model *base, const jd_model_config *cf
 /* Device bytes held by the model (weights + workspace; a shared handle counts its own memory only). */
 size_t jd_model_device_bytes(const jd_model *model);
 
-/* Full forward pass and read-outs on a packed batch in device memory.
- * `batch` is a host struct whose array pointers are device pointers (tokens,
- * cu_seqlens, mask_pos, opt_off, row_type; head_len / trunc are ignored).
- * n_tokens, n_rows, n_markers must not exceed the model's capacity
- * (JD_ERR_CAPACITY).  All outputs of `out` are written; `taps` may be NULL. */
+/* Full forward pass and read-outs on a packed batch in device memory ("The
+ * decision head", steps 1-4: encoder, type row, two head layers, one scorer
+ * logit per <mask> marker; "Three modes through one head": the per-question
+ * softmax and the choice / score / noul read-outs).  `batch` is a host struct
+ * whose array pointers are device pointers (tokens, cu_seqlens, mask_pos,
+ * opt_off, row_type; head_len / trunc are ignored), laid out as jd_serialize
+ * writes them.  All outputs of `out` are written; `taps` may be NULL.
+ * Errors: JD_ERR_INVALID_ARG (NULL model / batch / output, an empty batch, a
+ * row longer than 8192 tokens), JD_ERR_CAPACITY (n_tokens, n_rows or
+ * n_markers above the model's capacity), JD_ERR_CUDA (a launch or graph call
+ * failed).  Failed device-side checks (an id outside the vocabulary, a marker
+ * index outside the batch, a bounded wait that expired) are recorded in the
+ * model's status word and reported by jd_check_status. */
 jd_status jd_decide(jd_model *model, const jd_batch *batch, const jd_outputs *out,
                     const jd_taps *taps, void *stream);
 
-/* Raw logits only (the "logits(rows)" call): writes logits[M]. */
+/* Raw logits only ("Julia-1 MLX", "API": the logits(rows) call): writes
+ * logits[M] on the device; probabilities and read-outs go to the model's
+ * internal buffers.  Errors as jd_decide. */
 jd_status jd_forward(jd_model *model, const jd_batch *batch, float *logits, void *stream);
 
 /* Host outputs of jd_decide_host (caller-owned host memory, sizes as jd_outputs). */
@@ -198,10 +217,13 @@ typedef struct {
     int32_t n_rows, n_markers;    /* written by the call */
 } jd_host_outputs;
 
-/* End-to-end call: serialize `rows`, copy the packed batch to the device
- * through the model's pinned staging buffers, run jd_decide, copy the
- * outputs back and synchronize `stream`.  Output arrays must hold the total
- * number of options (logits/probs) and n_rows entries. */
+/* End-to-end call ("Julia-1 MLX", "API": predict(rows)): serialize `rows`,
+ * copy the packed batch to the device through the model's pinned staging
+ * buffers, run jd_decide, copy the outputs back and synchronize `stream`.
+ * Output arrays must hold the total number of options (logits/probs) and
+ * n_rows entries; any of them may be NULL to skip it.  Errors: those of
+ * jd_serialize and jd_decide, and JD_ERR_DEVICE_STATUS when a device-side
+ * check failed during this call (the outputs are then not written). */
 jd_status jd_decide_host(jd_model *model, const jd_row *rows, int32_t n_rows,
                          const jd_encode_opts *opts, jd_host_outputs *out, void *stream);
 
