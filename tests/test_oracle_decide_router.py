@@ -103,3 +103,33 @@ def test_router_group_of_one_passes_without_call():
 
     _, _, _, calls = route(41, score)        # 20 + 20 + 1
     assert 1 not in seen[:2] and calls[0] == 2
+
+
+def _closed_form_calls(n):
+    """Calls per round when no group ever keeps a single winner: a round over n > 20
+    candidates scores floor(n/20) full groups plus the tail group if it holds two or
+    more (a tail of one passes unscored), and leaves 2 floor(n/20) + min(n mod 20, 2);
+    at 20 or fewer, one final call if two or more remain."""
+    calls = []
+    while n > 20:
+        q, r = divmod(n, 20)
+        calls.append(q + (1 if r >= 2 else 0))
+        n = 2 * q + min(r, 2)
+    if n >= 2:
+        calls.append(1)
+    return calls
+
+
+@pytest.mark.parametrize("n", [1, 2, 20, 21, 22, 40, 41, 60, 72, 399, 400, 401, 1000, 4095, 4096])
+def test_router_call_counts_closed_form(n):
+    """Uniform probabilities in every group (p = 1/size <= 1/2 < 0.95): never a single
+    winner, so the counts follow the closed form; 4,096 is the pages' maximum."""
+    _, _, _, got = route(n, lambda groups: [np.full(len(g), 1.0 / len(g)) for g in groups])
+    assert got == _closed_form_calls(n)
+
+
+def test_router_closed_form_spot_values():
+    # worked by hand: 4096 -> 205 calls, 410 left -> 21 calls, 42 left -> 3 calls, 6 left -> final
+    assert _closed_form_calls(4096) == [205, 21, 3, 1]
+    assert _closed_form_calls(41) == [2, 1]
+    assert _closed_form_calls(1) == []
