@@ -82,3 +82,21 @@ def test_reference_arm_runs_on_rank0_only(capsys, monkeypatch):
         gpus = 2
     bench.run_reference(A)
     assert capsys.readouterr().out == ""
+
+
+def test_four_thread_oracle_leg():
+    """The cpu_baseline's 4-thread figure runs the same oracle with NumPy's BLAS
+    held to 4 threads, and reports that count."""
+    import bench
+    sys_argv = sys.argv
+    sys.argv = ["bench.py", "--rows", "4"]
+    try:
+        args = bench.parse()
+    finally:
+        sys.argv = sys_argv
+    rows, opts, _ = bench.workload(args, 0)
+    before = bench.blas_threads()
+    r = bench.oracle_four_threads(rows[:2], opts, 0.0)
+    assert r is not None and r["value"] > 0 and r["unit"] == bench.UNIT
+    assert r["cores"] == 4
+    assert bench.blas_threads() == before  # the limit is lifted afterwards
