@@ -95,6 +95,9 @@ def lib():
                                C.POINTER(C.POINTER(jd_batch)), C.POINTER(C.c_int32)]
     L.jd_batch_free.argtypes = [C.POINTER(jd_batch)]
     L.jd_batch_free.restype = None
+    L.jd_batch_info.argtypes = [C.POINTER(jd_batch), C.c_void_p]
+    L.jd_rows_encoding_info.argtypes = [C.POINTER(jd_row), C.c_int32, C.POINTER(jd_encode_opts), C.c_void_p,
+                                        C.POINTER(C.c_int32)]
     L.jd_model_create.argtypes = [C.POINTER(jd_model_config), C.c_char_p, C.c_int, C.POINTER(C.c_void_p)]
     L.jd_model_create_shared.argtypes = [C.c_void_p, C.POINTER(jd_model_config), C.POINTER(C.c_void_p)]
     L.jd_model_destroy.argtypes = [C.c_void_p]
@@ -251,6 +254,36 @@ def jd_serialize(rows, opts: jd_encode_opts):
              trunc=arr(b.trunc, b.n_rows, np.uint8))
     L.jd_batch_free(out)
     return HostBatch(d)
+
+
+# jd_encoding_info fields, in order (five int32 per row)
+ENCODING_INFO_FIELDS = ("length", "head_length", "state_length", "n_options", "truncated")
+
+
+def _info_dict(a):
+    return {k: a[:, i].copy() for i, k in enumerate(ENCODING_INFO_FIELDS)}
+
+
+def jd_rows_encoding_info(rows, opts: jd_encode_opts):
+    """Per-row encoding report of `rows` (jd_rows_encoding_info): dict of int32
+    arrays keyed by ENCODING_INFO_FIELDS.  Raises JDError like jd_serialize."""
+    keep = _RowKeep(rows)
+    a = np.zeros((max(1, len(rows)), len(ENCODING_INFO_FIELDS)), np.int32)
+    bad = C.c_int32(-1)
+    code = lib().jd_rows_encoding_info(keep.arr, len(rows), C.byref(opts), a.ctypes.data, C.byref(bad))
+    if code != JD_OK:
+        e = JDError(code, lib().jd_last_error().decode())
+        e.bad_row = bad.value
+        raise e
+    return _info_dict(a[:len(rows)])
+
+
+def jd_batch_info(hb: HostBatch):
+    """Per-row encoding report of a serialized host batch (jd_batch_info)."""
+    a = np.zeros((max(1, hb.n_rows), len(ENCODING_INFO_FIELDS)), np.int32)
+    bs = hb.as_struct()
+    _check(lib().jd_batch_info(C.byref(bs), a.ctypes.data))
+    return _info_dict(a[:hb.n_rows])
 
 
 class Model:

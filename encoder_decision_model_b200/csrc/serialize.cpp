@@ -223,3 +223,34 @@ extern "C" void jd_batch_free(jd_batch *b) {
     std::free(b->trunc);
     std::free(b);
 }
+
+extern "C" jd_status jd_batch_info(const jd_batch *b, jd_encoding_info *per_row) {
+    jd::clear_error();
+    if (!b || !per_row) return jd::fail(JD_ERR_INVALID_ARG, "NULL argument");
+    if (b->n_rows > 0 && (!b->cu_seqlens || !b->opt_off || !b->head_len || !b->trunc))
+        return jd::fail(JD_ERR_INVALID_ARG, "not a host batch from jd_serialize (no head_len / trunc)");
+    for (int r = 0; r < b->n_rows; ++r) {
+        jd_encoding_info &e = per_row[r];
+        e.length = b->cu_seqlens[r + 1] - b->cu_seqlens[r];
+        e.head_length = b->head_len[r];
+        e.state_length = e.length - e.head_length - 1;
+        e.n_options = b->opt_off[r + 1] - b->opt_off[r];
+        e.truncated = b->trunc[r];
+    }
+    return JD_OK;
+}
+
+extern "C" jd_status jd_rows_encoding_info(const jd_row *rows, int32_t n_rows, const jd_encode_opts *opts,
+                                           jd_encoding_info *per_row, int32_t *bad_row) {
+    if (bad_row) *bad_row = -1;
+    if (!per_row && n_rows > 0) {
+        jd::clear_error();
+        return jd::fail(JD_ERR_INVALID_ARG, "per_row is NULL");
+    }
+    jd_batch *b = nullptr;
+    jd_status s = jd_serialize(rows, n_rows, opts, &b, bad_row);
+    if (s != JD_OK) return s;
+    s = jd_batch_info(b, per_row);
+    jd_batch_free(b);
+    return s;
+}

@@ -159,6 +159,26 @@ jd_status jd_serialize(const jd_row *rows, int32_t n_rows, const jd_encode_opts 
                        jd_batch **out, int32_t *bad_row);
 void jd_batch_free(jd_batch *batch);
 
+/* Per-row encoding report ("Julia-1 MLX", "API": encoding_info(rows) gives the
+ * lengths a request encodes to and whether anything was truncated). */
+typedef struct {
+    int32_t length;       /* serialized tokens of the row (head + state + final eos) */
+    int32_t head_length;  /* tokens before the state: bos, question, eos, markers, options, eos */
+    int32_t state_length; /* state ids kept */
+    int32_t n_options;    /* k */
+    int32_t truncated;    /* JD_TRUNC_* bits; 0 when nothing was clipped (always 0 in strict mode) */
+} jd_encoding_info;
+
+/* The report of a host batch from jd_serialize: per_row[n_rows] (caller-owned
+ * host memory).  Errors: JD_ERR_INVALID_ARG for a NULL argument or a batch
+ * without its host-side head_len / trunc arrays (a device batch). */
+jd_status jd_batch_info(const jd_batch *batch, jd_encoding_info *per_row);
+
+/* The same report straight from rows, with jd_serialize's rules and errors
+ * (*bad_row as there); nothing is kept. */
+jd_status jd_rows_encoding_info(const jd_row *rows, int32_t n_rows, const jd_encode_opts *opts,
+                                jd_encoding_info *per_row, int32_t *bad_row);
+
 /* Load the .jdw weights file and allocate the device workspace for the given
  * capacity on `device` (the architecture of "The decision head" and "Julia-1
  * MLX", "Performance": 22 encoder layers of width 384, a 3 x 384 type table,

@@ -235,3 +235,58 @@ def test_route_requires_winner_output(L):
                            4096, 16, 64, ctypes.byref(out), None)
     assert code == jl.JD_ERR_INVALID_ARG
     assert "winner" in L.jd_last_error().decode()
+
+
+def _oracle_info(rows, opt):
+    out = {k: [] for k in jl.ENCODING_INFO_FIELDS}
+    for r in rows:
+        e = serialize_row(r, opt)
+        out["length"].append(len(e.ids))
+        out["head_length"].append(e.head_len)
+        out["state_length"].append(len(e.ids) - e.head_len - 1)
+        out["n_options"].append(len(e.mask_pos))
+        out["truncated"].append(e.trunc)
+    return out
+
+
+@pytest.mark.parametrize("case", ["c1", "c2", "c3", "random"])
+def test_encoding_info_matches_oracle(L, case):
+    """The encoding_info report ("Julia-1 MLX", "API"), from rows and from a host
+    batch, against the oracle serializer row by row."""
+    if case == "c1":
+        rows, args = rows_config1(), (1024, 512, True)
+    elif case == "c2":
+        rows, args = rows_config2(64), (1024, 512, True)
+    elif case == "c3":
+        rows, args = rows_config3(4), (8192, 256, False)
+    else:
+        rng = np.random.default_rng(21)
+        rows, args = [], (128, 64, False)
+        for r in _rand_rows(rng, 80):
+            try:
+                serialize_row(r, EncodeOptions(max_length=128, head_budget=64, strict=False))
+                rows.append(r)
+            except EncodingError:
+                pass
+    want = _oracle_info(rows, EncodeOptions(max_length=args[0], head_budget=args[1], strict=args[2]))
+    got = jl.jd_rows_encoding_info(rows, jl.encode_opts(*args))
+    got_b = jl.jd_batch_info(jl.jd_serialize(rows, jl.encode_opts(*args)))
+    for k in jl.ENCODING_INFO_FIELDS:
+        np.testing.assert_array_equal(got[k], want[k], err_msg=k)
+        np.testing.assert_array_equal(got_b[k], want[k], err_msg=k)
+    if case in ("c3", "random"):
+        assert any(want["truncated"]), "the non-strict cases must exercise truncation"
+
+
+def test_encoding_info_errors(L):
+    rows = rows_config1()
+    bad = Row(state=rows[0].state, question=rows[0].question, options=rows[0].options[:1], qtype=0)
+    with pytest.raises(jl.JDError) as ei:
+        jl.jd_rows_encoding_info(rows + [bad], jl.encode_opts(1024, 512, True))
+    assert ei.value.code == jl.JD_ERR_OPTION_COUNT and ei.value.bad_row == 3
+    # a device-style batch (no host-side head_len / trunc) is refused
+    hb = jl.jd_serialize(rows, jl.encode_opts(1024, 512, True))
+    bs = hb.as_struct()
+    bs.head_len = None
+    out = np.zeros((len(rows), 5), np.int32)
+    assert L.jd_batch_info(ctypes.byref(bs), out.ctypes.data) == jl.JD_ERR_INVALID_ARG
