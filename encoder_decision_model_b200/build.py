@@ -70,7 +70,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
         if log.strip() and (verbose or ptxas_verbose):
             print(log, file=sys.stderr)
     tmp = target.with_suffix(".so.tmp")
-    cmd = [nvcc, *ARCH, "-shared", "-o", str(tmp), *[str(o) for o, _ in results], "-lcuda" if False else "-lcudart_static",
+    cmd = [nvcc, *ARCH, "-shared", "-o", str(tmp), *[str(o) for o, _ in results], "-lcudart_static",
            "-lpthread", "-ldl", "-lrt"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
