@@ -71,6 +71,10 @@ class jd_route_outputs(C.Structure):
                 ("rows_per_round", i32p), ("max_rounds", C.c_int32), ("n_rounds", C.c_int32)]
 
 
+# jd_route_scorer: (user, rows, n_rows, probs) -> jd_status
+ROUTE_SCORER = C.CFUNCTYPE(C.c_int, C.c_void_p, C.POINTER(jd_row), C.c_int32, C.POINTER(C.c_float))
+
+
 class JDError(RuntimeError):
     def __init__(self, code, msg):
         super().__init__(f"[{code}] {msg}")
@@ -96,6 +100,8 @@ def lib():
     L.jd_batch_free.argtypes = [C.POINTER(jd_batch)]
     L.jd_batch_free.restype = None
     L.jd_batch_info.argtypes = [C.POINTER(jd_batch), C.c_void_p]
+    L.jd_route_scored.argtypes = [C.POINTER(jd_route_request), C.c_int32, ROUTE_SCORER, C.c_void_p,
+                                  C.POINTER(jd_route_outputs)]
     L.jd_rows_encoding_info.argtypes = [C.POINTER(jd_row), C.c_int32, C.POINTER(jd_encode_opts), C.c_void_p,
                                         C.POINTER(C.c_int32)]
     L.jd_model_create.argtypes = [C.POINTER(jd_model_config), C.c_char_p, C.c_int, C.POINTER(C.c_void_p)]
@@ -286,6 +292,77 @@ def jd_batch_info(hb: HostBatch):
     return _info_dict(a[:hb.n_rows])
 
 
+def _route_marshal(requests):
+    """jd_route_request records for `requests` (objects with state/question/labels),
+    the arrays they point into, and the outputs dict with its jd_route_outputs."""
+    n = len(requests)
+    st, st_off, st_len = _pack_lists([r.state for r in requests])
+    q, q_off, q_len = _pack_lists([r.question for r in requests])
+    nl = np.fromiter((len(r.labels) for r in requests), dtype=np.int64, count=n)
+    lab, l_off, l_len = _pack_lists([x for r in requests for x in r.labels])
+    labp = (lab.ctypes.data + 4 * l_off).astype(np.uint64) if len(l_off) else np.zeros(1, np.uint64)
+    llen = l_len.astype(np.int32) if len(l_len) else np.zeros(1, np.int32)
+    first = np.zeros(n, dtype=np.int64)
+    if n > 1:
+        np.cumsum(nl[:-1], out=first[1:])
+    req = np.zeros(max(1, n), dtype=_struct_dtype(jd_route_request))
+    if n:
+        req["state"][:n] = st.ctypes.data + 4 * st_off
+        req["n_state"][:n] = st_len
+        req["question"][:n] = q.ctypes.data + 4 * q_off
+        req["n_question"][:n] = q_len
+        req["labels"][:n] = labp.ctypes.data + 8 * first
+        req["n_label_ids"][:n] = llen.ctypes.data + 4 * first
+        req["n_labels"][:n] = nl
+    keep = (st, q, lab, labp, llen, req)
+    arr = req.ctypes.data_as(C.POINTER(jd_route_request))
+    o = dict(winner=np.zeros(n, np.int32), winner_p=np.zeros(n, np.float32),
+             final_candidates=np.zeros((n, 20), np.int32), final_probs=np.zeros((n, 20), np.float32),
+             rows_per_round=np.zeros(16, np.int32))
+    s = jd_route_outputs(o["winner"].ctypes.data_as(i32p), o["winner_p"].ctypes.data_as(f32p),
+                         o["final_candidates"].ctypes.data_as(i32p), o["final_probs"].ctypes.data_as(f32p),
+                         o["rows_per_round"].ctypes.data_as(i32p), 16, 0)
+    return arr, keep, o, s
+
+
+def _route_result(o, s):
+    o["rows_per_round"] = o["rows_per_round"][:s.n_rounds]
+    return o
+
+
+def jd_route_scored(requests, score):
+    """The Router's tournament (jd_route_scored) with `score` as the scorer:
+    score(rows) gets, per row, the list of its options' label-id arrays and
+    returns, per row, the option probabilities (float32 is what the library
+    keeps).  Returns the same dict as Model.jd_route_host."""
+    arr, keep, o, s = _route_marshal(requests)
+    err = []
+
+    def cb(user, rows, n_rows, probs):
+        try:
+            opts = []
+            for i in range(n_rows):
+                r = rows[i]
+                opts.append([np.ctypeslib.as_array(r.options[k], shape=(r.n_option_ids[k],)).copy()
+                             if r.n_option_ids[k] else np.zeros(0, np.int32) for k in range(r.k)])
+            ps = score(opts)
+            flat = np.concatenate([np.asarray(p, np.float32) for p in ps])
+            if len(flat) != sum(len(x) for x in opts):
+                raise ValueError("score() returned the wrong number of probabilities")
+            C.memmove(probs, flat.ctypes.data, flat.nbytes)
+            return JD_OK
+        except Exception as e:  # reported after the call; the library sees a failed status
+            err.append(e)
+            return JD_ERR_INVALID_ARG
+
+    fn = ROUTE_SCORER(cb)
+    code = lib().jd_route_scored(arr, len(requests), fn, None, C.byref(s))
+    if err:
+        raise err[0]
+    _check(code)
+    return _route_result(o, s)
+
+
 class Model:
     """Owner of a jd_model handle (weights + workspace on one device)."""
 
@@ -344,39 +421,12 @@ class Model:
                       stream=None):
         """Route requests (objects with state/question/labels); returns dict of
         winner, winner_p, final_candidates [n, 20], final_probs [n, 20], rows_per_round."""
-        n = len(requests)
-        st, st_off, st_len = _pack_lists([r.state for r in requests])
-        q, q_off, q_len = _pack_lists([r.question for r in requests])
-        nl = np.fromiter((len(r.labels) for r in requests), dtype=np.int64, count=n)
-        lab, l_off, l_len = _pack_lists([x for r in requests for x in r.labels])
-        labp = (lab.ctypes.data + 4 * l_off).astype(np.uint64) if len(l_off) else np.zeros(1, np.uint64)
-        llen = l_len.astype(np.int32) if len(l_len) else np.zeros(1, np.int32)
-        first = np.zeros(n, dtype=np.int64)
-        if n > 1:
-            np.cumsum(nl[:-1], out=first[1:])
-        req = np.zeros(max(1, n), dtype=_struct_dtype(jd_route_request))
-        if n:
-            req["state"][:n] = st.ctypes.data + 4 * st_off
-            req["n_state"][:n] = st_len
-            req["question"][:n] = q.ctypes.data + 4 * q_off
-            req["n_question"][:n] = q_len
-            req["labels"][:n] = labp.ctypes.data + 8 * first
-            req["n_label_ids"][:n] = llen.ctypes.data + 4 * first
-            req["n_labels"][:n] = nl
-        keep = (st, q, lab, labp, llen, req)
-        arr = req.ctypes.data_as(C.POINTER(jd_route_request))
-        o = dict(winner=np.zeros(n, np.int32), winner_p=np.zeros(n, np.float32),
-                 final_candidates=np.zeros((n, 20), np.int32), final_probs=np.zeros((n, 20), np.float32),
-                 rows_per_round=np.zeros(16, np.int32))
-        s = jd_route_outputs(o["winner"].ctypes.data_as(i32p), o["winner_p"].ctypes.data_as(f32p),
-                             o["final_candidates"].ctypes.data_as(i32p), o["final_probs"].ctypes.data_as(f32p),
-                             o["rows_per_round"].ctypes.data_as(i32p), 16, 0)
+        arr, keep, o, s = _route_marshal(requests)
         c = self.cfg
-        _check(lib().jd_route_host(self.h, arr, n, C.byref(opts), int(max_tokens or c.max_tokens),
+        _check(lib().jd_route_host(self.h, arr, len(requests), C.byref(opts), int(max_tokens or c.max_tokens),
                                    int(max_rows or c.max_rows), int(max_markers or c.max_markers), C.byref(s),
                                    _stream(stream)))
-        o["rows_per_round"] = o["rows_per_round"][:s.n_rounds]
-        return o
+        return _route_result(o, s)
 
     def jd_forward_noalloc(self, batch: jd_batch, logits, stream=None):
         """jd_forward with every intermediate in the library's static device

@@ -8,7 +8,8 @@
 // above 0.95 and every other is below 0.045, otherwise its two most probable
 // candidates (lower index first on ties), in their original order; a group of
 // one candidate passes through unscored.  When 20 or fewer remain, one final
-// call per request picks the winner.
+// call per request picks the winner.  jd_route_host scores through the model;
+// jd_route_scored runs the same tournament on a caller's scoring callback.
 
 #include <algorithm>
 #include <cstring>
@@ -79,18 +80,44 @@ void survivors(const float *p, int n, std::vector<int> &keep) {
     }
 }
 
-}  // namespace
+// Scoring through the model (jd_route_host): chunks within the capacity, serialised with opts.
+struct ModelScorer {
+    jd_model *m;
+    const jd_encode_opts *opts;
+    void *stream;
+    int32_t max_tokens, max_rows, max_markers;
+};
 
-extern "C" jd_status jd_route_host(jd_model *m, const jd_route_request *reqs, int32_t n_requests,
-                                   const jd_encode_opts *opts, int32_t max_tokens, int32_t max_rows,
-                                   int32_t max_markers, jd_route_outputs *out, void *stream) {
-    jd::clear_error();
-    if (!m || !opts || !out || (n_requests > 0 && !reqs) || n_requests < 0)
+jd_status model_scorer(void *user, const jd_row *rows, int32_t n_rows, float *probs) {
+    const ModelScorer &ms = *static_cast<const ModelScorer *>(user);
+    std::vector<jd_row> v(rows, rows + n_rows);
+    std::vector<float> p;
+    jd_status s = score_rows(ms.m, v, ms.opts, ms.stream, ms.max_tokens, ms.max_rows, ms.max_markers, p);
+    if (s != JD_OK) return s;
+    size_t n_opts = 0;
+    for (int32_t i = 0; i < n_rows; ++i) n_opts += (size_t)rows[i].k;
+    if (p.size() != n_opts) return jd::fail(JD_ERR_INVALID_ARG, "scored %zu options for %zu", p.size(), n_opts);
+    std::copy(p.begin(), p.end(), probs);
+    return JD_OK;
+}
+
+// One round's scoring: probs gets every option of every row, in row order.
+jd_status score(jd_route_scorer scorer, void *user, const std::vector<jd_row> &rows, size_t n_opts,
+                std::vector<float> &probs) {
+    probs.assign(n_opts, 0.f);
+    if (rows.empty()) return JD_OK;
+    jd_status s = scorer(user, rows.data(), (int32_t)rows.size(), probs.data());
+    if (s != JD_OK && jd_last_error()[0] == 0) jd::fail(s, "the scorer returned %d", (int)s);
+    return s;
+}
+
+// The tournament, scoring each round's rows through `scorer`.
+jd_status route_core(const jd_route_request *reqs, int32_t n_requests, jd_route_scorer scorer, void *user,
+                     jd_route_outputs *out) {
+    if (!scorer || !out || (n_requests > 0 && !reqs) || n_requests < 0)
         return jd::fail(JD_ERR_INVALID_ARG, "NULL argument");
     if (n_requests > 0 && !out->winner) return jd::fail(JD_ERR_INVALID_ARG, "out->winner is NULL");
     if (out->rows_per_round && out->max_rounds < 0) return jd::fail(JD_ERR_INVALID_ARG, "max_rounds < 0");
-    if (max_tokens < 1 || max_rows < 1 || max_markers < kGroup)
-        return jd::fail(JD_ERR_INVALID_ARG, "chunk capacities too small");
     for (int r = 0; r < n_requests; ++r)
         if (reqs[r].n_labels < 1 || reqs[r].n_labels > kMaxLabels || !reqs[r].labels || !reqs[r].n_label_ids)
             return jd::fail(JD_ERR_INVALID_ARG, "request %d: 1..4096 labels required", r);
@@ -146,7 +173,7 @@ extern "C" jd_status jd_route_host(jd_model *m, const jd_route_request *reqs, in
             rows.push_back(build_row(pend[g].req, cands[pend[g].req].data() + pend[g].first, pend[g].size, slot));
             slot += pend[g].size;
         }
-        jd_status s = score_rows(m, rows, opts, stream, max_tokens, max_rows, max_markers, probs);
+        jd_status s = score(scorer, user, rows, n_opts, probs);
         if (s != JD_OK) return s;
         if (out->rows_per_round && round < out->max_rounds) out->rows_per_round[round] = (int32_t)rows.size();
         ++round;
@@ -184,6 +211,8 @@ extern "C" jd_status jd_route_host(jd_model *m, const jd_route_request *reqs, in
         if (nc == 1) {
             out->winner[r] = cands[r][0];
             if (out->winner_p) out->winner_p[r] = 1.0f;
+            if (out->final_probs)
+                for (int k = 0; k < kGroup; ++k) out->final_probs[(size_t)r * kGroup + k] = k == 0 ? 1.0f : 0.f;
             continue;
         }
         rows.push_back(build_row(r, cands[r].data(), nc, slot));
@@ -191,7 +220,7 @@ extern "C" jd_status jd_route_host(jd_model *m, const jd_route_request *reqs, in
         slot += nc;
     }
     if (!rows.empty()) {
-        jd_status s = score_rows(m, rows, opts, stream, max_tokens, max_rows, max_markers, probs);
+        jd_status s = score(scorer, user, rows, n_opts, probs);
         if (s != JD_OK) return s;
         if (out->rows_per_round && round < out->max_rounds) out->rows_per_round[round] = (int32_t)rows.size();
         ++round;
@@ -211,4 +240,24 @@ extern "C" jd_status jd_route_host(jd_model *m, const jd_route_request *reqs, in
     }
     out->n_rounds = round;
     return JD_OK;
+}
+
+}  // namespace
+
+extern "C" jd_status jd_route_scored(const jd_route_request *requests, int32_t n_requests, jd_route_scorer scorer,
+                                     void *user, jd_route_outputs *out) {
+    jd::clear_error();
+    return route_core(requests, n_requests, scorer, user, out);
+}
+
+extern "C" jd_status jd_route_host(jd_model *m, const jd_route_request *reqs, int32_t n_requests,
+                                   const jd_encode_opts *opts, int32_t max_tokens, int32_t max_rows,
+                                   int32_t max_markers, jd_route_outputs *out, void *stream) {
+    jd::clear_error();
+    if (!m || !opts || !out || (n_requests > 0 && !reqs) || n_requests < 0)
+        return jd::fail(JD_ERR_INVALID_ARG, "NULL argument");
+    if (max_tokens < 1 || max_rows < 1 || max_markers < kGroup)
+        return jd::fail(JD_ERR_INVALID_ARG, "chunk capacities too small");
+    ModelScorer ms{m, opts, stream, max_tokens, max_rows, max_markers};
+    return route_core(reqs, n_requests, model_scorer, &ms, out);
 }

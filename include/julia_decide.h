@@ -267,7 +267,7 @@ typedef struct {
     int32_t *winner;            /* required [n_requests] index of the chosen label (NULL: JD_ERR_INVALID_ARG) */
     float *winner_p;            /* optional [n_requests] its probability in the final call (1 if unscored) */
     int32_t *final_candidates;  /* optional [n_requests * 20] label indices of the final call, -1 padded */
-    float *final_probs;         /* optional [n_requests * 20] their probabilities */
+    float *final_probs;         /* optional [n_requests * 20] their probabilities (1 for a lone, unscored candidate) */
     int32_t *rows_per_round;    /* optional [max_rounds] rows scored per round, all requests together */
     int32_t max_rounds;         /* >= 0 when rows_per_round is set; rounds beyond it are not recorded */
     int32_t n_rounds;           /* written: rounds including the final call */
@@ -285,6 +285,20 @@ typedef struct {
 jd_status jd_route_host(jd_model *model, const jd_route_request *requests, int32_t n_requests,
                         const jd_encode_opts *opts, int32_t max_tokens, int32_t max_rows, int32_t max_markers,
                         jd_route_outputs *out, void *stream);
+
+/* Scoring callback of jd_route_scored: score n_rows choice rows (host memory,
+ * valid during the call) and write the probabilities of every option of every
+ * row, in row order, into probs (host memory, one entry per option of the
+ * rows).  Any status other than JD_OK ends the route with that status. */
+typedef jd_status (*jd_route_scorer)(void *user, const jd_row *rows, int32_t n_rows, float *probs);
+
+/* The same tournament as jd_route_host with the scoring left to `scorer`
+ * (jd_route_host is this with the model's forward pass as the scorer): the
+ * grouping, the survivor rule, the final call and the outputs are identical.
+ * Needs no device.  Errors: JD_ERR_INVALID_ARG (NULL scorer / out / winner, a
+ * request without labels or with more than 4096), or the scorer's status. */
+jd_status jd_route_scored(const jd_route_request *requests, int32_t n_requests, jd_route_scorer scorer,
+                          void *user, jd_route_outputs *out);
 
 /* Synchronize the model's last stream and read the device status word;
  * JD_ERR_DEVICE_STATUS with a message if a kernel recorded a failure. */
