@@ -17,6 +17,16 @@
         }                                                          \
     } while (0)
 
+/* A scorer that gives every option of a row the same probability: no group
+ * ever keeps a single winner, so each keeps its first two candidates. */
+static jd_status uniform_scorer(void *user, const jd_row *rows, int32_t n_rows, float *probs) {
+    int *calls = (int *)user;
+    ++*calls;
+    for (int32_t r = 0; r < n_rows; ++r)
+        for (int32_t k = 0; k < rows[r].k; ++k) *probs++ = 1.0f / (float)rows[r].k;
+    return JD_OK;
+}
+
 int main(void) {
     int32_t q[10], o0[4], o1[3], o2[4], st[9];
     for (int i = 0; i < 10; ++i) q[i] = 100 + i;
@@ -66,6 +76,29 @@ int main(void) {
     tight.strict = 0;
     CHECK(jd_rows_encoding_info(&row, 1, &tight, &info, &bad) == JD_OK);
     CHECK(info.head_length <= 26 && (info.truncated & JD_TRUNC_OPTION_CAP));
+
+    /* the Router on the explainer's example ("More than 20 options: the Router"):
+     * sixty labels cost three calls in the first round and one final call */
+    int32_t lab_ids[60];
+    const int32_t *labels[60];
+    int32_t lab_n[60];
+    for (int i = 0; i < 60; ++i) {
+        lab_ids[i] = 1000 + i;
+        labels[i] = &lab_ids[i];
+        lab_n[i] = 1;
+    }
+    jd_route_request req = {st, 9, q, 10, labels, lab_n, 60};
+    int32_t winner = -1, rounds[4] = {0, 0, 0, 0}, fc[20];
+    float wp = 0.f;
+    jd_route_outputs ro = {&winner, &wp, fc, NULL, rounds, 4, 0};
+    int scorer_calls = 0;
+    CHECK(jd_route_scored(&req, 1, uniform_scorer, &scorer_calls, &ro) == JD_OK);
+    CHECK(ro.n_rounds == 2 && rounds[0] == 3 && rounds[1] == 1 && scorer_calls == 2);
+    /* groups 0-19, 20-39, 40-59 keep their first two; the final call's tie goes to the first */
+    CHECK(fc[0] == 0 && fc[1] == 1 && fc[2] == 20 && fc[3] == 21 && fc[4] == 40 && fc[5] == 41 && fc[6] == -1);
+    CHECK(winner == 0 && wp > 0.16f && wp < 0.17f);
+    ro.winner = NULL;
+    CHECK(jd_route_scored(&req, 1, uniform_scorer, &scorer_calls, &ro) == JD_ERR_INVALID_ARG);
 
     /* a model needs arguments; NULL ones are refused before any device work */
     jd_model *m = NULL;
