@@ -354,3 +354,20 @@ def test_type_row_changes_only_through_type(weights_file):
     za, zb = m.logits(e), m.logits(e1)
     assert za.shape == (3,) and np.abs(za - zb).max() > 1e-6
     np.testing.assert_allclose(enc.mean(-1), 0, atol=1e-12)  # final norm output
+
+
+def test_scorer_is_per_marker_for_any_k(oracle_model):
+    """"The decision head": the head's output width is 1, so two options and twenty use the
+    same weights -- each option's logit depends on its own marker state only.  Scoring 20
+    marker states, their first 2, a permutation of them, or each alone gives the same
+    logits (to 1e-12: only the matrix product's blocking may change the rounding)."""
+    rng = np.random.default_rng(20)
+    hm = rng.normal(size=(20, 384))
+    W, mo = oracle_model.W, oracle_model.mo
+    z = om.scorer(hm, W, mo)
+    assert z.shape == (20,)
+    np.testing.assert_allclose(om.scorer(hm[:2], W, mo), z[:2], rtol=0, atol=1e-12)
+    perm = rng.permutation(20)
+    np.testing.assert_allclose(om.scorer(hm[perm], W, mo), z[perm], rtol=0, atol=1e-12)
+    alone = np.array([om.scorer(hm[k:k + 1], W, mo)[0] for k in range(20)])
+    np.testing.assert_allclose(alone, z, rtol=0, atol=1e-12)
