@@ -20,9 +20,10 @@ Sources (page title, section):
     bias / ReLU epilogues, marker-only last head layer).
 
 Parity status per function is listed in the module docstrings; every function
-here has at least one pin in tests/test_oracle_*.py except the full-model
-logits against a trained checkpoint, which no page provides (parity unpinned
-for that end-to-end value; the oracle is pinned component by component).
+here has at least one pin in tests/test_oracle_*.py, and the whole chain of
+"The decision head" (encoder, final norm, type row, both head layers, gather,
+scorer) has a closed-form pin on tiny structured weights.  Logits of the
+trained model are not pinned: no page provides a checkpoint or its outputs.
 """
 from .serialize import (  # noqa: F401
     EncodeOptions, EncodingError, Encoded, serialize_row, serialize_rows,

@@ -33,8 +33,10 @@ plausible):
     "linear": LayerNorm -> Linear(384 -> 1)).
 Arithmetic is float64 end to end; weights are the float32 values of the file.
 Parity: each function is pinned in tests/test_oracle_model.py by closed forms,
-brute force on tiny inputs and invariants; full-model logits have no printed
-value to pin against (parity unpinned end to end, pinned per component).
+brute force on tiny inputs and invariants, and the whole chain (encoder ->
+final norm -> type row -> head layer 0 -> head layer 1 -> gather -> scorer) by
+a closed form on tiny structured weights.  Logits of the trained model have
+no printed value to pin against (no checkpoint offline).
 """
 from __future__ import annotations
 
@@ -205,38 +207,45 @@ def scorer(hm, W, mo: ModelOptions):
 
 
 class OracleModel:
-    """Forward pass of one serialised row at a time."""
+    """Forward pass of one serialised row at a time.
 
-    def __init__(self, weights_path, options: ModelOptions | None = None):
-        self.W = Weights(weights_path)
+    `weights` is a .jdw path, or any mapping of tensor names to arrays that
+    also has `embed_rows(ids)` (the tests build tiny structured ones)."""
+
+    def __init__(self, weights, options: ModelOptions | None = None):
+        self.W = weights if hasattr(weights, "embed_rows") else Weights(weights)
         self.mo = options or ModelOptions()
 
     def encode(self, ids):
-        """Encoder output after the final norm, [L, 384]."""
+        """Encoder output after the final norm, [L, d]."""
         W, mo = self.W, self.mo
         x = layer_norm(W.embed_rows(ids), W["embed.norm.g"], eps=mo.eps)
         for l in range(mo.n_layers):
             x = encoder_layer(x, W, l, mo)
         return layer_norm(x, W["enc.final_norm.g"], eps=mo.eps)
 
-    def hidden(self, ids, qtype):
-        """State after the type-row add and both head layers, [L, 384]."""
-        h = self.encode(ids) + self.W["head.type_table"][qtype]
+    def head(self, e, qtype):
+        """"The decision head", steps 1-2: the type-table row added to every
+        position of the encoder output e, then both head layers, [L, d]."""
+        h = e + self.W["head.type_table"][qtype]
         for i in range(2):
             h = head_layer(h, self.W, i, self.mo)
         return h
 
-    def logits(self, enc):
-        """Raw option logits for one serialised row (oracle.serialize.Encoded)."""
-        h = self.hidden(enc.ids, enc.qtype)
-        return scorer(h[np.asarray(enc.mask_pos, dtype=np.int64)], self.W, self.mo)
+    def hidden(self, ids, qtype):
+        """State after the type-row add and both head layers, [L, d]."""
+        return self.head(self.encode(ids), qtype)
 
     def forward_all(self, enc):
-        """The same pass, returning the encoder output (after the final norm),
-        the marker states after both head layers, and the logits."""
+        """The whole pass for one serialised row (oracle.serialize.Encoded):
+        encoder -> final norm -> steps 1-2 (head) -> step 3 (gather at the
+        <mask> positions) -> step 4 (scorer).  Returns the encoder output
+        (after the final norm), the marker states after both head layers,
+        and the raw option logits."""
         e = self.encode(enc.ids)
-        h = e + self.W["head.type_table"][enc.qtype]
-        for i in range(2):
-            h = head_layer(h, self.W, i, self.mo)
-        hm = h[np.asarray(enc.mask_pos, dtype=np.int64)]
+        hm = self.head(e, enc.qtype)[np.asarray(enc.mask_pos, dtype=np.int64)]
         return dict(encoder_out=e, marker_state=hm, logits=scorer(hm, self.W, self.mo))
+
+    def logits(self, enc):
+        """Raw option logits for one serialised row (the same chain as forward_all)."""
+        return self.forward_all(enc)["logits"]

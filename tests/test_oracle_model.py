@@ -371,3 +371,170 @@ def test_scorer_is_per_marker_for_any_k(oracle_model):
     np.testing.assert_allclose(om.scorer(hm[perm], W, mo), z[perm], rtol=0, atol=1e-12)
     alone = np.array([om.scorer(hm[k:k + 1], W, mo)[0] for k in range(20)])
     np.testing.assert_allclose(alone, z, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ whole-model composition
+
+
+class _ArrayWeights(dict):
+    """Tensor name -> float64 array, with the embedding lookup OracleModel uses."""
+
+    def embed_rows(self, ids):
+        return self["embed.E"][np.asarray(ids, dtype=np.int64)]
+
+
+def _composition_weights(d=8, vocab=16, hf=6, layers=2, seed=30):
+    """Tiny structured weights whose whole forward pass has a closed form.
+
+    Every encoder projection is zero, so each encoder layer leaves x unchanged
+    and the encoder output is LN_final(LN_embed(E[id])).  Both head layers have
+    in_proj.W = 0, so every query sees equal scores and a constant value row
+    b_v: attention returns b_v exactly.  Head layer 0's feed-forward reads
+    nothing of h (linear1.W = 0): the layer adds a constant c0.  Head layer 1's
+    feed-forward reads LN2(h) through a non-negative selection P and ReLU, so
+    its result depends on what head layer 0 added before it (the order of the
+    two layers shows)."""
+    rng = np.random.default_rng(seed)
+    W = _ArrayWeights(_tiny_weights(d=d, H=2, f=4, hf=hf, layers=layers))
+    W["embed.E"] = rng.normal(size=(vocab, d))
+    W["embed.norm.g"] = np.linspace(0.5, 1.5, d)
+    W["enc.final_norm.g"] = np.linspace(2.0, 0.7, d)
+    W["head.type_table"] = rng.normal(size=(3, d))
+    for i in range(2):
+        p = f"head.{i}."
+        W[p + "in_proj.b"][2 * d:] = rng.normal(size=d)        # b_v
+        W[p + "out_proj.W"][:] = rng.normal(size=(d, d))
+        W[p + "out_proj.b"][:] = rng.normal(size=d)
+        W[p + "linear2.W"][:] = rng.normal(size=(d, hf))
+        W[p + "linear2.b"][:] = rng.normal(size=d)
+        W[p + "norm2.g"][:] = np.linspace(0.8, 1.3, d)
+        W[p + "norm2.b"][:] = 0.1 * (i + 1)
+    W["head.0.linear1.b"][:] = np.array([1.0, -2.0, 0.5, -0.1, 3.0, -4.0])
+    P = np.zeros((hf, d))
+    P[np.arange(hf), [1, 3, 4, 0, 6, 7]] = [1.0, -1.5, 2.0, 0.7, -0.4, 1.1]
+    W["head.1.linear1.W"][:] = P
+    W["scorer.norm.g"] = np.linspace(1.5, 0.5, d)
+    W["scorer.norm.b"] = np.full(d, 0.05)
+    W["scorer.linear1.W"] = rng.normal(size=(d, d)) / math.sqrt(d)
+    W["scorer.linear1.b"] = rng.normal(size=d) * 0.1
+    W["scorer.linear2.W"] = rng.normal(size=(1, d))
+    W["scorer.linear2.b"] = np.array([0.3])
+    return W
+
+
+def _composition_expected(W, ids, mask_pos, qtype, eps=1e-5):
+    """The logits of "The decision head", steps 1-4, for the weights above,
+    written out vector by vector from their construction."""
+    def ln(v, g, b=0.0):
+        mu = sum(v) / len(v)
+        var = sum((t - mu) ** 2 for t in v) / len(v)
+        return np.array([(t - mu) / math.sqrt(var + eps) for t in v]) * g + b
+
+    def gelu(t):
+        return 0.5 * t * (1.0 + math.erf(t / math.sqrt(2.0)))
+
+    out = []
+    for m in mask_pos:
+        x = ln(W["embed.E"][ids[m]], W["embed.norm.g"])         # embedding norm
+        e = ln(x, W["enc.final_norm.g"])                         # encoder (identity layers) + final norm
+        h = e + W["head.type_table"][qtype]                      # step 1: type row after the final norm
+        p = "head.0."                                            # step 2, head layer 0: constant c0
+        h = h + W[p + "out_proj.W"] @ W[p + "in_proj.b"][16:] + W[p + "out_proj.b"]
+        h = h + W[p + "linear2.W"] @ np.maximum(W[p + "linear1.b"], 0) + W[p + "linear2.b"]
+        p = "head.1."                                            # head layer 1: reads LN2(h)
+        h = h + W[p + "out_proj.W"] @ W[p + "in_proj.b"][16:] + W[p + "out_proj.b"]
+        f = ln(h, W[p + "norm2.g"], W[p + "norm2.b"])
+        h = h + W[p + "linear2.W"] @ np.maximum(W[p + "linear1.W"] @ f, 0) + W[p + "linear2.b"]
+        n = ln(h, W["scorer.norm.g"], W["scorer.norm.b"])        # step 3 gathers h at the marker; step 4
+        z = np.array([gelu(t) for t in W["scorer.linear1.W"] @ n + W["scorer.linear1.b"]])
+        out.append(float(W["scorer.linear2.W"][0] @ z + W["scorer.linear2.b"][0]))
+    return np.array(out)
+
+
+def _composition_case():
+    from oracle.serialize import Encoded
+    # the identity encoder layers mix no positions, so the ids at the three marker positions
+    # differ (4, 12, 3) to give each marker its own logit; a gather that reads the wrong
+    # position then reads a different embedding row
+    ids = np.array([2, 11, 7, 1, 4, 9, 12, 13, 3, 5, 1, 15, 8, 1], dtype=np.int32)
+    return Encoded(ids=ids, mask_pos=np.array([4, 6, 8], dtype=np.int32), qtype=1, trunc=0, head_len=11)
+
+
+def test_whole_model_composition_closed_form():
+    """"Julia-1: one score per mask token", "The decision head", steps 1-4: the
+    encoder output after its final norm gets the type row, then head layer 0,
+    then head layer 1, then the hidden state is gathered at each <mask> and
+    scored.  The oracle's whole chain (forward_all, logits, hidden) must give
+    the logits written out by hand for structured tiny weights."""
+    W = _composition_weights()
+    mo = om.ModelOptions(n_layers=2, n_heads=2)
+    m = om.OracleModel(W, mo)
+    e = _composition_case()
+    ref = _composition_expected(W, e.ids, e.mask_pos, e.qtype)
+    out = m.forward_all(e)
+    np.testing.assert_allclose(out["logits"], ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(m.logits(e), ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(m.hidden(e.ids, e.qtype)[e.mask_pos], out["marker_state"], rtol=0, atol=0)
+    assert np.ptp(ref) > 1e-3  # the markers are told apart
+
+
+class _TypeRowBeforeFinalNorm(om.OracleModel):
+    def forward_all(self, enc):
+        W, mo = self.W, self.mo
+        x = om.layer_norm(W.embed_rows(enc.ids), W["embed.norm.g"], eps=mo.eps)
+        for l in range(mo.n_layers):
+            x = om.encoder_layer(x, W, l, mo)
+        h = om.layer_norm(x + W["head.type_table"][enc.qtype], W["enc.final_norm.g"], eps=mo.eps)
+        for i in range(2):
+            h = om.head_layer(h, W, i, mo)
+        hm = h[enc.mask_pos]
+        return dict(logits=om.scorer(hm, W, mo))
+
+
+class _HeadLayersSwapped(om.OracleModel):
+    def head(self, e, qtype):
+        h = e + self.W["head.type_table"][qtype]
+        for i in (1, 0):
+            h = om.head_layer(h, self.W, i, self.mo)
+        return h
+
+
+class _HeadLayerSkipped(om.OracleModel):
+    def head(self, e, qtype):
+        return om.head_layer(e + self.W["head.type_table"][qtype], self.W, 1, self.mo)
+
+
+class _UnnormedEncoderOutput(om.OracleModel):
+    def encode(self, ids):
+        W, mo = self.W, self.mo
+        x = om.layer_norm(W.embed_rows(ids), W["embed.norm.g"], eps=mo.eps)
+        for l in range(mo.n_layers):
+            x = om.encoder_layer(x, W, l, mo)
+        return x
+
+
+class _GatherShifted(om.OracleModel):
+    def forward_all(self, enc):
+        e = self.encode(enc.ids)
+        hm = self.head(e, enc.qtype)[np.asarray(enc.mask_pos) + 1]
+        return dict(logits=om.scorer(hm, self.W, self.mo))
+
+
+@pytest.mark.parametrize("planted", [_TypeRowBeforeFinalNorm, _HeadLayersSwapped, _HeadLayerSkipped,
+                                     _UnnormedEncoderOutput, _GatherShifted])
+def test_whole_model_composition_pin_catches_planted_mistakes(planted):
+    """Each plausible slip in the chain, planted in a copy of the oracle, moves
+    the logits far outside the closed form's tolerance."""
+    W = _composition_weights()
+    e = _composition_case()
+    ref = _composition_expected(W, e.ids, e.mask_pos, e.qtype)
+    z = planted(W, om.ModelOptions(n_layers=2, n_heads=2)).forward_all(e)["logits"]
+    assert np.abs(z - ref).max() > 1e-4
+
+
+def test_forward_all_and_logits_agree_on_the_47_token_row(oracle_model):
+    (r,) = rows_config0()
+    e = serialize_row(r, EncodeOptions())
+    out = oracle_model.forward_all(e)
+    np.testing.assert_array_equal(out["logits"], oracle_model.logits(e))
+    np.testing.assert_array_equal(out["marker_state"], oracle_model.hidden(e.ids, e.qtype)[e.mask_pos])
