@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=3)
+    ap.add_argument("--fp8-steps", type=int, default=3, help="profiled steps of the FP8-mode leg (0: skip)")
+    ap.add_argument("--long-rows", type=int, default=4,
+                    help="rows of the bounded long-context leg (8192 tokens each; 0: skip)")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
 
@@ -74,14 +77,17 @@ def workload(args, rank):
     return rows, opts, desc
 
 
-def algorithmic_cost(name, lens, n_markers, kper=None):
+def algorithmic_cost(name, lens, n_markers, kper=None, n_unique_ids=None):
     """(bytes, flops) per launch of kernel `name` for rows of lengths `lens`
-    (`kper`: options per row, needed for the marker attention)."""
+    (`kper`: options per row, needed for the marker attention; `n_unique_ids`:
+    distinct token ids of the batch, whose FP32 embedding rows are the gather's
+    compulsory reads -- a repeated id is an L2 hit, not a second HBM read)."""
     lens = np.asarray(lens, dtype=np.float64)
     T = lens.sum()
     M = float(n_markers)
     if name == "embed_ln":
-        return T * (4 + 1536 + 1536 + 768), T * 3 * D
+        U = T if n_unique_ids is None else float(n_unique_ids)
+        return T * 4 + U * 1536 + T * (1536 + 768), T * 3 * D
     if name in ("gemm_qkv_rope", "head0_gemm_in"):
         return T * (768 + 2304), T * 2 * D * 3 * D
     if name in ("gemm_wo_res_ln", "head0_gemm_out"):
@@ -108,11 +114,10 @@ def algorithmic_cost(name, lens, n_markers, kper=None):
         return M * (4 + 2 * (1536 + 768)), 0.0
     if name == "head1_marker_attn" and kper is not None:  # K,V of every row once; q in, o out
         return T * 1536 + M * (768 + 768), 4.0 * 64 * NH * float((np.asarray(kper, np.float64) * lens).sum())
-    if name == "scorer":  # FP32 marker states, the scorer weights, one logit per marker
-        return M * (1536 + 4) + 4 * (D * D + 4 * D + 1), M * (2 * D * D + 2 * D + 8 * D)
-    if name == "readout":  # logits in, probs out, four values per row
-        lens_b = len(lens)
-        return M * 8 + lens_b * (4 + 1 + 16), M * 4.0
+    if name == "head":  # FP32 marker states and the scorer weights in; logits, probs and read-outs out
+        nb = len(lens)
+        return (M * (1536 + 4 + 4) + 4 * (D * D + 4 * D + 1) + 4 * (nb + 1) + nb * (4 + 16),
+                M * (2 * D * D + 2 * D + 8 * D))
     return None
 
 
@@ -125,26 +130,40 @@ def read_peaks():
     return dict(hbm=6650.0, tc_burst=1590.0, tc_sust=1400.0, src="fallback")
 
 
-def kernel_source_sha():
-    """SHA-256 (first 16 hex digits) of the sources that decide what the GPU runs:
-    the kernels and their launch code (*.cu, *.cuh) and their shared declarations
-    (kernels.h).  The host-only serializer, router and API files are not part of
-    it: they launch nothing."""
+# The source file that defines each timed kernel (and its launcher); every kernel also
+# depends on the shared device headers.
+KERNEL_FILES = {"gemm": ("gemm.cu", "epilogue.cuh"), "attn_global": ("attention_tc.cu",),
+                "head0_attn": ("attention_tc.cu",), "attn_local": ("attention.cu",),
+                "head1_marker_attn": ("attention.cu",), "head": ("head.cu",)}
+SHARED_FILES = ("common.cuh", "kernels.h")
+
+
+def kernel_source_sha(kernel=None):
+    """SHA-256 (first 16 hex digits) of the sources that decide what the GPU runs.
+    kernel=None: every kernel and launcher (*.cu, *.cuh) and their shared
+    declarations (kernels.h); the host-only serializer, router and API files
+    launch nothing and are not part of it.  kernel=name: only the file that
+    defines that kernel (gemm.cu for every GEMM, small.cu for the bandwidth
+    kernels) and the shared device headers."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "encoder_decision_model_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")) or f == "kernels.h":
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    if kernel is None:
+        files = [f for f in sorted(os.listdir(csrc)) if f.endswith((".cu", ".cuh")) or f == "kernels.h"]
+    else:
+        own = KERNEL_FILES.get("gemm" if "gemm" in kernel else kernel, ("small.cu",))
+        files = sorted(set(own) | set(SHARED_FILES))
+    for f in files:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel, workload_tag):
     """DRAM bytes per token from a committed ncu summary, if its source hash
-    matches the current kernels (else None)."""
+    matches the kernel's current sources (else None)."""
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
         return None
-    sha = kernel_source_sha()
+    sha = kernel_source_sha(kernel)
     for f in sorted(os.listdir(pdir)):
         if not f.endswith(".md"):
             continue
@@ -329,7 +348,146 @@ def run_reference(args):
 
 
 ROUTER_KERNELS = ("embed_ln", "attn_local", "attn_global", "head0_attn", "head1_gather", "head1_marker_attn",
-                  "scorer", "readout")
+                  "head")
+ENCODER_GEMMS = ("gemm_qkv_rope", "gemm_wo_res_ln", "gemm_wi_geglu", "gemm_wo2_res_ln")
+
+
+def _r(x, n=4):
+    return None if x is None else float(f"{x:.{n}g}")
+
+
+def kernel_fractions(prof, steps, lens, n_markers, kper, n_unique_ids, peaks):
+    """Per kernel: launches and ms per step, and the fraction of the measured
+    HBM copy bandwidth and of the sustained BF16 tensor rate its algorithmic
+    bytes and FLOPs reach per launch (CUDA events on the launching stream)."""
+    out = {}
+    for name, (n, tot) in prof.items():
+        d = dict(launches_per_step=n // max(1, steps), ms_per_step=_r(tot / max(1, steps)))
+        c = algorithmic_cost(name, lens, n_markers, kper, n_unique_ids)
+        if c is not None and n:
+            a = tot / n / 1000.0
+            d["hbm_frac"] = _r(c[0] / a / 1e9 / peaks["hbm"], 3)
+            d["tensor_frac"] = _r(c[1] / a / 1e12 / peaks["tc_sust"], 3)
+        out[name] = d
+    return out
+
+
+def upload_batch(jl, hb, dev):
+    import torch
+    up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    keep = [up(hb.tokens), up(hb.cu_seqlens), up(hb.mask_pos), up(hb.opt_off), up(hb.row_type)]
+    batch = jl.Model.device_batch(hb.n_rows, hb.n_tokens, hb.n_markers, hb.max_row_len, *keep)
+    B, M = hb.n_rows, hb.n_markers
+    outs = dict(logits=torch.empty(M, device=dev), probs=torch.empty(M, device=dev),
+                choice=torch.empty(B, dtype=torch.int32, device=dev), score=torch.empty(B, device=dev),
+                noul=torch.empty(B, device=dev), max_p=torch.empty(B, device=dev))
+    return batch, outs, keep
+
+
+def profile_batch(jl, wpath, local, hb, steps, peaks, warmup=2, precision=None):
+    """Run one packed batch with per-kernel events; per-kernel fractions."""
+    import torch
+    dev = torch.device("cuda", local)
+    prec = jl.JD_PREC_BF16 if precision is None else precision
+    m = jl.Model(wpath, hb.n_tokens, hb.n_rows, hb.n_markers, precision=prec, device=local)
+    batch, outs, keep = upload_batch(jl, hb, dev)
+    st = torch.cuda.Stream(device=dev)
+    for _ in range(warmup):
+        m.jd_decide(batch, **outs, stream=st)
+    torch.cuda.synchronize()
+    m.jd_check_status()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        m.jd_decide(batch, **outs, stream=st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    m.jd_set_profiling(True)
+    for _ in range(steps):
+        m.jd_decide(batch, **outs, stream=st)
+    prof = m.jd_profile_report()
+    m.jd_set_profiling(False)
+    torch.cuda.synchronize()
+    m.jd_check_status()
+    m.close()
+    lens = np.diff(hb.cu_seqlens)
+    pk = kernel_fractions(prof, steps, lens, hb.n_markers, np.diff(hb.opt_off), len(np.unique(hb.tokens)), peaks)
+    return ms, pk
+
+
+def measure_long(jl, wpath, local, rows, steps, peaks):
+    """A bounded leg of the long-context workload (rows of exactly 8192 tokens,
+    20 options capped to the 256-token head budget, non-strict): decisions/s and
+    the per-kernel fractions, the encoder GEMMs' share of the tensor peak first."""
+    from workloads import rows_config3
+    r = rows_config3(rows, seed=103)
+    hb = jl.jd_serialize(r, jl.encode_opts(8192, 256, False))
+    ms, pk = profile_batch(jl, wpath, local, hb, steps, peaks)
+    return {"workload": f"long context: {rows} rows x 8192 tokens (20 options capped to the 256-token head "
+                        "budget, non-strict), choice/score", "rows": int(hb.n_rows), "tokens": int(hb.n_tokens),
+            "decisions_per_s": _r(hb.n_rows / (ms / 1000.0)), "ms_per_batch": _r(ms),
+            "encoder_gemm_tensor_frac": {k: pk[k].get("tensor_frac") for k in ENCODER_GEMMS if k in pk},
+            "encoder_gemm_hbm_frac": {k: pk[k].get("hbm_frac") for k in ENCODER_GEMMS if k in pk},
+            "per_kernel": pk}
+
+
+def measure_fp8(jl, wpath, local, hb, steps, peaks):
+    """The same batch with the encoder QKV projections on E4M3 operands (JD_PREC_FP8):
+    decisions/s and the QKV kernel against the FP8 dense peak, taken as twice the measured
+    BF16 one (the tensor cores' nominal FP8 / BF16 ratio)."""
+    ms, pk = profile_batch(jl, wpath, local, hb, steps, peaks, precision=jl.JD_PREC_FP8)
+    q = dict(pk.get("gemm_qkv_rope", {}))
+    if "tensor_frac" in q:
+        q["tensor_frac_of_fp8_peak"] = _r(q["tensor_frac"] / 2.0, 3)
+    return {"precision": "E4M3 encoder QKV projections, everything else as the BF16 line",
+            "decisions_per_s": _r(hb.n_rows / (ms / 1000.0)), "ms_per_step": _r(ms), "gemm_qkv_rope": q,
+            "fp8_peak_tflops": _r(2.0 * peaks["tc_sust"]), "per_kernel": pk}
+
+
+def measure_latency(jl, wpath, local, calls, n_distinct=128):
+    """Batch-1 latency of the 3-question request (choice/4, score/3, noul/2 on one
+    200-token state) through jd_decide_host, host serialisation and copies included.
+    `distinct`: a pool of `n_distinct` seeded requests of that recipe (questions
+    8..24 ids, options 3..20 ids, so each has its own length), called in turn;
+    eager launches and CUDA-graph mode side by side.  `repeated`: one request
+    called over and over in graph mode (every call replays the same graph)."""
+    from workloads import rows_config1
+    o1 = jl.encode_opts(1024, 512, True)
+    pool = [rows_config1(seed=101 + k) for k in range(n_distinct)]
+    lm = jl.Model(wpath, 2048, 8, 64, precision=jl.JD_PREC_BF16, device=local)
+
+    def run(graph, reqs):
+        lm.jd_set_graph_mode(graph)
+        for k in range(20):
+            lm.jd_decide_host(reqs[k % len(reqs)], o1)
+        ts = []
+        for k in range(calls):
+            t = time.perf_counter()
+            lm.jd_decide_host(reqs[k % len(reqs)], o1)
+            ts.append(1000 * (time.perf_counter() - t))
+        return {"p50_ms": _r(float(np.percentile(ts, 50))), "p99_ms": _r(float(np.percentile(ts, 99)))}
+
+    out = {"distinct_eager": run(False, pool), "distinct_graph": run(True, pool),
+           "repeated_graph": run(True, pool[:1])}
+    lm.jd_set_graph_mode(False)
+    # per-kernel device time of one call (events around every launch; these calls synchronise)
+    n_prof = 50
+    lm.jd_set_profiling(True)
+    for k in range(n_prof):
+        lm.jd_decide_host(pool[k % len(pool)], o1)
+    prof = lm.jd_profile_report()
+    lm.jd_set_profiling(False)
+    lm.close()
+    out["per_kernel_us_per_call"] = {k: _r(1000.0 * ms / n_prof) for k, (n, ms) in
+                                     sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    out["timed_launch_groups_per_call"] = int(sum(n for n, _ in prof.values()) // n_prof)
+    out["device_us_per_call"] = _r(1000.0 * sum(ms for _, ms in prof.values()) / n_prof)
+    best = min(("distinct_eager", "distinct_graph"), key=lambda k: out[k]["p50_ms"])
+    out["reported"] = best
+    out["workload"] = (f"{n_distinct} distinct 3-question requests (choice/4, score/3, noul/2) on a 200-token "
+                       "state, called in turn through jd_decide_host (serialise + H2D + forward + D2H + sync)")
+    return out
 
 
 def measure_serving(jl, wpath, local, seconds, thread_counts=(1, 2, 4)):
@@ -373,13 +531,14 @@ def measure_serving(jl, wpath, local, seconds, thread_counts=(1, 2, 4)):
             t.join()
         el = time.perf_counter() - t0
         allv = np.concatenate([np.asarray(v) for v in lat])
-        out.append({"threads": n, "requests_per_s": float(len(allv) / el),
-                    "p50_ms_per_call": float(np.percentile(allv, 50)), "p99_ms_per_call": float(np.percentile(allv, 99))})
+        out.append({"threads": n, "requests_per_s": _r(float(len(allv) / el)),
+                    "p50_ms_per_call": _r(float(np.percentile(allv, 50))),
+                    "p99_ms_per_call": _r(float(np.percentile(allv, 99)))})
         for h in handles:
             h.jd_check_status()
             h.close()
     base.close()
-    return {"workload": "3 questions (choice/4, score/3, noul/2) on one 200-token state per request, "
+    return {"workload": "one 3-question request (choice/4, score/3, noul/2, 200-token state) repeated, "
                         "each thread its own shared handle and stream, CUDA-graph replay, host work included",
             "results": out}
 
@@ -391,7 +550,6 @@ def measure_router(jl, wpath, local, rank, ranks, reps, peaks):
     of jd_route_host (serialisation, both forward rounds, survivor rule, copies).
     Round 1 is also run alone with per-kernel events to give the HBM fraction of
     the attention, norm and gather kernels at this shape."""
-    import torch
     from workloads import Row, requests_config4
     reqs = requests_config4(512, seed=104 + 1000 * rank)
     opts = jl.encode_opts(1024, 512, True)
@@ -404,47 +562,44 @@ def measure_router(jl, wpath, local, rank, ranks, reps, peaks):
         out = m.jd_route_host(reqs, opts)
     el = ranks.max(time.perf_counter() - t0)
     total = ranks.sum(float(len(reqs) * reps))
+    m.jd_check_status()
+    m.close()
 
     rows = [Row(state=q.state, question=q.question, options=q.labels[g:g + 20], qtype=0)
             for q in reqs for g in range(0, len(q.labels), 20)]
     hb = jl.jd_serialize(rows, opts)
-    dev = torch.device("cuda", local)
-    up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-    keep = [up(hb.tokens), up(hb.cu_seqlens), up(hb.mask_pos), up(hb.opt_off), up(hb.row_type)]
-    B, M, T = hb.n_rows, hb.n_markers, hb.n_tokens
-    batch = jl.Model.device_batch(B, T, M, hb.max_row_len, *keep)
-    outs = dict(logits=torch.empty(M, device=dev), probs=torch.empty(M, device=dev),
-                choice=torch.empty(B, dtype=torch.int32, device=dev), score=torch.empty(B, device=dev),
-                noul=torch.empty(B, device=dev), max_p=torch.empty(B, device=dev))
-    st = torch.cuda.Stream(device=dev)
-    m.jd_decide(batch, **outs, stream=st)
-    torch.cuda.synchronize()
-    m.jd_set_profiling(True)
-    for _ in range(3):
-        m.jd_decide(batch, **outs, stream=st)
-    prof = m.jd_profile_report()
-    m.jd_set_profiling(False)
-    torch.cuda.synchronize()
-    m.jd_check_status()
-    m.close()
-    lens = np.diff(hb.cu_seqlens)
-    r1 = {}
-    for name, (n, tot) in prof.items():
-        d = dict(launches=n // 3, ms=tot / 3)
-        c = algorithmic_cost(name, lens, M, np.diff(hb.opt_off))
-        if c is not None and n:
-            a = tot / n / 1000.0
-            d["hbm_frac"] = c[0] / a / 1e9 / peaks["hbm"]
-            d["tensor_frac"] = c[1] / a / 1e12 / peaks["tc_sust"]
-        r1[name] = d
+    ms, r1 = profile_batch(jl, wpath, local, hb, 3, peaks)
     return {"workload": "512 requests x 72 labels of 3..12 ids on a 256-id state; groups of <=20, then one "
                         "final row of the survivors; head budget 512, max_length 1024, strict",
-            "value": total / el, "unit": "requests/s", "ms_per_call": 1000 * el / reps,
+            "value": _r(total / el), "unit": "requests/s", "ms_per_call": _r(1000 * el / reps),
             "rows_per_round": [int(x) for x in out["rows_per_round"]],
-            "round1": {"rows": int(B), "tokens": int(T), "markers": int(M),
-                       "ms_forward": sum(v["ms"] for v in r1.values()),
-                       "hbm_bound_kernels": {k: r1[k] for k in ROUTER_KERNELS if k in r1},
-                       "per_kernel": r1}}
+            "round1": {"rows": int(hb.n_rows), "tokens": int(hb.n_tokens), "markers": int(hb.n_markers),
+                       "ms_forward": _r(ms),
+                       "hbm_bound_kernels": {k: r1[k] for k in ROUTER_KERNELS if k in r1}}}
+
+
+def roofline_line(name, n, tot, cost, peaks, workload_tag, T):
+    """The roofline object of one kernel from its event totals (n launches, tot ms)."""
+    avg_s = tot / n / 1000.0
+    byt, fl = cost
+    t_hbm = byt / (peaks["hbm"] * 1e9)
+    t_tc = fl / (peaks["tc_sust"] * 1e12)
+    tr = recorded_traffic(name, workload_tag)
+    if t_tc > t_hbm:
+        ach = fl / avg_s / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["tc_sust"], "unit": "TFLOP/s",
+                "frac": ach / peaks["tc_sust"], "traffic": None if tr is None else tr * T,
+                "kernel": name, "peak_source": f"{peaks['src']} sustained bf16 (cuBLAS)",
+                "peak_burst": peaks["tc_burst"], "frac_of_burst": ach / peaks["tc_burst"]}
+    else:
+        ach = byt / avg_s / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": ach / peaks["hbm"], "traffic": None if tr is None else tr * T,
+                "kernel": name, "peak_source": f"{peaks['src']} copy bandwidth"}
+    roof["algorithmic_per_launch"] = {"bytes": byt, "flops": fl}
+    roof["avg_launch_ms"] = avg_s * 1000.0
+    roof["kernel_source_sha"] = kernel_source_sha(name)
+    return roof
 
 
 def run_ours(args):
@@ -477,6 +632,7 @@ def run_ours(args):
     hb = jl.jd_serialize(rows, jl.encode_opts(**opts))
     T, B, M = hb.n_tokens, hb.n_rows, hb.n_markers
     lens = np.diff(hb.cu_seqlens)
+    n_unique = len(np.unique(hb.tokens))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -486,12 +642,7 @@ def run_ours(args):
         cpu["threads_4"] = oracle_four_threads(rows, opts, args.cpu_seconds)
 
     model = jl.Model(weights_path(0), T, B, M, precision=jl.JD_PREC_BF16, device=local)
-    up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-    keep = [up(hb.tokens), up(hb.cu_seqlens), up(hb.mask_pos), up(hb.opt_off), up(hb.row_type)]
-    batch = jl.Model.device_batch(B, T, M, hb.max_row_len, *keep)
-    outs = dict(logits=torch.empty(M, device=dev), probs=torch.empty(M, device=dev),
-                choice=torch.empty(B, dtype=torch.int32, device=dev), score=torch.empty(B, device=dev),
-                noul=torch.empty(B, device=dev), max_p=torch.empty(B, device=dev))
+    batch, outs, keep = upload_batch(jl, hb, dev)
     stream = torch.cuda.Stream(device=dev)
 
     def step():
@@ -545,74 +696,55 @@ def run_ours(args):
     e2e_val = sum_over_ranks(float(B * e2e_steps)) / e2e_s
     h2d = 4 * (T + (B + 1) + M + (B + 1) + B)
     d2h = 4 * (2 * M + 4 * B)
+    model.close()
 
-    # ---- batch-1 latency: the 3-question request on one 200-token state, graph replay
+    peaks = read_peaks()
+    # ---- batch-1 latency over distinct requests, eager and graph side by side
     lat = {}
+    latency = None
     if rank == 0 and args.latency_calls > 0:
-        from workloads import rows_config1
-        r1 = rows_config1()
-        o1 = jl.encode_opts(1024, 512, True)
-        lm = jl.Model(weights_path(0), 2048, 8, 64, precision=jl.JD_PREC_BF16, device=local)
-        lm.jd_set_graph_mode(True)
-        for _ in range(20):
-            lm.jd_decide_host(r1, o1)
-        ts = []
-        for _ in range(args.latency_calls):
-            t = time.perf_counter()
-            lm.jd_decide_host(r1, o1)
-            ts.append(1000 * (time.perf_counter() - t))
-        lat = dict(p50_ms_per_call=float(np.percentile(ts, 50)), p99_ms_per_call=float(np.percentile(ts, 99)),
-                   latency_workload="3 questions (choice/4, score/3, noul/2) on one 200-token state, "
-                                    "jd_decide_host with CUDA-graph replay, host serialisation and copies included")
-        lm.close()
+        latency = measure_latency(jl, weights_path(0), local, args.latency_calls)
+        best = latency[latency["reported"]]
+        lat = dict(p50_ms_per_call=best["p50_ms"], p99_ms_per_call=best["p99_ms"])
 
     serving = None
     if rank == 0 and args.serve_seconds > 0:
         serving = measure_serving(jl, weights_path(0), local, args.serve_seconds)
 
     # ---- router: 512 requests x 72 labels, both rounds and the host work between them
-    peaks = read_peaks()
     router = None
     if args.router_reps > 0:
         router = measure_router(jl, weights_path(0), local, rank, ranks, args.router_reps, peaks)
 
+    # ---- bounded long-context leg (rows of 8192 tokens)
+    long_leg = None
+    if rank == 0 and args.long_rows > 0 and args.workload == "throughput":
+        long_leg = measure_long(jl, weights_path(0), local, args.long_rows, 3, peaks)
+
+    # ---- the same batch in FP8 mode (E4M3 encoder QKV projections)
+    fp8 = None
+    if rank == 0 and args.fp8_steps > 0:
+        fp8 = measure_fp8(jl, weights_path(0), local, hb, args.fp8_steps, peaks)
+
     # ---- roofline of the dominant kernel
     roof = None
-    per_kernel = {}
-    for name, (n, tot) in prof.items():
-        per_kernel[name] = dict(launches_per_step=n // max(1, args.profile_steps), ms_per_step=tot / args.profile_steps)
+    per_kernel = kernel_fractions(prof, args.profile_steps, lens, M, np.diff(hb.opt_off), n_unique, peaks) \
+        if prof else {}
     if prof:
         top = max(prof, key=lambda k: prof[k][1])
         n, tot = prof[top]
-        avg_s = tot / n / 1000.0
-        cost = algorithmic_cost(top, lens, M, np.diff(hb.opt_off))
+        cost = algorithmic_cost(top, lens, M, np.diff(hb.opt_off), n_unique)
         if cost is not None:
-            byt, fl = cost
-            t_hbm = byt / (peaks["hbm"] * 1e9)
-            t_tc = fl / (peaks["tc_sust"] * 1e12)
-            wl_tag = args.workload
-            tr = recorded_traffic(top, wl_tag)
-            if t_tc > t_hbm:
-                ach = fl / avg_s / 1e12
-                roof = {"bound": "tensor", "achieved": ach, "peak": peaks["tc_sust"], "unit": "TFLOP/s",
-                        "frac": ach / peaks["tc_sust"], "traffic": None if tr is None else tr * T,
-                        "kernel": top, "peak_source": f"{peaks['src']} sustained bf16 (cuBLAS)"}
-            else:
-                ach = byt / avg_s / 1e9
-                roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
-                        "frac": ach / peaks["hbm"], "traffic": None if tr is None else tr * T,
-                        "kernel": top, "peak_source": f"{peaks['src']} copy bandwidth"}
-            roof["algorithmic_per_launch"] = {"bytes": byt, "flops": fl}
-            roof["avg_launch_ms"] = avg_s * 1000.0
-            roof["kernel_source_sha"] = kernel_source_sha()
-        for name, d in per_kernel.items():
-            c = algorithmic_cost(name, lens, M, np.diff(hb.opt_off))
-            if c is None or d["launches_per_step"] == 0:
-                continue
-            a = d["ms_per_step"] / d["launches_per_step"] / 1000.0
-            d["hbm_frac"] = c[0] / a / 1e9 / peaks["hbm"]
-            d["tensor_frac"] = c[1] / a / 1e12 / peaks["tc_sust"]
+            roof = roofline_line(top, n, tot, cost, peaks, args.workload, T)
 
+    targets = {"peaks": {k: peaks[k] for k in ("hbm", "tc_sust", "tc_burst", "src")}}
+    if long_leg:
+        targets["long_encoder_gemm_tensor_frac"] = long_leg["encoder_gemm_tensor_frac"]
+    if fp8:
+        targets["fp8_qkv_tensor_frac_of_fp8_peak"] = fp8["gemm_qkv_rope"].get("tensor_frac_of_fp8_peak")
+    if router:
+        targets["router_round1_hbm_frac"] = {k: v.get("hbm_frac") for k, v in
+                                             router["round1"]["hbm_bound_kernels"].items()}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -628,13 +760,13 @@ def run_ours(args):
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "call": "jd_decide_host (serialise + H2D from pinned staging + forward + D2H + sync)"},
             "gpu_launches": int(launches_per_step * args.steps),
-            "clocks": ck, "per_kernel": per_kernel, "router": router, "concurrent_serving": serving}
+            "clocks": ck, "per_kernel": per_kernel, "latency": latency, "concurrent_serving": serving,
+            "router": router, "long_context": long_leg, "fp8": fp8, "targets": targets}
     if rank == 0:
         s = json.dumps(line)
         print(s, flush=True)
         if args.json_out:
             open(args.json_out, "w").write(s + "\n")
-    model.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -62,3 +62,13 @@ def test_marker_attention_cost():
     assert b == sum(lens) * 2 * 768 + M * 2 * 768
     # every marker attends to every key of its row
     assert f == 4 * DH * H * sum(k * L for k, L in zip(kper, lens))
+
+
+def test_embedding_reads_count_distinct_ids():
+    """The gather's compulsory reads are one FP32 embedding row per distinct id (a
+    repeated id is served from L2); its writes are one FP32 and one BF16 row per token."""
+    T = sum(LENS)
+    b, _ = bench.algorithmic_cost("embed_ln", LENS, 0, n_unique_ids=100)
+    assert b == T * 4 + 100 * 1536 + T * (1536 + 768)
+    b_all, _ = bench.algorithmic_cost("embed_ln", LENS, 0, n_unique_ids=T)
+    assert b_all == T * (4 + 1536 + 1536 + 768)
