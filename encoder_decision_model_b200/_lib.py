@@ -17,7 +17,7 @@ LIB_PATH = Path(__file__).resolve().parent / "libjulia_decide.so"
 
 JD_OK, JD_ERR_INVALID_ARG, JD_ERR_OPTION_COUNT, JD_ERR_OVERFLOW, JD_ERR_TOKEN_RANGE = 0, 1, 2, 3, 4
 JD_ERR_CAPACITY, JD_ERR_CUDA, JD_ERR_DEVICE_STATUS, JD_ERR_IO = 5, 6, 7, 8
-JD_PREC_BF16, JD_PREC_FP32 = 0, 1
+JD_PREC_BF16, JD_PREC_FP32, JD_PREC_FP8 = 0, 1, 2
 JD_SCORER_MLP, JD_SCORER_LINEAR = 0, 1
 JD_ACT_RELU, JD_ACT_GELU = 0, 1
 
@@ -122,6 +122,8 @@ def lib():
     L.jd_route_host.restype = C.c_int
     L.jd_forward_noalloc.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.c_void_p, C.c_void_p]
     L.jd_forward_noalloc.restype = C.c_int
+    L.jd_noalloc_check_status.argtypes = [C.c_void_p, C.c_void_p]
+    L.jd_noalloc_check_status.restype = C.c_int
     L.jd_last_launch_count.argtypes = [C.c_void_p]
     L.jd_last_launch_count.restype = C.c_int32
     L.jd_set_profiling.argtypes = [C.c_void_p, C.c_int]
@@ -432,6 +434,11 @@ class Model:
         """jd_forward with every intermediate in the library's static device
         array (no allocation); at most 1024 tokens, 32 rows, 128 markers."""
         _check(lib().jd_forward_noalloc(self.h, C.byref(batch), _ptr(logits), _stream(stream)))
+
+    def jd_noalloc_check_status(self, stream=None):
+        """Synchronize `stream` and raise JDError if the last jd_forward_noalloc
+        call's kernels recorded a failed check."""
+        _check(lib().jd_noalloc_check_status(self.h, _stream(stream)))
 
     def jd_check_status(self):
         _check(lib().jd_check_status(self.h))

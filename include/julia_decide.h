@@ -119,7 +119,19 @@ typedef struct {
     float *marker_state;  /* [M, 384] marker states after both head layers (scorer input) */
 } jd_taps;
 
-enum { JD_PREC_BF16 = 0, JD_PREC_FP32 = 1 };
+/* Precision of jd_model_config.precision.
+ *   JD_PREC_BF16  BF16 tensor-core projections and attention, FP32 accumulation, FP32 residual
+ *                 stream, norms, embedding, scorer and read-outs ("Julia-1 MLX", "Performance":
+ *                 the projections may run at lower precision, the residual stream stays FP32).
+ *   JD_PREC_FP32  FP32 everywhere (validation mode).
+ *   JD_PREC_FP8   JD_PREC_BF16 with the QKV projections of the 22 encoder layers on FP8 E4M3
+ *                 operands (tensor-core kind::f8f6f4, FP32 accumulation): each weight row has
+ *                 its own scale (max |row| / 448), and each layer's normalized input one static
+ *                 scale, sqrt(384) * max |gain| / 448, the bound of a LayerNorm output, so it
+ *                 never saturates.  Every other projection stays BF16: E4M3 inputs of the GEGLU
+ *                 up-projection carry their 3-bit mantissa error into residual channels that a
+ *                 later projection scales to the thousands the page describes. */
+enum { JD_PREC_BF16 = 0, JD_PREC_FP32 = 1, JD_PREC_FP8 = 2 };
 enum { JD_SCORER_MLP = 0, JD_SCORER_LINEAR = 1 };
 enum { JD_ACT_RELU = 0, JD_ACT_GELU = 1 };
 
@@ -127,9 +139,8 @@ typedef struct {
     int32_t max_tokens;    /* capacity: packed tokens per call */
     int32_t max_rows;      /* capacity: rows per call */
     int32_t max_markers;   /* capacity: markers per call */
-    int32_t precision;     /* JD_PREC_BF16: BF16 tensor-core GEMMs / attention with FP32
-                              accumulation and an FP32 residual stream;
-                              JD_PREC_FP32: FP32 everywhere (validation mode) */
+    int32_t precision;     /* JD_PREC_BF16, JD_PREC_FP32 (validation mode) or JD_PREC_FP8
+                              (E4M3 encoder QKV projections); see the enum above */
     int32_t scorer;        /* JD_SCORER_MLP: LayerNorm -> Linear(384,384) -> GELU -> Linear(384,1)
                               ("The decision head", step 4); JD_SCORER_LINEAR: LayerNorm -> Linear(384,1) */
     int32_t head_act;      /* feed-forward activation of the two head layers (default ReLU) */
@@ -334,16 +345,29 @@ jd_status jd_profile_report(jd_model *model, char *buf, size_t n);
  * that each GPU loading the library holds until the process exits.
  *   - Limits: at most 1024 packed tokens, 32 rows and 128 markers per call
  *     (JD_ERR_CAPACITY beyond them); BF16 models only (JD_ERR_INVALID_ARG).
- *   - The first call on a device resolves the array's device address and
- *     describes its buffers for TMA; make that first call before any stream
- *     capture.
+ *   - jd_model_create (BF16) loads the module holding the array, resolves its
+ *     device address and describes its buffers for TMA, so that this entry
+ *     point allocates nothing from its first call on.  The model (weights)
+ *     must therefore come from jd_model_create, called at start-up.
  *   - All calls share the array, and each call leaves its intermediates there:
  *     calls whose work overlaps on the GPU (different streams, or models on
  *     the same device used concurrently) race and must be serialized by the
- *     caller.  The status word the kernels write is cleared at the start of
- *     every call; it is not reported by jd_check_status.
- *   - The model (weights) must come from jd_model_create, called at start-up. */
+ *     caller.
+ *   - The kernels' device status word (an id outside the vocabulary, a marker
+ *     index outside the batch, a bounded wait that expired) lives in the array
+ *     too and is cleared at the start of every call: read it with
+ *     jd_noalloc_check_status after the call and before the next one.
+ *     jd_check_status does not cover these calls. */
 jd_status jd_forward_noalloc(jd_model *model, const jd_batch *batch, float *logits, void *stream);
+
+/* Status of the last jd_forward_noalloc call on the model's device (no
+ * counterpart on the pages): synchronizes `stream` (the call's stream), reads
+ * the array's device status word (a copy into host memory; nothing is
+ * allocated) and returns JD_ERR_DEVICE_STATUS with a message when a kernel
+ * recorded a failed check, JD_OK otherwise.  The logits of a call that
+ * reports a failure are not meaningful.  Errors: JD_ERR_INVALID_ARG (NULL
+ * model, FP32 model), JD_ERR_CUDA (the synchronization or copy failed). */
+jd_status jd_noalloc_check_status(jd_model *model, void *stream);
 
 #ifdef __cplusplus
 }
