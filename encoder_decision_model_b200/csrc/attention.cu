@@ -244,7 +244,10 @@ __global__ void __launch_bounds__(128)
 // [q0 - 64, q0 + 128), loaded once by TMA (three 64 x 64 tiles of K and of V);
 // warp w's 16 queries need only the 144 keys [q0 + 16w - 64, q0 + 16w + 80),
 // i.e. nine 16-key chunks, so each warp visits just those and runs an exact
-// two-pass softmax over them in registers (no running rescale).
+// two-pass softmax over them in registers (no running rescale).  A CTA finds
+// its row in the prep kernel's table of the row of every 64-query block (tb_row)
+// with one load: the binary search over the row offsets it replaced cost about
+// a fifth of the kernel's time (a chain of dependent L2 loads per CTA).
 constexpr int LW_CHUNKS = 9;  // (16 + 2 * 64) / 16
 // Two heads per CTA (8 warps, 2 CTAs per SM): 16 resident warps per SM instead of 12.
 constexpr int LOC_HEADS = 2;
@@ -255,7 +258,8 @@ constexpr int LOC_SMEM = LOC_HEADS * LOC_HEAD_BYTES + 1024;
 
 __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
     k_attn_local_bf16(const __grid_constant__ CUtensorMap tm, __nv_bfloat16 *__restrict__ out,
-                      const int *__restrict__ cu, const int *__restrict__ qb_off, int n_rows, unsigned *status) {
+                      const int *__restrict__ cu, const int *__restrict__ qb_off, const int *__restrict__ tb_row,
+                      int n_rows, unsigned *status) {
     extern __shared__ __align__(16) uint8_t sm_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 8 * LOC_HEADS + 1023) &
                                               ~uintptr_t(1023));
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
 
     const int tile = blockIdx.x, h = blockIdx.y * LOC_HEADS + hh;
     if (tile >= qb_off[n_rows]) return;
-    const int row = find_row(qb_off, n_rows, tile);
+    const int row = tb_row[tile];
     const int cs = cu[row], ce = cu[row + 1];
     const int q0 = cs + (tile - qb_off[row]) * BQ;
     const int kbase = q0 - 64;         // band start (may precede the row: masked)
@@ -318,7 +322,8 @@ __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
     // Masks on the raw scores; the scale goes into the exponent's FMA below.  Key kj of 8-column
     // block j lies kj - qi = 8j - 64 + (2tq + e) - g (- 8 for qi1) from the query, which is inside
     // [-63, 63] for 2 <= j < 16: only the two outer chunks at each end need the window test.
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+    // four interleaved partial maxima per query row: dependency chains of 9, not 36
+    float mp0[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, mp1[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
     for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
         const bool edge = j < 2 || j >= 2 * LW_CHUNKS - 2;
@@ -330,26 +335,29 @@ __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
             const bool v1 = in_row && (!edge || abs(qi1 - kj) <= 64);
             sc[j][e] = v0 ? sc[j][e] : -INFINITY;
             sc[j][2 + e] = v1 ? sc[j][2 + e] : -INFINITY;
-            mx0 = fmaxf(mx0, sc[j][e]);
-            mx1 = fmaxf(mx1, sc[j][2 + e]);
+            mp0[(2 * j + e) & 3] = fmaxf(mp0[(2 * j + e) & 3], sc[j][e]);
+            mp1[(2 * j + e) & 3] = fmaxf(mp1[(2 * j + e) & 3], sc[j][2 + e]);
         }
     }
+    float mx0 = fmaxf(fmaxf(mp0[0], mp0[1]), fmaxf(mp0[2], mp0[3]));
+    float mx1 = fmaxf(fmaxf(mp1[0], mp1[1]), fmaxf(mp1[2], mp1[3]));
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
     const float mu0 = mx0 == -INFINITY ? 0.f : -mx0 * sl2, mu1 = mx1 == -INFINITY ? 0.f : -mx1 * sl2;
-    float l0 = 0.f, l1 = 0.f;
+    float lp0[2] = {0.f, 0.f}, lp1[2] = {0.f, 0.f};  // two interleaved partial sums per row
     uint32_t pa[LW_CHUNKS][4];
 #pragma unroll
     for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
         const float p0 = ex2_ftz(fmaf(sc[j][0], sl2, mu0)), p1 = ex2_ftz(fmaf(sc[j][1], sl2, mu0));
         const float p2 = ex2_ftz(fmaf(sc[j][2], sl2, mu1)), p3 = ex2_ftz(fmaf(sc[j][3], sl2, mu1));
-        l0 += p0 + p1;
-        l1 += p2 + p3;
+        lp0[j & 1] += p0 + p1;
+        lp1[j & 1] += p2 + p3;
         pa[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p0, p1);
         pa[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p2, p3);
     }
+    float l0 = lp0[0] + lp0[1], l1 = lp1[0] + lp1[1];
     float o[8][4];
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
@@ -489,7 +497,8 @@ cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st) {
         const int smem = 5 * 8192 + 64 + 1024;
         if (local && a.window == 64)
             k_attn_local_bf16<<<dim3(max_tiles, NH / LOC_HEADS), 128 * LOC_HEADS, LOC_SMEM, st>>>(
-                *a.tm_qkv, (__nv_bfloat16 *)a.o, a.cu_seqlens, a.qb_off, a.n_rows, a.status);
+                *a.tm_qkv, (__nv_bfloat16 *)a.o, a.cu_seqlens, a.qb_off,
+                a.qb_off + qb_row64_offset(a.n_rows, a.n_tokens), a.n_rows, a.status);
         else if (local)
             k_attn_bf16<true><<<grid, 128, smem, st>>>(*a.tm_qkv, (__nv_bfloat16 *)a.o, a.cu_seqlens, a.qb_off,
                                                        a.n_rows, a.window, a.status);

@@ -73,6 +73,57 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// Packed FP32 pairs on the FMA pipe (sm_100 f32x2 forms: one instruction per pair).
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// 2^x for a pair, on the FMA and integer pipes instead of the special-function unit.
+// x = j + f with j = round(x) and f in [-1/2, 1/2]: adding 1.5 * 2^23 leaves j in the low
+// mantissa bits of t (|x| < 2^22), so t - 1.5 * 2^23 is j exactly and f = x - j exactly.
+// 2^f is the degree-3 polynomial of least maximum relative error on [-1/2, 1/2], found by
+// the Remez exchange algorithm (|p(f) / 2^f - 1| <= 7.5e-5; the bf16 rounding P receives
+// is 2^-9 = 2.0e-3), and 2^j enters as j added to p's exponent field (bits(t) << 23 is
+// j << 23: the constant's own bits shift out).  x is clamped at -126, so the masked keys
+// (x = -inf) give 2^-126 ~ 1e-38 for 0, still a normal float.
+constexpr float EX2_C0 = 0.9999280571937561f, EX2_C1 = 0.6932609677314758f, EX2_C2 = 0.2426111251115799f,
+                EX2_C3 = 0.0551716685295105f;
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float &y0, float &y1) {
+    const float2 x = make_float2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const float2 t = add2(x, make_float2(12582912.f, 12582912.f));
+    const float2 j = add2(t, make_float2(-12582912.f, -12582912.f));
+    const float2 f = add2(x, make_float2(-j.x, -j.y));
+    float2 p = fma2(f, make_float2(EX2_C3, EX2_C3), make_float2(EX2_C2, EX2_C2));
+    p = fma2(p, f, make_float2(EX2_C1, EX2_C1));
+    p = fma2(p, f, make_float2(EX2_C0, EX2_C0));
+    y0 = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
+    y1 = __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
+}
+
+// Of every eight key pairs a softmax thread exponentiates, this many take the polynomial
+// above and the rest the special-function unit.  Measured on the throughput and long-row
+// workloads, 2, 3 or 4 of 8 ran no faster than 0 (the softmax warps are bound by issued
+// instructions, not by the special-function unit alone), so the default is 0; the build
+// option stays for other shapes.
+#ifndef JD_EX2_POLY_OF8
+#define JD_EX2_POLY_OF8 0
+#endif
+
 // D[tmem] (+)= A[tmem] * B[smem]: A is M x K in TMEM (lane = row, two bf16 per column)
 __device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                                uint32_t accumulate) {
@@ -244,6 +295,34 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             const int qi = t.q0 + x * TQ + r;
             const bool pp = t.nx == 2;  // both groups busy: alternate the exponential phases
             if (pp) named_bar_sync(BAR_ITEM, 256);
+            // A warp whose 32 query rows all lie past the row's end (the tail of a short row's
+            // last tile) reads nothing of S, P or O: it keeps every wait and arrival of the
+            // pipeline, so the barrier phases stay those of the other warps, and skips the math.
+            if (t.q0 + x * TQ + (warp & 3) * 32 >= t.ce) {
+                for (int j = 0; j < t.nt; ++j, ++c) {
+                    mbar_wait(&sfull[x], c & 1, status);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sfree[x]);
+                    if (pp) {
+                        if (x == 0) {
+                            if (j != 0) named_bar_sync(BAR_G1_DONE, 256);
+                        } else {
+                            named_bar_sync(BAR_G0_DONE, 256);
+                        }
+                    }
+                    if (j != 0) mbar_wait(&pvdone[x], (c - 1) & 1, status);
+                    if (pp) {
+                        if (x == 0) named_bar_arrive(BAR_G0_DONE, 256);
+                        else if (j != t.nt - 1) named_bar_arrive(BAR_G1_DONE, 256);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pready[x]);
+                }
+                mbar_wait(&pvdone[x], (c - 1) & 1, status);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ofree[x]);
+                continue;
+            }
             float m = -INFINITY, l = 0.f;
             for (int j = 0; j < t.nt; ++j, ++c) {
                 const int k0 = t.cs + j * TK;
@@ -306,8 +385,15 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     uint32_t pk[32];
 #pragma unroll
                     for (int e = 0; e < 64; e += 2) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[64 * hk + e]), sl2, -m));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[64 * hk + e + 1]), sl2, -m));
+                        const float2 xv = fma2(make_float2(__uint_as_float(sv[64 * hk + e]), __uint_as_float(sv[64 * hk + e + 1])),
+                                               make_float2(sl2, sl2), make_float2(-m, -m));
+                        float p0, p1;
+                        if (((e >> 1) & 7) < JD_EX2_POLY_OF8) {
+                            ex2_poly2(xv.x, xv.y, p0, p1);
+                        } else {
+                            p0 = ex2_approx(xv.x);
+                            p1 = ex2_approx(xv.y);
+                        }
                         ls[(e >> 1) & 3] += p0 + p1;
                         pk[e >> 1] = pack_bf16x2(p0, p1);
                     }

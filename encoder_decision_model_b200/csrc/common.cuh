@@ -70,6 +70,13 @@ __device__ __forceinline__ float gelu_as(float x) {
     return x >= 0.f ? x - xh : xh;
 }
 
+// Two floats to FP8 E4M3 bytes (round to nearest even, saturating at +-448): lo in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
@@ -263,6 +270,22 @@ __device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
     d |= (uint64_t)1 << 46;                     // descriptor version (sm_100)
     d |= (uint64_t)4 << 61;                     // 64-byte swizzle
     return d;
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 with E4M3 inputs (K = 32 per instruction), f32 accumulate.
+__device__ __forceinline__ void tc_mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor for kind::f8f6f4: E4M3 A and B (format code 0), f32 D, K-major A and B, M = 128.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
 // Instruction descriptor for kind::f16: bf16 A/B, f32 D, K-major A and B, M = 128.

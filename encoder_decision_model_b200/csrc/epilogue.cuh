@@ -45,6 +45,8 @@ struct EpiParams {
     int act;                 // 0 ReLU, 1 GELU
     float eps;
     unsigned *status;
+    const float *col_scale;  // FP8 QKV GEMM: [N] per output column, activation scale x weight row scale
+    float out8_inv_scale;    // FP8 LayerNorm output of the residual GEMM: E4M3(y * out8_inv_scale) into out
 };
 
 // LayerNorm of the 384 values held 12 per lane (columns j*128 + lane*4 + e).

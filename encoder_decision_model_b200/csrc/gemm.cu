@@ -225,7 +225,7 @@ __device__ __forceinline__ void stage_row32(uint8_t *box, int r, int c0, const u
             make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
 }
 
-template <int EPI, int BN, int NPART>
+template <int EPI, int BN, int NPART, bool F8 = false>
 __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0, int n0, const EpiParams &ep,
                                                  const CUtensorMap *tmO, OutStage &os, int lane,
                                                  const float2 (&cs)[32], bool have_cs, int part) {
@@ -312,6 +312,21 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
                 ba[4 * j4] = x.x; ba[4 * j4 + 1] = x.y; ba[4 * j4 + 2] = x.z; ba[4 * j4 + 3] = x.w;
                 bb[4 * j4] = y.x; bb[4 * j4 + 1] = y.y; bb[4 * j4 + 2] = y.z; bb[4 * j4 + 3] = y.w;
             }
+            if constexpr (F8) {  // E4M3 product: undo the activation and weight-row scales
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 x = reinterpret_cast<const float4 *>(ep.col_scale + n)[j4];
+                    const float4 y = reinterpret_cast<const float4 *>(ep.col_scale + n + 32)[j4];
+                    a[4 * j4] = __float_as_uint(__uint_as_float(a[4 * j4]) * x.x);
+                    a[4 * j4 + 1] = __float_as_uint(__uint_as_float(a[4 * j4 + 1]) * x.y);
+                    a[4 * j4 + 2] = __float_as_uint(__uint_as_float(a[4 * j4 + 2]) * x.z);
+                    a[4 * j4 + 3] = __float_as_uint(__uint_as_float(a[4 * j4 + 3]) * x.w);
+                    b[4 * j4] = __float_as_uint(__uint_as_float(b[4 * j4]) * y.x);
+                    b[4 * j4 + 1] = __float_as_uint(__uint_as_float(b[4 * j4 + 1]) * y.y);
+                    b[4 * j4 + 2] = __float_as_uint(__uint_as_float(b[4 * j4 + 2]) * y.z);
+                    b[4 * j4 + 3] = __float_as_uint(__uint_as_float(b[4 * j4 + 3]) * y.w);
+                }
+            }
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
                 float r2[2], s2[2];
@@ -338,7 +353,10 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
     }
 }
 
-template <int EPI, int BN, int EW>
+// F8: A and W are E4M3 (128-element k-blocks of 128 bytes, the same swizzled layout as 64
+// bf16), the MMAs kind::f8f6f4 with K = 32, and the epilogue multiplies each column by
+// ep.col_scale before its bias / RoPE.
+template <int EPI, int BN, int EW, bool F8 = false>
 __global__ void __launch_bounds__(64 + 32 * EW, 1)
     k_gemm_pc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmO, int K, int n_tiles, int nblk, EpiParams ep) {
@@ -353,7 +371,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int KB = K / 64;
+    constexpr int KBW = F8 ? 128 : 64;  // elements per 128-byte k-block row
+    const int KB = K / KBW;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -393,14 +412,14 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
                     }
                     uint8_t *sa = smem + s * C::STAGE;
                     mbar_arrive_expect_tx(&full[s], C::STAGE);
-                    tma_load_2d(sa, &tmA, &full[s], kb * 64, m0);
-                    tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * 64, n0);
+                    tma_load_2d(sa, &tmA, &full[s], kb * KBW, m0);
+                    tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * KBW, n0);
                 }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BN);
+            constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(BN) : idesc_bf16_f32(BN);
             uint32_t it = 0, tc = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tc) {
@@ -415,9 +434,14 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
                     const uint32_t a_base = smem_u32(smem + s * C::STAGE);
                     const uint32_t b_base = a_base + C::A_BYTES;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        tc_mma_bf16(dacc, sdesc_sw128(a_base + k * 32), sdesc_sw128(b_base + k * 32), idesc,
-                                    (kb | k) != 0);
+                    for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction: 16 bf16 or 32 E4M3
+                        if constexpr (F8)
+                            tc_mma_e4m3(dacc, sdesc_sw128(a_base + k * 32), sdesc_sw128(b_base + k * 32), idesc,
+                                        (kb | k) != 0);
+                        else
+                            tc_mma_bf16(dacc, sdesc_sw128(a_base + k * 32), sdesc_sw128(b_base + k * 32), idesc,
+                                        (kb | k) != 0);
+                    }
                     tc_commit(&empty[s]);
                 }
                 tc_commit(&accf[buf]);
@@ -452,7 +476,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
             __syncwarp();
             tc_fence_after();
             const uint32_t tacc = tmem + buf * C::BUF_COLS + ((uint32_t)(q * 32) << 16);
-            pc_epilogue_rows<EPI, BN, EW / 4>(tacc, lane, row0, n0, ep, &tmO, os, lane, cs, have_cs, part);
+            pc_epilogue_rows<EPI, BN, EW / 4, F8>(tacc, lane, row0, n0, ep, &tmO, os, lane, cs, have_cs, part);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acce[buf]);
@@ -513,8 +537,15 @@ struct RlCfg {
 #endif
 constexpr int RL_STAGES = JD_RL_STAGES, RL_NXB = JD_RL_NXB;
 using RlCur = RlCfg<RL_STAGES, RL_NXB>;
+#ifndef JD_RL_SPLIT_PERSISTENT
+#define JD_RL_SPLIT_PERSISTENT 0
+#endif
+constexpr int RS_NS = 3;  // CTAs per row tile of the split residual GEMM (128 columns each)
+constexpr int RP_NS = 2;  // CTAs per row tile of the persistent split residual GEMM (192 columns each)
 
-template <int STAGES_, int NXB_>
+// OUT8: the LayerNorm output goes out as E4M3 bytes, y * ep.out8_inv_scale, rows of 384 bytes
+// (the operand of the FP8 QKV GEMM).
+template <int STAGES_, int NXB_, bool OUT8 = false>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_rl(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXN, int K, int n_tiles,
@@ -695,6 +726,37 @@ __global__ void __launch_bounds__(192, 1)
             // ---- pass 2: xn = LN(v) from TMEM, written straight from registers
             const int row = m0 + r;
             __nv_bfloat16 *xo = reinterpret_cast<__nv_bfloat16 *>(ep.out) + (size_t)row * ep.ldo;
+            if constexpr (OUT8) {
+                uint8_t *xo8 = reinterpret_cast<uint8_t *>(ep.out) + (size_t)row * ep.ldo;
+#pragma unroll 1
+                for (int j = 0; j < 6; ++j) {
+                    uint32_t a[32], b2[32];
+                    tmem_ld32(tl + j * 64, a);
+                    tmem_ld32(tl + j * 64 + 32, b2);
+                    tmem_ld_wait();
+                    uint32_t w[16];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const int col = j * 64 + h * 32 + j4 * 4;
+                            const float4 gg = *reinterpret_cast<const float4 *>(ep.ln_g + col);
+                            const uint32_t *src = h ? b2 : a;
+                            const float sc = rstd * ep.out8_inv_scale;
+                            const float y0 = (__uint_as_float(src[4 * j4 + 0]) - mean) * sc * gg.x;
+                            const float y1 = (__uint_as_float(src[4 * j4 + 1]) - mean) * sc * gg.y;
+                            const float y2 = (__uint_as_float(src[4 * j4 + 2]) - mean) * sc * gg.z;
+                            const float y3 = (__uint_as_float(src[4 * j4 + 3]) - mean) * sc * gg.w;
+                            w[h * 8 + j4] = pack_e4m3x2(y0, y1) | (pack_e4m3x2(y2, y3) << 16);
+                        }
+                    }
+                    if (row < ep.rows) {  // 64 bytes of the row: two 32-byte stores
+                        uint8_t *dst = xo8 + j * 64;
+                        st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+                        st_global_v8(dst + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+                    }
+                }
+            } else {
 #pragma unroll 1
             for (int j = 0; j < 6; ++j) {
                 uint32_t a[32], b2[32];
@@ -727,6 +789,7 @@ __global__ void __launch_bounds__(192, 1)
                                      w[8 * cc + 5], w[8 * cc + 6], w[8 * cc + 7]);
                 }
             }
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acce);
@@ -734,6 +797,592 @@ __global__ void __launch_bounds__(192, 1)
         if (leader) bulk_wait_all();
         __syncwarp();
     }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- residual + LayerNorm GEMM, split over a cluster
+//
+// For batches of a few row tiles (a single request of some hundred tokens makes
+// seven), the persistent residual GEMM keeps one SM per tile busy: each loads
+// the whole weight (884 KB for Wo2) and streams the tile's whole residual.  Here
+// a cluster of NS CTAs shares a 128-row tile: CTA r computes the NC = 384 / NS
+// output columns [NC r, NC r + NC) (an N = NC accumulator, the weight rows of
+// its columns only), adds the residual of its columns, stores them, and sends
+// each row's mean and M2 over its columns to every CTA of the cluster through
+// distributed shared memory; after a cluster barrier each CTA merges the NS
+// partial moments in rank order (equal counts: the mean of the means, M2 plus
+// the spread of the means) and writes the LayerNorm output of its columns.
+//   warp 0 lane 0  TMA producer: A box 128 x 64 and W box NC x 64 (128-byte swizzle) per stage
+//   warp 1         TMEM allocation; lane 0 issues the N = NC MMAs
+//   warps 2..5     epilogue, one row per thread; the NC / 32 residual chunks (FP32,
+//                  128 x 32) are loaded by TMA at the start, under the mainloop
+template <int NS>
+struct RsCfg {
+    static constexpr int NC = D / NS;            // output columns per CTA
+    static constexpr int A_BYTES = 128 * 128;    // 128 rows x 64 bf16
+    static constexpr int B_BYTES = NC * 128;     // NC rows x 64 bf16
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int STAGES = NS == 2 ? 3 : 4;
+    static constexpr int RING = STAGES * STAGE;
+    static constexpr int XCH = 128 * 32 * 4;     // residual chunk: 128 rows x 32 FP32
+    static constexpr int NX = NC / 32;
+    static constexpr int MOM = NS * 128 * 8;     // (mean, M2) of every row from every rank
+    static constexpr int DATA = RING + NX * XCH + MOM;
+    static constexpr int BAR_BYTES = (2 * STAGES + 1 + NX) * 8 + 8;
+    static constexpr int SMEM = DATA + BAR_BYTES + 1024;
+    static constexpr uint32_t TMEM_COLS = NC <= 128 ? 128 : 256;
+    static_assert(NC % 32 == 0 && NC % 16 == 0 && NC <= 256, "column share");
+    static_assert(SMEM <= 227 * 1024, "split residual GEMM shared memory");
+};
+
+__device__ __forceinline__ uint32_t rs_cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void rs_cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int NS, bool OUT8>
+__global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
+    k_gemm_rls(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmX, int K, EpiParams ep) {
+    using C = RsCfg<NS>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *xbuf = smem + C::RING;
+    float2 *mom = reinterpret_cast<float2 *>(smem + C::RING + C::NX * C::XCH);  // [NS][128]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::DATA);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *accf = empty + C::STAGES;
+    uint64_t *xfull = accf + 1;  // [NX]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xfull + C::NX);
+
+    const uint32_t rank = rs_cluster_rank();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = (int)(blockIdx.x / NS) * 128;
+    const int c0 = (int)rank * C::NC;
+    const int KB = K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        for (int c = 0; c < C::NX; ++c) mbar_init(&xfull[c], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmX);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const bool leader = threadIdx.x == 64;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int kb = 0; kb < KB; ++kb) {
+                const int s = kb % C::STAGES;
+                if (kb >= C::STAGES && !mbar_wait(&empty[s], ((kb / C::STAGES) - 1) & 1, ep.status)) break;
+                uint8_t *sa = smem + s * C::STAGE;
+                mbar_arrive_expect_tx(&full[s], C::STAGE);
+                tma_load_2d(sa, &tmA, &full[s], kb * 64, m0);
+                tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * 64, c0);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(C::NC);
+            for (int kb = 0; kb < KB; ++kb) {
+                const int s = kb % C::STAGES;
+                if (!mbar_wait(&full[s], (kb / C::STAGES) & 1, ep.status)) break;
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(smem + s * C::STAGE);
+                const uint32_t b_base = a_base + C::A_BYTES;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    tc_mma_bf16(tmem, sdesc_sw128(a_base + k * 32), sdesc_sw128(b_base + k * 32), idesc, (kb | k) != 0);
+                tc_commit(&empty[s]);
+            }
+            tc_commit(accf);
+        }
+    } else if (leader) {  // the residual of this CTA's columns, under the mainloop
+        for (int c = 0; c < C::NX; ++c) {
+            mbar_arrive_expect_tx(&xfull[c], C::XCH);
+            tma_load_2d(xbuf + c * C::XCH, &tmX, &xfull[c], c0 + c * 32, m0);
+        }
+    }
+
+    const int q = warp & 3;
+    const int r = q * 32 + lane;  // row inside the tile (epilogue warps)
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    float mean = 0.f, m2 = 0.f;
+    if (warp >= 2) {
+        mbar_wait(accf, 0, ep.status);
+        __syncwarp();
+        tc_fence_after();
+        // ---- pass 1: v = x + acc (+ bias) for this CTA's columns; moments over them
+        float cnt = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < C::NX; ++c) {
+            uint32_t a[32];
+            tmem_ld32(tl + c * 32, a);
+            mbar_wait(&xfull[c], 0, ep.status);
+            tmem_ld_wait();
+            uint8_t *xb = xbuf + c * C::XCH;
+            float v[32];
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+                const float4 x = *reinterpret_cast<const float4 *>(xb + r * 128 + ((j4 ^ (r & 7)) << 4));
+                float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (ep.bias) bb = reinterpret_cast<const float4 *>(ep.bias + c0 + c * 32)[j4];
+                v[4 * j4 + 0] = x.x + __uint_as_float(a[4 * j4 + 0]) + bb.x;
+                v[4 * j4 + 1] = x.y + __uint_as_float(a[4 * j4 + 1]) + bb.y;
+                v[4 * j4 + 2] = x.z + __uint_as_float(a[4 * j4 + 2]) + bb.z;
+                v[4 * j4 + 3] = x.w + __uint_as_float(a[4 * j4 + 3]) + bb.w;
+            }
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s += v[j];
+            const float cm = s * (1.0f / 32.f);
+            float cq = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) cq += (v[j] - cm) * (v[j] - cm);
+            if (c == 0) {
+                mean = cm;
+                m2 = cq;
+                cnt = 32.f;
+            } else {
+                const float tot = cnt + 32.f, dl = cm - mean;
+                mean += dl * (32.f / tot);
+                m2 += cq + dl * dl * (cnt * 32.f / tot);
+                cnt = tot;
+            }
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4)
+                *reinterpret_cast<float4 *>(xb + r * 128 + ((j4 ^ (r & 7)) << 4)) =
+                    make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+            uint32_t w[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
+            tmem_st32(tl + c * 32, w);
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (leader) {
+                tma_store_2d(&tmX, xb, c0 + c * 32, m0);
+                bulk_commit();
+            }
+        }
+        tmem_st_wait();
+        // this CTA's (mean, M2) of row r, to slot [rank][r] of every CTA of the cluster
+        const uint32_t local = smem_u32(&mom[rank * 128 + r]);
+#pragma unroll
+        for (int j = 0; j < NS; ++j) {
+            uint32_t remote;
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(j));
+            asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(mean), "f"(m2) : "memory");
+        }
+    }
+    __syncwarp();
+    rs_cluster_sync();
+    if (warp >= 2) {
+        // ---- merge the NS partial moments (equal counts NC) in rank order
+        float mu = 0.f;
+#pragma unroll
+        for (int j = 0; j < NS; ++j) mu += mom[j * 128 + r].x;
+        mu *= 1.0f / NS;
+        float tot = 0.f;
+#pragma unroll
+        for (int j = 0; j < NS; ++j) {
+            const float2 p = mom[j * 128 + r];
+            tot += p.y + (float)C::NC * (p.x - mu) * (p.x - mu);
+        }
+        const float rstd = 1.0f / sqrtf(tot * (1.0f / D) + ep.eps);
+        // ---- pass 2: LayerNorm of this CTA's columns from TMEM, stored from registers
+        const int row = m0 + r;
+#pragma unroll 1
+        for (int c = 0; c < C::NX; ++c) {
+            uint32_t a[32];
+            tmem_ld32(tl + c * 32, a);
+            tmem_ld_wait();
+            const int col0 = c0 + c * 32;
+            uint32_t w[16];
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+                const int col = col0 + j4 * 4;
+                const float4 gg = *reinterpret_cast<const float4 *>(ep.ln_g + col);
+                float4 be = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (!OUT8 && ep.ln_b) be = *reinterpret_cast<const float4 *>(ep.ln_b + col);
+                const float sc = OUT8 ? rstd * ep.out8_inv_scale : rstd;
+                const float y0 = (__uint_as_float(a[4 * j4 + 0]) - mu) * sc * gg.x + be.x;
+                const float y1 = (__uint_as_float(a[4 * j4 + 1]) - mu) * sc * gg.y + be.y;
+                const float y2 = (__uint_as_float(a[4 * j4 + 2]) - mu) * sc * gg.z + be.z;
+                const float y3 = (__uint_as_float(a[4 * j4 + 3]) - mu) * sc * gg.w + be.w;
+                if (OUT8) {
+                    if (j4 < 8) w[j4] = pack_e4m3x2(y0, y1) | (pack_e4m3x2(y2, y3) << 16);
+                } else {
+                    w[2 * j4] = pack_bf16x2(y0, y1);
+                    w[2 * j4 + 1] = pack_bf16x2(y2, y3);
+                }
+            }
+            if (row < ep.rows) {
+                if (OUT8) {
+                    uint8_t *dst = reinterpret_cast<uint8_t *>(ep.out) + (size_t)row * ep.ldo + col0;
+                    st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+                } else {
+                    uint8_t *dst = reinterpret_cast<uint8_t *>(reinterpret_cast<__nv_bfloat16 *>(ep.out) +
+                                                               (size_t)row * ep.ldo + col0);
+                    st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+                    st_global_v8(dst + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+                }
+            }
+        }
+        if (leader) bulk_wait_all();
+        tc_fence_before();
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- persistent residual + LayerNorm GEMM split over a cluster
+//
+// The same product as k_gemm_rl for batches of many row tiles, with the 384 output
+// columns of every tile split over a cluster of NS = 2 CTAs (CTA r: columns [192 r,
+// 192 r + 192)).  With 192 columns per CTA, two accumulators fit in TMEM, so the
+// epilogue of one tile overlaps the MMAs of the next (with 384 columns per CTA the next
+// tile's MMAs wait for the whole epilogue).  The clusters walk the row tiles (cluster c:
+// tiles c, c + C, ...); the two CTAs of a cluster take the same tiles.  Per tile each CTA
+// sends its rows' (mean, M2) over its columns into both CTAs' shared memory (slots
+// double-buffered by tile parity; every epilogue thread arrives on both CTAs' moment
+// barriers after its stores); a CTA merges the two halves in rank order once all have
+// arrived.  A slot is rewritten two tiles later only after the other CTA has sent the
+// next tile's moments, which it does after merging this one.
+//   warp 0 lane 0  TMA producer: A box 128 x 64 and W box 192 x 64 (128-byte swizzle)
+//   warp 1         TMEM allocation (two accumulators); lane 0 issues the N = 192 MMAs
+//   warps 2..5     epilogue, one row per thread: residual chunks (128 x 32 FP32) through a
+//                  ring of NXB buffers refilled across tiles, as in k_gemm_rl
+template <int NS>
+struct RpCfg {
+    static constexpr int NC = D / NS;              // output columns per CTA
+    static constexpr int A_BYTES = 128 * 128;      // 128 rows x 64 bf16
+    static constexpr int B_BYTES = NC * 128;       // NC rows x 64 bf16
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int STAGES = 3;
+    static constexpr int RING = STAGES * STAGE;
+    static constexpr int XCH = 128 * 32 * 4;       // residual chunk: 128 rows x 32 FP32
+    static constexpr int NX = NC / 32;             // residual chunks per tile
+    static constexpr int NXB = 4;                  // residual buffers
+    static constexpr int MOM = 2 * NS * 128 * 8;   // (mean, M2): [tile parity][rank][row]
+    static constexpr int DATA = RING + NXB * XCH + MOM;
+    static constexpr int NBAR = 2 * STAGES + 2 + 2 + NXB + 2;
+    static constexpr int SMEM = DATA + NBAR * 8 + 8 + 1024;
+    static constexpr uint32_t ACC_STRIDE = 256;    // TMEM columns between the two accumulators
+    static_assert(NC % 32 == 0 && NC <= 256 && SMEM <= 227 * 1024, "persistent split residual GEMM");
+};
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (the arrivals come from the other CTAs of the cluster).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, unsigned *status) {
+    const uint32_t addr = smem_u32(bar);
+    uint64_t t0 = 0;
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_cluster(addr, parity)) return true;
+        if ((it & 255u) == 0) {
+            if (status && (*reinterpret_cast<volatile unsigned *>(status) & ST_WAIT_TIMEOUT)) return false;
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > 2000000000ull) {
+                if (status) atomicOr(status, ST_WAIT_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+// Arrive on the barrier at the address of `local_bar` in CTA `rank` of this cluster.
+__device__ __forceinline__ void mbar_arrive_remote(const uint64_t *local_bar, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local_bar)), "r"(rank));
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+}
+
+template <int NS, bool OUT8>
+__global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
+    k_gemm_rlp(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmX, int K, int n_tiles, EpiParams ep) {
+    using C = RpCfg<NS>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *xbuf = smem + C::RING;
+    float2 *mom = reinterpret_cast<float2 *>(smem + C::RING + C::NXB * C::XCH);  // [2][NS][128]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::DATA);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *accf = empty + C::STAGES;  // [2]
+    uint64_t *acce = accf + 2;           // [2]
+    uint64_t *xfull = acce + 2;          // [NXB]
+    uint64_t *momf = xfull + C::NXB;     // [2]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(momf + 2);
+
+    const uint32_t rank = rs_cluster_rank();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cid = (int)(blockIdx.x / NS), ncl = (int)(gridDim.x / NS);
+    const int c0 = (int)rank * C::NC;
+    const int KB = K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], 4);
+            mbar_init(&momf[b], NS * 128);  // one arrival per epilogue thread of every CTA
+        }
+        for (int b = 0; b < C::NXB; ++b) mbar_init(&xfull[b], 1);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmX);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    rs_cluster_sync();  // both CTAs' barriers exist before the first remote arrival
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = cid; t < n_tiles && ok; t += ncl) {
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const uint32_t s = it % C::STAGES;
+                    if (it >= (uint32_t)C::STAGES && !mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1, ep.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = smem + s * C::STAGE;
+                    mbar_arrive_expect_tx(&full[s], C::STAGE);
+                    tma_load_2d(sa, &tmA, &full[s], kb * 64, t * 128);
+                    tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * 64, c0);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(C::NC);
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int t = cid; t < n_tiles && ok; t += ncl, ++tc) {
+                const uint32_t b = tc & 1;
+                if (tc >= 2 && !mbar_wait(&acce[b], ((tc >> 1) - 1) & 1, ep.status)) break;
+                tc_fence_after();
+                const uint32_t dacc = tmem + b * C::ACC_STRIDE;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const uint32_t s = it % C::STAGES;
+                    if (!mbar_wait(&full[s], (it / C::STAGES) & 1, ep.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smem + s * C::STAGE);
+                    const uint32_t b_base = a_base + C::A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        tc_mma_bf16(dacc, sdesc_sw128(a_base + k * 32), sdesc_sw128(b_base + k * 32), idesc,
+                                    (kb | k) != 0);
+                    tc_commit(&empty[s]);
+                }
+                tc_commit(&accf[b]);
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const bool leader = threadIdx.x == 64;
+        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+        // residual chunk g (local tile g / NX, chunk g % NX) goes into buffer g % NXB
+        if (leader && cid < n_tiles) {
+            for (int g = 0; g < C::NXB; ++g) {
+                const int th = cid + (g / C::NX) * ncl;
+                if (th >= n_tiles) break;
+                mbar_arrive_expect_tx(&xfull[g], C::XCH);
+                tma_load_2d(xbuf + g * C::XCH, &tmX, &xfull[g], c0 + (g % C::NX) * 32, th * 128);
+            }
+        }
+        uint32_t tc = 0;
+        for (int t = cid; t < n_tiles; t += ncl, ++tc) {
+            const int m0 = t * 128;
+            const uint32_t b = tc & 1;
+            const uint32_t tacc = tl + b * C::ACC_STRIDE;
+            mbar_wait(&accf[b], (tc >> 1) & 1, ep.status);
+            __syncwarp();
+            tc_fence_after();
+            float cnt = 0.f, mean = 0.f, m2 = 0.f;
+            // ---- pass 1: v = x + acc (+ bias) for this CTA's columns; moments over them
+#pragma unroll 1
+            for (int c = 0; c < C::NX; ++c) {
+                const uint32_t g = tc * C::NX + c, xb_i = g % C::NXB;
+                uint32_t a[32];
+                tmem_ld32(tacc + c * 32, a);
+                mbar_wait(&xfull[xb_i], (g / C::NXB) & 1, ep.status);
+                tmem_ld_wait();
+                uint8_t *xb = xbuf + xb_i * C::XCH;
+                float v[32];
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(xb + r * 128 + ((j4 ^ (r & 7)) << 4));
+                    float4 bb = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (ep.bias) bb = reinterpret_cast<const float4 *>(ep.bias + c0 + c * 32)[j4];
+                    v[4 * j4 + 0] = x.x + __uint_as_float(a[4 * j4 + 0]) + bb.x;
+                    v[4 * j4 + 1] = x.y + __uint_as_float(a[4 * j4 + 1]) + bb.y;
+                    v[4 * j4 + 2] = x.z + __uint_as_float(a[4 * j4 + 2]) + bb.z;
+                    v[4 * j4 + 3] = x.w + __uint_as_float(a[4 * j4 + 3]) + bb.w;
+                }
+                float s = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) s += v[j];
+                const float cm = s * (1.0f / 32.f);
+                float cq = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) cq += (v[j] - cm) * (v[j] - cm);
+                if (c == 0) {
+                    mean = cm;
+                    m2 = cq;
+                    cnt = 32.f;
+                } else {
+                    const float tot = cnt + 32.f, dl = cm - mean;
+                    mean += dl * (32.f / tot);
+                    m2 += cq + dl * dl * (cnt * 32.f / tot);
+                    cnt = tot;
+                }
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4)
+                    *reinterpret_cast<float4 *>(xb + r * 128 + ((j4 ^ (r & 7)) << 4)) =
+                        make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+                uint32_t w[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[j]);
+                tmem_st32(tacc + c * 32, w);
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (leader) {
+                    tma_store_2d(&tmX, xb, c0 + c * 32, m0);
+                    bulk_commit();
+                    // refill the previous chunk's buffer (its store has read it once at most this
+                    // chunk's store is pending) with chunk g - 1 + NXB
+                    if (g >= 1) {
+                        const uint32_t h = g - 1 + C::NXB;
+                        const int th = cid + (int)(h / C::NX) * ncl;
+                        if (th < n_tiles) {
+                            const uint32_t bp = (g - 1) % C::NXB;
+                            bulk_wait_read<1>();
+                            mbar_arrive_expect_tx(&xfull[bp], C::XCH);
+                            tma_load_2d(xbuf + bp * C::XCH, &tmX, &xfull[bp], c0 + (int)(h % C::NX) * 32, th * 128);
+                        }
+                    }
+                }
+            }
+            tmem_st_wait();
+            // ---- moments of this CTA's half to both CTAs, then merge the halves in rank order
+            float2 *slot = mom + (size_t)(b * NS + rank) * 128 + r;
+#pragma unroll
+            for (int j = 0; j < NS; ++j) {
+                uint32_t remote;
+                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(slot)), "r"(j));
+                asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(mean), "f"(m2) : "memory");
+            }
+            // each thread releases its own stores with its arrivals
+#pragma unroll
+            for (int j = 0; j < NS; ++j) mbar_arrive_remote(&momf[b], (uint32_t)j);
+            mbar_wait_cluster(&momf[b], (tc >> 1) & 1, ep.status);
+            float mu = 0.f;
+#pragma unroll
+            for (int j = 0; j < NS; ++j) mu += mom[(size_t)(b * NS + j) * 128 + r].x;
+            mu *= 1.0f / NS;
+            float tot = 0.f;
+#pragma unroll
+            for (int j = 0; j < NS; ++j) {
+                const float2 p = mom[(size_t)(b * NS + j) * 128 + r];
+                tot += p.y + (float)C::NC * (p.x - mu) * (p.x - mu);
+            }
+            const float rstd = 1.0f / sqrtf(tot * (1.0f / D) + ep.eps);
+            // ---- pass 2: LayerNorm of this CTA's columns from TMEM
+            const int row = m0 + r;
+#pragma unroll 1
+            for (int c = 0; c < C::NX; ++c) {
+                uint32_t a[32];
+                tmem_ld32(tacc + c * 32, a);
+                tmem_ld_wait();
+                const int col0 = c0 + c * 32;
+                uint32_t w[16];
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const int col = col0 + j4 * 4;
+                    const float4 gg = *reinterpret_cast<const float4 *>(ep.ln_g + col);
+                    float4 be = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (!OUT8 && ep.ln_b) be = *reinterpret_cast<const float4 *>(ep.ln_b + col);
+                    const float sc = OUT8 ? rstd * ep.out8_inv_scale : rstd;
+                    const float y0 = (__uint_as_float(a[4 * j4 + 0]) - mu) * sc * gg.x + be.x;
+                    const float y1 = (__uint_as_float(a[4 * j4 + 1]) - mu) * sc * gg.y + be.y;
+                    const float y2 = (__uint_as_float(a[4 * j4 + 2]) - mu) * sc * gg.z + be.z;
+                    const float y3 = (__uint_as_float(a[4 * j4 + 3]) - mu) * sc * gg.w + be.w;
+                    if (OUT8) {
+                        w[j4] = pack_e4m3x2(y0, y1) | (pack_e4m3x2(y2, y3) << 16);
+                    } else {
+                        w[2 * j4] = pack_bf16x2(y0, y1);
+                        w[2 * j4 + 1] = pack_bf16x2(y2, y3);
+                    }
+                }
+                if (row < ep.rows) {
+                    if (OUT8) {
+                        uint8_t *dst = reinterpret_cast<uint8_t *>(ep.out) + (size_t)row * ep.ldo + col0;
+                        st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+                    } else {
+                        uint8_t *dst = reinterpret_cast<uint8_t *>(reinterpret_cast<__nv_bfloat16 *>(ep.out) +
+                                                                   (size_t)row * ep.ldo + col0);
+                        st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+                        st_global_v8(dst + 32, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[b]);
+        }
+        if (leader) bulk_wait_all();
+        __syncwarp();
+    }
+    __syncwarp();
+    rs_cluster_sync();  // no CTA leaves while the other may still write into it
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -828,7 +1477,25 @@ cudaError_t gemm_init_attributes() {
     if ((e = cudaFuncSetAttribute(k_gemm_rl<RL_STAGES, RL_NXB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   RlCur::SMEM)) != cudaSuccess)
         return e;
+    if ((e = cudaFuncSetAttribute(k_gemm_rl<RL_STAGES, RL_NXB, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  RlCur::SMEM)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_gemm_rlp<RP_NS, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  RpCfg<RP_NS>::SMEM)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_gemm_rlp<RP_NS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  RpCfg<RP_NS>::SMEM)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_gemm_rls<RS_NS, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  RsCfg<RS_NS>::SMEM)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_gemm_rls<RS_NS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  RsCfg<RS_NS>::SMEM)) != cudaSuccess)
+        return e;
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 192, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  PcCfg<192>::SMEM)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 192, 4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<192>::SMEM)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_GEGLU, 256, GEGLU_EW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -859,16 +1526,16 @@ static cudaError_t launch_f32(const GemmOp &op, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-template <int EPI, int BN>
+template <int EPI, int BN, bool F8 = false>
 static cudaError_t launch_pc(const GemmOp &op, cudaStream_t st) {
-    if (op.N % BN != 0) return cudaErrorInvalidValue;
+    if (op.N % BN != 0 || (F8 && (op.K % 128 != 0 || !op.ep.col_scale))) return cudaErrorInvalidValue;
     const int nblk = op.N / BN;
     const int n_tiles = nblk * ((op.ep.rows + 127) / 128);
     const int grid = n_tiles < g_num_sms ? n_tiles : g_num_sms;
     if (!op.tmO) return cudaErrorInvalidValue;
     constexpr int EW = EPI == EPI_GEGLU ? GEGLU_EW : 4;  // epilogue warps
-    k_gemm_pc<EPI, BN, EW><<<grid, 64 + 32 * EW, PcCfg<BN>::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmO, op.K, n_tiles,
-                                                                         nblk, op.ep);
+    k_gemm_pc<EPI, BN, EW, F8><<<grid, 64 + 32 * EW, PcCfg<BN>::SMEM, st>>>(*op.tmA, *op.tmB, *op.tmO, op.K,
+                                                                             n_tiles, nblk, op.ep);
     return cudaGetLastError();
 }
 
@@ -879,12 +1546,43 @@ cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st) {
         op.N == D && op.K % 32 == 0) {
         const int n_tiles = (op.ep.rows + 127) / 128;
         const int grid = n_tiles < g_num_sms ? n_tiles : g_num_sms;
-        k_gemm_rl<RL_STAGES, RL_NXB><<<grid, 192, RlCur::SMEM, st>>>(*op.tmA64, *op.tmB64, *op.tmX, *op.tmXN, op.K,
-                                                                     n_tiles, op.ep);
+        if (op.tmA && op.tmBs && op.K % 64 == 0 && RS_NS * n_tiles <= g_num_sms) {
+            // few row tiles: split each tile's columns over a cluster, so RS_NS SMs share it
+            if (op.out8 && (op.ep.ln_b || op.ep.out8_inv_scale <= 0.f)) return cudaErrorInvalidValue;
+            if (op.out8)
+                k_gemm_rls<RS_NS, true><<<RS_NS * n_tiles, 192, RsCfg<RS_NS>::SMEM, st>>>(*op.tmA, *op.tmBs, *op.tmX,
+                                                                                          op.K, op.ep);
+            else
+                k_gemm_rls<RS_NS, false><<<RS_NS * n_tiles, 192, RsCfg<RS_NS>::SMEM, st>>>(*op.tmA, *op.tmBs, *op.tmX,
+                                                                                           op.K, op.ep);
+            return cudaGetLastError();
+        }
+#if JD_RL_SPLIT_PERSISTENT
+        if (op.tmA && op.tmBp && op.K % 64 == 0) {  // many row tiles: persistent, columns split over 2 CTAs
+            if (op.out8 && (op.ep.ln_b || op.ep.out8_inv_scale <= 0.f)) return cudaErrorInvalidValue;
+            const int ncl = std::min(n_tiles, g_num_sms / RP_NS);
+            if (op.out8)
+                k_gemm_rlp<RP_NS, true><<<RP_NS * ncl, 192, RpCfg<RP_NS>::SMEM, st>>>(*op.tmA, *op.tmBp, *op.tmX, op.K,
+                                                                                       n_tiles, op.ep);
+            else
+                k_gemm_rlp<RP_NS, false><<<RP_NS * ncl, 192, RpCfg<RP_NS>::SMEM, st>>>(*op.tmA, *op.tmBp, *op.tmX, op.K,
+                                                                                        n_tiles, op.ep);
+            return cudaGetLastError();
+        }
+#endif
+        if (op.out8) {
+            if (op.ep.ln_b || op.ep.out8_inv_scale <= 0.f) return cudaErrorInvalidValue;
+            k_gemm_rl<RL_STAGES, RL_NXB, true><<<grid, 192, RlCur::SMEM, st>>>(*op.tmA64, *op.tmB64, *op.tmX,
+                                                                               *op.tmXN, op.K, n_tiles, op.ep);
+        } else {
+            k_gemm_rl<RL_STAGES, RL_NXB><<<grid, 192, RlCur::SMEM, st>>>(*op.tmA64, *op.tmB64, *op.tmX, *op.tmXN,
+                                                                         op.K, n_tiles, op.ep);
+        }
         return cudaGetLastError();
     }
+    if (op.out8 || (op.f8 && (fp32 || op.epi != EPI_QKV))) return cudaErrorInvalidValue;
     if (!fp32) {  // persistent tcgen05 kernels for the column-split epilogues
-        if (op.epi == EPI_QKV) return launch_pc<EPI_QKV, 192>(op, st);
+        if (op.epi == EPI_QKV) return op.f8 ? launch_pc<EPI_QKV, 192, true>(op, st) : launch_pc<EPI_QKV, 192>(op, st);
         if (op.epi == EPI_GEGLU) return launch_pc<EPI_GEGLU, 256>(op, st);
         if (op.epi == EPI_BIAS_ACT) return launch_pc<EPI_BIAS_ACT, 256>(op, st);
     }

@@ -25,22 +25,31 @@ struct GemmOp {
     const CUtensorMap *tmXN;  // BF16 residual epilogue: LayerNorm output, box 64 x 128, 128-byte swizzle
     const CUtensorMap *tmA64; // BF16 residual GEMM: A box 32 x 128, 64-byte swizzle
     const CUtensorMap *tmB64; // BF16 residual GEMM: W box 32 x 192, 64-byte swizzle
+    const CUtensorMap *tmBs;  // BF16 residual GEMM split over a cluster: W box 64 x 128, 128-byte swizzle
+    const CUtensorMap *tmBp;  // BF16 persistent split residual GEMM: W box 64 x 192, 128-byte swizzle
     const float *A32;         // FP32 path: A [rows, lda]
     int lda;
     const float *W32;         // FP32 path: W [N, K]
     EpiParams ep;
+    bool f8 = false;          // QKV on E4M3 operands (tmA, tmB: byte maps, box 128 x rows); needs ep.col_scale
+    bool out8 = false;        // residual GEMM: LayerNorm output as E4M3 bytes (ep.out8_inv_scale); no ln_b
 };
 cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st);
 
 // Per-token row index / position and per-row attention work-unit offsets
 // (qb_off holds 2 * (n_rows + 1) ints: 64-query then 256-query block offsets,
-// followed by the row of every 256-query block: n_tokens / 256 + n_rows ints).
+// followed by the row of every 256-query block (n_tokens / 256 + n_rows ints)
+// and the row of every 64-query block (n_tokens / 64 + n_rows ints), in all
+// qb_ints(n_rows, n_tokens) ints).
+inline int qb_row64_offset(int n_rows, int n_tokens) { return 2 * (n_rows + 1) + n_tokens / 256 + n_rows; }
+inline size_t qb_ints(int n_rows, int n_tokens) { return (size_t)qb_row64_offset(n_rows, n_tokens) + n_tokens / 64 + n_rows; }
 cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
                         cudaStream_t st);
 
-// x = LN(E[token]) (gain only); xn = x in the activation type.
+// x = LN(E[token]) (gain only); xn = x in the activation type (inv8 > 0, BF16 models: xn holds
+// the E4M3 bytes of x * inv8 instead).
 cudaError_t launch_embed_ln(const int *tokens, int n_tokens, const float *E, int vocab, const float *g, float eps,
-                            float *x, void *xn, bool fp32, unsigned *status, cudaStream_t st);
+                            float *x, void *xn, bool fp32, unsigned *status, cudaStream_t st, float inv8 = 0.f);
 
 // Varlen bidirectional attention inside each row.  qkv [T, 1152] holds
 // q | k | v per token (head h at column h * 64 of each part); window < 0
@@ -49,7 +58,7 @@ struct AttnArgs {
     const void *qkv;
     void *o;
     const int *cu_seqlens;
-    const int *qb_off;        // the prep kernel's block offsets and 256-query block rows
+    const int *qb_off;        // the prep kernel's block offsets and block rows
     int n_rows, n_tokens;
     int window;
     const CUtensorMap *tm_qkv; // BF16 path: box 64 x 64 over [T_cap, 1152]
@@ -78,22 +87,24 @@ cudaError_t launch_marker_attention(const void *qm, const void *qkv, void *om, c
 constexpr int MARKER_PART_ENTRIES_MIN = 4096;  // scratch entries: max(marker capacity, this)
 int marker_attention_splits(int n_markers, int max_row_len, const float *part, int part_entries);
 
-// Scorer: logits[m] from the marker states hm [M, 384].
-struct ScorerArgs {
+// The decision head after the last head layer, one launch: LayerNorm and scorer of every marker
+// state hm [M, 384] (FP32), logits, per-row softmax and read-outs.
+struct HeadArgs {
     const float *hm;
-    int n_markers;
+    int n_markers, n_rows;
+    const int *opt_off;        // [n_rows + 1] markers of each row
+    const int *row_type;       // [n_rows]
     const float *ln_g, *ln_b;
     const float *w1t, *b1;     // MLP: W1 transposed [384 in][384 out], bias [384]
     const float *w2, *b2;      // MLP: [384], [1]; linear variant: W [384], b [1]
     int linear;
     float eps;
-    float *logits;
+    float *logits, *probs;     // [M]
+    int *choice;               // [n_rows]
+    float *score, *noul, *max_p;
     float *tap;                // optional copy of hm
+    unsigned *status;
 };
-cudaError_t launch_scorer(const ScorerArgs &a, cudaStream_t st);
-
-// Per-row softmax and read-outs.
-cudaError_t launch_readout(const float *logits, const int *opt_off, const int *row_type, int n_rows, float *probs,
-                           int *choice, float *score, float *noul, float *max_p, cudaStream_t st);
+cudaError_t launch_head(const HeadArgs &a, cudaStream_t st);
 
 }  // namespace jd

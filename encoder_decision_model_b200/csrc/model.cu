@@ -26,6 +26,7 @@
 #include <string>
 #include <vector>
 
+#include "e4m3.h"
 #include "host_common.h"
 #include "kernels.h"
 
@@ -132,16 +133,19 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D map over [rows, cols] with row stride ld (elements); box = box_cols x box_rows, 128-byte
-// swizzle unless sw64 (64-byte swizzle, for boxes of 32 bf16 columns).
+// swizzle unless sw64 (64-byte swizzle, for boxes of 32 bf16 columns).  Elements are bf16,
+// FP32 (fp32) or bytes (u8: the E4M3 operands of the FP8 QKV GEMM).
 jd_status make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_cols,
-                   uint32_t box_rows, bool fp32 = false, bool sw64 = false) {
+                   uint32_t box_rows, bool fp32 = false, bool sw64 = false, bool u8 = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(JD_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {ld * (fp32 ? 4 : 2)};
+    cuuint64_t strides[1] = {ld * (fp32 ? 4 : (u8 ? 1 : 2))};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t es[2] = {1, 1};
-    CUresult r = fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+    const CUtensorMapDataType dt = fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                        : (u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+    CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, sw64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -153,7 +157,13 @@ struct ProjW {            // one projection weight [N, K]
     void *w = nullptr;    // bf16 or f32 on device
     CUtensorMap tm{};     // BF16 mode only
     CUtensorMap tm64{};   // BF16 mode, 384-wide tiles: box 32 x 192, 64-byte swizzle (residual GEMM)
+    CUtensorMap tm128{};  // BF16 mode, 384-wide tiles: box 64 x 128 (residual GEMM split over a cluster)
     int N = 0, K = 0;
+    // FP8 mode, encoder QKV: E4M3 codes of W[n, :] / s_n (s_n = max_k |W[n, k]| / 448), box 128 x 192,
+    // and per output column the product of the input's activation scale and s_n
+    void *w8 = nullptr;
+    CUtensorMap tm8{};
+    float *col_scale = nullptr;
 };
 
 }  // namespace
@@ -162,6 +172,8 @@ struct jd_model {
     jd_model_config cfg{};
     int device = 0;
     bool fp32 = false;
+    bool fp8 = false;           // JD_PREC_FP8: the encoder QKV projections on E4M3 operands
+    float inv8[22] = {};        // FP8 mode: 1 / activation scale of each encoder layer's QKV input
     int T_cap = 0, B_cap = 0, M_cap = 0;
     size_t bytes = 0;
     std::vector<void *> allocs;
@@ -186,6 +198,8 @@ struct jd_model {
     int mk_part_entries = 0;
     void *xm = nullptr, *qm = nullptr, *om = nullptr, *xnm = nullptr, *ym = nullptr;
     unsigned *status = nullptr;
+    uint8_t *xn8 = nullptr;     // FP8 mode: E4M3 QKV input [T, 384]
+    CUtensorMap tm_xn8{};       // box 128 x 128 bytes
     CUtensorMap tm_xn{}, tm_o{}, tm_y_enc{}, tm_y_head{}, tm_qkv{}, tm_xm{}, tm_om{}, tm_xnm{}, tm_ym{};
     CUtensorMap tm_o64{}, tm_y_enc64{}, tm_y_head64{};  // residual GEMM A operands: box 32 x 128, 64-byte swizzle
     // output maps of the column-split epilogues (box 64 x 32)
@@ -278,9 +292,45 @@ jd_status upload_proj(jd_model *m, const std::vector<float> &h, int r0, int N, i
         // one TMA box per MMA: 192 rows for 384-wide tiles (two N=192 MMAs), else the tile width
         const uint32_t box_rows = bn == 384 ? 192 : (uint32_t)bn;
         TRY(make_map(&p.tm, d, K, N, K, 64, box_rows));
-        if (bn == 384) TRY(make_map(&p.tm64, d, K, N, K, 32, 192, false, true));
+        if (bn == 384) {
+            TRY(make_map(&p.tm64, d, K, N, K, 32, 192, false, true));
+            TRY(make_map(&p.tm128, d, K, N, K, 64, 128));
+        }
     }
     return JD_OK;
+}
+
+// FP8 mode: E4M3 copy of a [N, K] projection with one scale per output row, the row scales
+// multiplied by the scale of its input's activations (act_scale) into col_scale.
+jd_status upload_proj_e4m3(jd_model *m, const std::vector<float> &h, int N, int K, float act_scale, ProjW &p) {
+    p.N = N;
+    p.K = K;
+    std::vector<uint8_t> q((size_t)N * K);
+    std::vector<float> cs(N);
+    for (int n = 0; n < N; ++n) {
+        const float *row = h.data() + (size_t)n * K;
+        float amax = 0.f;
+        for (int k = 0; k < K; ++k) amax = std::max(amax, std::fabs(row[k]));
+        const float sn = amax > 0.f ? amax / 448.0f : 1.0f;
+        for (int k = 0; k < K; ++k) q[(size_t)n * K + k] = e4m3_encode(row[k] / sn);
+        cs[n] = act_scale * sn;
+    }
+    uint8_t *d = nullptr;
+    TRY(m->dalloc(&d, q.size()));
+    CK(cudaMemcpy(d, q.data(), q.size(), cudaMemcpyHostToDevice));
+    p.w8 = d;
+    TRY(make_map(&p.tm8, d, K, N, K, 128, 192, false, false, true));
+    TRY(m->dalloc(&p.col_scale, N));
+    CK(cudaMemcpy(p.col_scale, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice));
+    return JD_OK;
+}
+
+// Scale of an E4M3 LayerNorm output with gain g (no bias): every |y_k| <= sqrt(384) * max |g|
+// (a row's whole variance in one channel), so y / scale never saturates at 448.
+float ln_e4m3_scale(const std::vector<float> &g) {
+    float gm = 0.f;
+    for (float v : g) gm = std::max(gm, std::fabs(v));
+    return std::sqrt((float)D) * (gm > 0.f ? gm : 1.0f) / 448.0f;
 }
 
 jd_status load_proj(jd_model *m, WeightFile &wf, const std::string &name, int N, int K, int bn, ProjW &p) {
@@ -320,6 +370,7 @@ void share_weights(jd_model &v, const jd_model *m) {
     }
     v.sc_g = m->sc_g; v.sc_b = m->sc_b; v.sc_w1t = m->sc_w1t; v.sc_b1 = m->sc_b1; v.sc_w2 = m->sc_w2;
     v.sc_b2 = m->sc_b2; v.lin_w = m->lin_w; v.lin_b = m->lin_b; v.rope_g = m->rope_g; v.rope_l = m->rope_l;
+    for (int l = 0; l < NL; ++l) v.inv8[l] = m->inv8[l];
 }
 
 jd_status load_weights(jd_model *m, const char *path) {
@@ -332,7 +383,16 @@ jd_status load_weights(jd_model *m, const char *path) {
         const std::string p = "enc." + std::to_string(l) + ".";
         if (l != 0) TRY(upload_f32(m, wf, p + "attn_norm.g", {d}, &m->attn_g[l]));
         TRY(upload_f32(m, wf, p + "mlp_norm.g", {d}, &m->mlp_g[l]));
-        TRY(load_proj(m, wf, p + "Wqkv", QKV, D, 384, m->Wqkv[l]));
+        if (m->fp8) {  // the QKV input is the embedding norm's output (layer 0) or this layer's attention norm's
+            std::vector<float> g, w;
+            TRY(read_tensor(wf, l == 0 ? std::string("embed.norm.g") : p + "attn_norm.g", {d}, g));
+            const float sa = ln_e4m3_scale(g);
+            m->inv8[l] = 1.0f / sa;
+            TRY(read_tensor(wf, p + "Wqkv", {(uint32_t)QKV, d}, w));
+            TRY(upload_proj_e4m3(m, w, QKV, D, sa, m->Wqkv[l]));
+        } else {
+            TRY(load_proj(m, wf, p + "Wqkv", QKV, D, 384, m->Wqkv[l]));
+        }
         TRY(load_proj(m, wf, p + "Wo", D, D, 384, m->Wo[l]));
         TRY(load_proj(m, wf, p + "Wo2", D, FF, 384, m->Wo2[l]));
         std::vector<float> wi, il((size_t)2 * FF * D);
@@ -398,7 +458,7 @@ jd_status alloc_workspace(jd_model *m) {
     TRY(m->dalloc(&p, T * HFF * es)); m->y = p;
     TRY(m->dalloc(&m->tok_row, T));
     TRY(m->dalloc(&m->pos, T));
-    TRY(m->dalloc(&m->qb_off, 2 * (B + 1) + T / 256 + B));
+    TRY(m->dalloc(&m->qb_off, qb_ints((int)B, (int)T)));
     TRY(m->dalloc(&m->hm, M * D));
     m->mk_part_entries = std::max((int)M, MARKER_PART_ENTRIES_MIN);
     TRY(m->dalloc(&m->mk_part, (size_t)m->mk_part_entries * NH * (DH + 2)));
@@ -408,6 +468,10 @@ jd_status alloc_workspace(jd_model *m) {
     TRY(m->dalloc(&p, M * D * es)); m->xnm = p;
     TRY(m->dalloc(&p, M * HFF * es)); m->ym = p;
     TRY(m->dalloc(&m->status, 1));
+    if (m->fp8) {
+        TRY(m->dalloc(&m->xn8, T * D));
+        TRY(make_map(&m->tm_xn8, m->xn8, D, T, D, 128, 128, false, false, true));
+    }
     TRY(m->dalloc(&m->i_logits, M));
     TRY(m->dalloc(&m->i_probs, M));
     TRY(m->dalloc(&m->i_choice, B));
@@ -473,6 +537,8 @@ GemmOp make_op(int epi, int bn, const ProjW &w, const CUtensorMap *tmA, const vo
     op.tmXN = tmXN;
     op.tmA64 = tmA64;
     op.tmB64 = tmA64 ? &w.tm64 : nullptr;
+    op.tmBs = tmA64 ? &w.tm128 : nullptr;
+    op.tmBp = tmA64 ? &w.tm : nullptr;  // box 64 x 192 of the 384-wide weights
     op.epi = epi;
     op.bn = bn;
     op.K = w.K;
@@ -517,7 +583,9 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
     const int T = b->n_tokens, B = b->n_rows, M = b->n_markers;
     LK(cudaMemsetAsync(m->status, 0, sizeof(unsigned), st));
     KL("prep", 3, launch_prep(b->cu_seqlens, B, T, m->tok_row, m->pos, m->qb_off, st));
-    KL("embed_ln", 1, launch_embed_ln(b->tokens, T, m->E, VOCAB, m->emb_g, EPS, m->x, m->xn, f32, m->status, st));
+    const bool f8 = m->fp8;
+    KL("embed_ln", 1, launch_embed_ln(b->tokens, T, m->E, VOCAB, m->emb_g, EPS, m->x, f8 ? (void *)m->xn8 : m->xn, f32,
+                                      m->status, st, f8 ? m->inv8[0] : 0.f));
 
     AttnArgs aa;
     aa.qkv = m->qkv;
@@ -538,7 +606,15 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.rope = glob ? m->rope_g : m->rope_l;
         e.pos = m->pos;
         e.rope_cols = 2 * D;
-        KL("gemm_qkv_rope", 1, launch_gemm(make_op(EPI_QKV, 384, m->Wqkv[l], &m->tm_xn, m->xn, D, e, &m->to_qkv), f32, st));
+        if (f8) {
+            e.col_scale = m->Wqkv[l].col_scale;
+            GemmOp op = make_op(EPI_QKV, 384, m->Wqkv[l], &m->tm_xn8, m->xn8, D, e, &m->to_qkv);
+            op.tmB = &m->Wqkv[l].tm8;
+            op.f8 = true;
+            KL("gemm_qkv_rope", 1, launch_gemm(op, false, st));
+        } else {
+            KL("gemm_qkv_rope", 1, launch_gemm(make_op(EPI_QKV, 384, m->Wqkv[l], &m->tm_xn, m->xn, D, e, &m->to_qkv), f32, st));
+        }
 
         aa.window = glob ? -1 : 64;
         KL(glob ? "attn_global" : "attn_local", 1, launch_attention(aa, f32, st));
@@ -570,7 +646,14 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
             e.ln_g = m->n1g[0];
             e.ln_b = m->n1b[0];
         }
-        KL("gemm_wo2_res_ln", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->Wo2[l], &m->tm_y_enc, m->y, FF, e, nullptr, &m->tm_x32, &m->tm_xn, &m->tm_y_enc64), f32, st));
+        GemmOp o2 = make_op(EPI_RESID_LN, 384, m->Wo2[l], &m->tm_y_enc, m->y, FF, e, nullptr, &m->tm_x32, &m->tm_xn,
+                            &m->tm_y_enc64);
+        if (f8 && l + 1 < NL) {  // the next layer's QKV input, as E4M3
+            o2.ep.out = m->xn8;
+            o2.ep.out8_inv_scale = m->inv8[l + 1];
+            o2.out8 = true;
+        }
+        KL("gemm_wo2_res_ln", 1, launch_gemm(o2, f32, st));
     }
 
     // ---- head layer 0 (all tokens)
@@ -640,23 +723,30 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
         e.resid = m->hm;
         KL("head1_gemm_ffn2", 1, launch_gemm(make_op(EPI_RESID_LN, 384, m->lin2[1], &m->tm_ym, m->ym, HFF, e), f32, st));
     }
-    // ---- scorer + read-outs
-    ScorerArgs sa;
-    sa.hm = m->hm;
-    sa.n_markers = M;
-    sa.ln_g = m->sc_g;
-    sa.ln_b = m->sc_b;
-    sa.w1t = m->sc_w1t;
-    sa.b1 = m->sc_b1;
-    sa.linear = m->cfg.scorer == JD_SCORER_LINEAR;
-    sa.w2 = sa.linear ? m->lin_w : m->sc_w2;
-    sa.b2 = sa.linear ? m->lin_b : m->sc_b2;
-    sa.eps = EPS;
-    sa.logits = out->logits;
-    sa.tap = taps ? taps->marker_state : nullptr;
-    KL("scorer", 1, launch_scorer(sa, st));
-    KL("readout", 1, launch_readout(out->logits, b->opt_off, b->row_type, B, out->probs, out->choice, out->score, out->noul,
-                      out->max_p, st));
+    // ---- scorer, softmax and read-outs in one launch
+    HeadArgs ha;
+    ha.hm = m->hm;
+    ha.n_markers = M;
+    ha.n_rows = B;
+    ha.opt_off = b->opt_off;
+    ha.row_type = b->row_type;
+    ha.ln_g = m->sc_g;
+    ha.ln_b = m->sc_b;
+    ha.w1t = m->sc_w1t;
+    ha.b1 = m->sc_b1;
+    ha.linear = m->cfg.scorer == JD_SCORER_LINEAR;
+    ha.w2 = ha.linear ? m->lin_w : m->sc_w2;
+    ha.b2 = ha.linear ? m->lin_b : m->sc_b2;
+    ha.eps = EPS;
+    ha.logits = out->logits;
+    ha.probs = out->probs;
+    ha.choice = out->choice;
+    ha.score = out->score;
+    ha.noul = out->noul;
+    ha.max_p = out->max_p;
+    ha.tap = taps ? taps->marker_state : nullptr;
+    ha.status = m->status;
+    KL("head", 1, launch_head(ha, st));
     if (m->prof && m->n_ev < (int)m->ev.size()) {
         LK(cudaEventRecord(m->ev[m->n_ev], st));
         m->ev_name[m->n_ev++] = nullptr;
@@ -691,6 +781,9 @@ jd_status check_batch(jd_model *m, const jd_batch *b) {
     return JD_OK;
 }
 
+// Resolves the no-allocation path's static array on `dev` (defined with it below).
+jd_status noalloc_prepare(int dev);
+
 }  // namespace
 
 // ================================================================== C ABI
@@ -702,7 +795,7 @@ extern "C" jd_status jd_model_create(const jd_model_config *cfg, const char *wei
     *out = nullptr;
     if (cfg->max_tokens < 1 || cfg->max_rows < 1 || cfg->max_markers < 1)
         return fail(JD_ERR_INVALID_ARG, "capacities must be positive");
-    if (cfg->precision != JD_PREC_BF16 && cfg->precision != JD_PREC_FP32)
+    if (cfg->precision != JD_PREC_BF16 && cfg->precision != JD_PREC_FP32 && cfg->precision != JD_PREC_FP8)
         return fail(JD_ERR_INVALID_ARG, "unknown precision %d", cfg->precision);
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) return fail(JD_ERR_CUDA, "no CUDA device");
@@ -716,6 +809,7 @@ extern "C" jd_status jd_model_create(const jd_model_config *cfg, const char *wei
     m->cfg = *cfg;
     m->device = device;
     m->fp32 = cfg->precision == JD_PREC_FP32;
+    m->fp8 = cfg->precision == JD_PREC_FP8;
     m->T_cap = (cfg->max_tokens + 127) / 128 * 128;
     m->B_cap = cfg->max_rows;
     m->M_cap = (cfg->max_markers + 127) / 128 * 128;
@@ -726,6 +820,9 @@ extern "C" jd_status jd_model_create(const jd_model_config *cfg, const char *wei
     }
     if (s == JD_OK) s = load_weights(m, weights_path);
     if (s == JD_OK) s = alloc_workspace(m);
+    // BF16 models can serve jd_forward_noalloc: load the module that holds its static array
+    // now, at start-up, so that no later call of that entry point allocates.
+    if (s == JD_OK && cfg->precision == JD_PREC_BF16) s = noalloc_prepare(device);
     if (s == JD_OK) {
         cudaError_t e = cudaDeviceSynchronize();
         if (e != cudaSuccess) s = fail(JD_ERR_CUDA, "setup: %s", cudaGetErrorString(e));
@@ -753,6 +850,7 @@ extern "C" jd_status jd_model_create_shared(const jd_model *base, const jd_model
     m->cfg = *cfg;
     m->device = base->device;
     m->fp32 = base->fp32;
+    m->fp8 = base->fp8;
     m->T_cap = (cfg->max_tokens + 127) / 128 * 128;
     m->B_cap = cfg->max_rows;
     m->M_cap = (cfg->max_markers + 127) / 128 * 128;
@@ -977,7 +1075,8 @@ constexpr size_t NA_Y = NA_O + na_up((size_t)NA_TOKENS * D * 2);
 constexpr size_t NA_TOKROW = NA_Y + na_up((size_t)NA_TOKENS * HFF * 2);
 constexpr size_t NA_POS = NA_TOKROW + na_up((size_t)NA_TOKENS * 4);
 constexpr size_t NA_QBOFF = NA_POS + na_up((size_t)NA_TOKENS * 4);
-constexpr size_t NA_HM = NA_QBOFF + na_up((size_t)(2 * (NA_ROWS + 1) + NA_TOKENS / 256 + NA_ROWS) * 4);
+constexpr size_t NA_HM =
+    NA_QBOFF + na_up((size_t)(2 * (NA_ROWS + 1) + NA_TOKENS / 256 + NA_ROWS + NA_TOKENS / 64 + NA_ROWS) * 4);
 constexpr size_t NA_XM = NA_HM + na_up((size_t)NA_MARKERS * D * 4);
 constexpr size_t NA_QM = NA_XM + na_up((size_t)NA_MARKERS * D * 2);
 constexpr size_t NA_OM = NA_QM + na_up((size_t)NA_MARKERS * D * 2);
@@ -1046,6 +1145,7 @@ void noalloc_view(jd_model &v, const jd_model *m, const NoAllocSlot &s) {
     v.cfg = m->cfg;
     v.device = m->device;
     v.fp32 = false;
+    v.fp8 = false;
     share_weights(v, m);
     uint8_t *b = s.base;
     v.x = reinterpret_cast<float *>(b + NA_X);
@@ -1066,12 +1166,18 @@ void noalloc_view(jd_model &v, const jd_model *m, const NoAllocSlot &s) {
     v.graph_mode = false;
 }
 
+jd_status noalloc_prepare(int dev) {
+    if (dev < 0 || dev >= NA_MAX_DEVICES) return JD_OK;  // jd_forward_noalloc refuses such devices
+    std::lock_guard<std::mutex> lock(g_na_mutex);
+    return noalloc_setup(dev);
+}
+
 }  // namespace
 
 extern "C" jd_status jd_forward_noalloc(jd_model *m, const jd_batch *b, float *logits, void *stream) {
     clear_error();
     if (!m || !b || !logits) return fail(JD_ERR_INVALID_ARG, "NULL argument");
-    if (m->fp32) return fail(JD_ERR_INVALID_ARG, "jd_forward_noalloc serves BF16 models only");
+    if (m->cfg.precision != JD_PREC_BF16) return fail(JD_ERR_INVALID_ARG, "jd_forward_noalloc serves BF16 models only");
     if (m->device < 0 || m->device >= NA_MAX_DEVICES) return fail(JD_ERR_INVALID_ARG, "device ordinal too large");
     if (b->n_rows < 1 || b->n_tokens < 1 || b->n_markers < 1) return fail(JD_ERR_INVALID_ARG, "empty batch");
     if (b->n_tokens > NA_TOKENS || b->n_rows > NA_ROWS || b->n_markers > NA_MARKERS)
@@ -1091,4 +1197,25 @@ extern "C" jd_status jd_forward_noalloc(jd_model *m, const jd_batch *b, float *l
                  reinterpret_cast<float *>(base + NA_MAXP)};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return enqueue_forward(&v, b, &o, nullptr, st);
+}
+
+extern "C" jd_status jd_noalloc_check_status(jd_model *m, void *stream) {
+    clear_error();
+    if (!m) return fail(JD_ERR_INVALID_ARG, "model is NULL");
+    if (m->cfg.precision != JD_PREC_BF16) return fail(JD_ERR_INVALID_ARG, "jd_forward_noalloc serves BF16 models only");
+    if (m->device < 0 || m->device >= NA_MAX_DEVICES) return fail(JD_ERR_INVALID_ARG, "device ordinal too large");
+    CK(cudaSetDevice(m->device));
+    uint8_t *base = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_na_mutex);
+        TRY(noalloc_setup(m->device));
+        base = g_na_slot[m->device].base;
+    }
+    CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    unsigned stv = 0;
+    CK(cudaMemcpy(&stv, base + NA_STATUS, sizeof(unsigned), cudaMemcpyDeviceToHost));
+    if (stv)
+        return fail(JD_ERR_DEVICE_STATUS, "jd_forward_noalloc device status 0x%x (1: wait timeout, 2: token id range, 4: index)",
+                    stv);
+    return JD_OK;
 }

@@ -55,15 +55,17 @@ def test_outlier_channels_reach_thousands(outlier_weights):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+@pytest.mark.parametrize("precision", ["bf16", "fp32", "fp8"])
 def test_outlier_residual_parity(outlier_weights, precision):
+    """FP8 mode (E4M3 encoder QKV projections) is held to the BF16 bounds."""
     from encoder_decision_model_b200 import _lib as jl
     from encoder_decision_model_b200.build import build
     from gpu_helpers import compare, device_run, oracle_run
 
     build()
-    bf16 = precision == "bf16"
-    m = jl.Model(outlier_weights, 16384, 64, 1024, precision=jl.JD_PREC_BF16 if bf16 else jl.JD_PREC_FP32)
+    bf16 = precision != "fp32"
+    prec = {"bf16": jl.JD_PREC_BF16, "fp32": jl.JD_PREC_FP32, "fp8": jl.JD_PREC_FP8}[precision]
+    m = jl.Model(outlier_weights, 16384, 64, 1024, precision=prec)
     rows = rows_config1() + rows_config2(4)
     hb, res = device_run(m, rows, OPT1, taps=True)
     ref = oracle_run(outlier_weights, rows, OPT1)

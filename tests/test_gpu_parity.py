@@ -1,7 +1,8 @@
 """GPU parity: the CUDA path through the C ABI against the CPU oracle.
 
 Tolerances (per row, against the float64 oracle):
-  BF16 mode  |delta logit| <= 3e-2, |delta p| <= 5e-3, same argmax where the
+  BF16 mode, and FP8 mode (E4M3 encoder QKV projections) at the same bounds:
+             |delta logit| <= 3e-2, |delta p| <= 5e-3, same argmax where the
              oracle's top-2 gap exceeds 0.05; relative L2 error of the encoder
              output and of the marker states <= 3e-2.
   FP32 mode  |delta logit| <= 1e-3, |delta p| <= 1e-4, relative L2 error of
@@ -37,6 +38,13 @@ def fp32_model(lib_built, weights_file):
 
 
 @pytest.fixture(scope="module")
+def fp8_model(lib_built, weights_file):
+    m = jl.Model(weights_file, 65536, 256, 4096, precision=jl.JD_PREC_FP8)
+    yield m
+    m.close()
+
+
+@pytest.fixture(scope="module")
 def bf16_model(lib_built, weights_file):
     m = jl.Model(weights_file, 65536, 256, 4096, precision=jl.JD_PREC_BF16)
     yield m
@@ -67,6 +75,15 @@ def test_fp32_mode_matches_oracle(fp32_model, weights_file, cfg):
     hb, res = device_run(fp32_model, rows, opts, taps=True)
     ref = oracle_run(weights_file, rows, opts)
     compare(hb, res, ref, bf16=False, label=f"fp32 {cfg}")
+
+
+@pytest.mark.parametrize("cfg", ["c0", "c1", "c2", "edge"])
+def test_fp8_qkv_mode_matches_oracle_at_bf16_bounds(fp8_model, weights_file, cfg):
+    rows, opts = {"c0": (rows_config0(), OPT0), "c1": (rows_config1(), OPT1),
+                  "c2": (rows_config2(12), OPT1), "edge": (edge_rows(), OPT1)}[cfg]
+    hb, res = device_run(fp8_model, rows, opts, taps=True)
+    ref = oracle_run(weights_file, rows, opts)
+    compare(hb, res, ref, bf16=True, label=f"fp8 {cfg}")
 
 
 @pytest.mark.parametrize("cfg", ["c0", "c1", "c2", "edge"])

@@ -1,0 +1,122 @@
+"""Why the FP8 mode quantizes the encoder QKV projections and nothing else.
+
+"Julia-1 MLX", "Performance": the projections may run below FP32 while the
+residual stream stays FP32, because a few residual channels reach values near
+4000.  This test emulates FP8 E4M3 operands inside the oracle's encoder layer
+(round to nearest even on the E4M3 grid, saturating at 448) and measures the
+relative error of the encoder output against the exact oracle, for the
+seed-0 weights and for the outlier construction of the GPU outlier test
+(layer 0's Wo2 rows 5, 77, 200, 311 scaled by 6e4, so those residual channels
+sit in the thousands):
+
+  * E4M3 QKV inputs and weights (static per-layer activation scale, per-row
+    weight scales, as the library's FP8 mode): well inside the BF16 tap bound
+    3e-2 on both weight sets;
+  * E4M3 QKV and GEGLU up-projection (per-token activation scale): beyond 3e-2
+    on the outlier construction -- the GEGLU output's 3-bit-mantissa error
+    reaches the outlier channels through Wo2 and, from there, every later
+    LayerNorm.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import model as om
+from oracle import serialize_row, EncodeOptions
+from workloads import rows_config1
+
+CH = [5, 77, 200, 311]
+
+
+def e4m3(x):
+    """Nearest E4M3 value (ties to the even mantissa), saturating at +-448."""
+    x = np.asarray(x, np.float64)
+    a = np.abs(x)
+    e = np.maximum(np.floor(np.log2(np.maximum(a, 1e-300))), -6.0)  # subnormals share 2^-6's quantum
+    q = 2.0 ** (e - 3)
+    return np.sign(x) * np.minimum(np.round(a / q) * q, 448.0)
+
+
+def test_e4m3_grid():
+    # the normal grid of [1, 2): 1 + m/8; ties go to the even mantissa; 2^-9 is the smallest step
+    np.testing.assert_array_equal(e4m3([1.0, 1.0625, 1.1875, 1.3125, 447.0, 460.0, 2.0 ** -10, 3 * 2.0 ** -10]),
+                                  [1.0, 1.0, 1.25, 1.25, 448.0, 448.0, 0.0, 2.0 ** -8])
+    v = np.array([(1 + m / 8) * 2.0 ** e for e in range(-6, 9) for m in range(8)] + [m * 2.0 ** -9 for m in range(8)])
+    v = v[v <= 448]
+    np.testing.assert_array_equal(e4m3(v), v)
+
+
+def _q_rows(W):
+    s = np.abs(W).max(axis=-1, keepdims=True) / 448.0
+    return e4m3(W / s) * s
+
+
+def _q_tokens(x):
+    s = np.abs(x).max(axis=-1, keepdims=True) / 448.0
+    s = np.where(s == 0, 1.0, s)
+    return e4m3(x / s) * s
+
+
+class _Overrides:
+    def __init__(self, base, over):
+        self.base, self.over = base, over
+
+    def __getitem__(self, k):
+        return self.over[k] if k in self.over else self.base[k]
+
+    def embed_rows(self, ids):
+        return self.base.embed_rows(ids)
+
+
+def _layer(fp8_wi):
+    """The oracle's encoder layer with E4M3 QKV (and, with fp8_wi, E4M3 GEGLU up-projection)."""
+    def layer(x, W, l, mo):
+        L, d = x.shape
+        H = mo.n_heads
+        p = f"enc.{l}."
+        h = x if l == 0 else om.layer_norm(x, W[p + "attn_norm.g"], eps=mo.eps)
+        gmax = np.abs(W["embed.norm.g"] if l == 0 else W[p + "attn_norm.g"]).max()
+        s = math.sqrt(d) * gmax / 448.0  # the bound of a LayerNorm output
+        qkv = (e4m3(h / s) * s) @ _q_rows(W[p + "Wqkv"]).T
+        q, k, v = (qkv[:, i * d:(i + 1) * d].reshape(L, H, d // H) for i in range(3))
+        glob = (l % mo.global_every) == 0
+        th = mo.theta_global if glob else mo.theta_local
+        o = om.attention(om.rope(q, th), om.rope(k, th), v, window=None if glob else mo.window)
+        x = x + o.reshape(L, d) @ W[p + "Wo"].T
+        xn = om.layer_norm(x, W[p + "mlp_norm.g"], eps=mo.eps)
+        ug = (_q_tokens(xn) @ _q_rows(W[p + "Wi"]).T) if fp8_wi else xn @ W[p + "Wi"].T
+        f = ug.shape[1] // 2
+        return x + (om.gelu(ug[:, :f]) * ug[:, f:]) @ W[p + "Wo2"].T
+    return layer
+
+
+def _encoder_error(m, enc, fp8_wi, monkeypatch):
+    ref = m.encode(enc.ids)
+    with monkeypatch.context() as mp:
+        mp.setattr(om, "encoder_layer", _layer(fp8_wi))
+        got = m.encode(enc.ids)
+    return float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+
+
+@pytest.fixture(scope="module")
+def row():
+    return serialize_row(rows_config1()[2], EncodeOptions(max_length=1024, head_budget=512))
+
+
+def test_fp8_qkv_only_stays_inside_the_bf16_bound(oracle_model, row, monkeypatch):
+    err = _encoder_error(oracle_model, row, False, monkeypatch)
+    assert err < 1e-2, err
+    W = oracle_model.W
+    out = om.OracleModel(_Overrides(W, {"enc.0.Wo2": W["enc.0.Wo2"] * np.where(
+        np.isin(np.arange(384), CH), 6.0e4, 1.0)[:, None]}))
+    err_o = _encoder_error(out, row, False, monkeypatch)
+    assert err_o < 1e-2, err_o
+
+
+def test_fp8_geglu_input_breaks_the_bound_on_outlier_channels(oracle_model, row, monkeypatch):
+    W = oracle_model.W
+    out = om.OracleModel(_Overrides(W, {"enc.0.Wo2": W["enc.0.Wo2"] * np.where(
+        np.isin(np.arange(384), CH), 6.0e4, 1.0)[:, None]}))
+    err_o = _encoder_error(out, row, True, monkeypatch)
+    assert err_o > 3e-2, err_o
