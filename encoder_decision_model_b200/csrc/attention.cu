@@ -322,21 +322,41 @@ __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
     // Masks on the raw scores; the scale goes into the exponent's FMA below.  Key kj of 8-column
     // block j lies kj - qi = 8j - 64 + (2tq + e) - g (- 8 for qi1) from the query, which is inside
     // [-63, 63] for 2 <= j < 16: only the two outer chunks at each end need the window test.
-    // four interleaved partial maxima per query row: dependency chains of 9, not 36
+    // Four interleaved partial maxima per query row: dependency chains of 9, not 36.  A warp whose
+    // 144 keys all lie in the row (most warps of rows longer than a few hundred tokens) skips the
+    // per-key row tests: a warp-uniform branch between two copies of the loop.
     float mp0[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, mp1[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    const int kw = kbase + warp * 16;  // the warp's first key
+    if (kw >= cs && kw + 16 * LW_CHUNKS <= ce) {
 #pragma unroll
-    for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
-        const bool edge = j < 2 || j >= 2 * LW_CHUNKS - 2;
+        for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
+            const bool edge = j < 2 || j >= 2 * LW_CHUNKS - 2;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int kj = kbase + (warp * 2 + j) * 8 + 2 * tq + e;
-            const bool in_row = kj >= cs && kj < ce;
-            const bool v0 = in_row && (!edge || abs(qi0 - kj) <= 64);
-            const bool v1 = in_row && (!edge || abs(qi1 - kj) <= 64);
-            sc[j][e] = v0 ? sc[j][e] : -INFINITY;
-            sc[j][2 + e] = v1 ? sc[j][2 + e] : -INFINITY;
-            mp0[(2 * j + e) & 3] = fmaxf(mp0[(2 * j + e) & 3], sc[j][e]);
-            mp1[(2 * j + e) & 3] = fmaxf(mp1[(2 * j + e) & 3], sc[j][2 + e]);
+            for (int e = 0; e < 2; ++e) {
+                if (edge) {
+                    const int kj = kw + j * 8 + 2 * tq + e;
+                    sc[j][e] = abs(qi0 - kj) <= 64 ? sc[j][e] : -INFINITY;
+                    sc[j][2 + e] = abs(qi1 - kj) <= 64 ? sc[j][2 + e] : -INFINITY;
+                }
+                mp0[(2 * j + e) & 3] = fmaxf(mp0[(2 * j + e) & 3], sc[j][e]);
+                mp1[(2 * j + e) & 3] = fmaxf(mp1[(2 * j + e) & 3], sc[j][2 + e]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
+            const bool edge = j < 2 || j >= 2 * LW_CHUNKS - 2;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int kj = kw + j * 8 + 2 * tq + e;
+                const bool in_row = kj >= cs && kj < ce;
+                const bool v0 = in_row && (!edge || abs(qi0 - kj) <= 64);
+                const bool v1 = in_row && (!edge || abs(qi1 - kj) <= 64);
+                sc[j][e] = v0 ? sc[j][e] : -INFINITY;
+                sc[j][2 + e] = v1 ? sc[j][2 + e] : -INFINITY;
+                mp0[(2 * j + e) & 3] = fmaxf(mp0[(2 * j + e) & 3], sc[j][e]);
+                mp1[(2 * j + e) & 3] = fmaxf(mp1[(2 * j + e) & 3], sc[j][2 + e]);
+            }
         }
     }
     float mx0 = fmaxf(fmaxf(mp0[0], mp0[1]), fmaxf(mp0[2], mp0[3]));

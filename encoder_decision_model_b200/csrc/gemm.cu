@@ -830,7 +830,7 @@ struct RsCfg {
     static constexpr int RING = STAGES * STAGE;
     static constexpr int XCH = 128 * 32 * 4;     // residual chunk: 128 rows x 32 FP32
     static constexpr int NX = NC / 32;
-    static constexpr int MOM = NS * 128 * 8;     // (mean, M2) of every row from every rank
+    static constexpr int MOM = 12 * 128 * 8;     // (mean, M2) of every row's twelve 32-column chunks
     static constexpr int DATA = RING + NX * XCH + MOM;
     static constexpr int BAR_BYTES = (2 * STAGES + 1 + NX) * 8 + 8;
     static constexpr int SMEM = DATA + BAR_BYTES + 1024;
@@ -856,7 +856,7 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *xbuf = smem + C::RING;
-    float2 *mom = reinterpret_cast<float2 *>(smem + C::RING + C::NX * C::XCH);  // [NS][128]
+    float2 *mom = reinterpret_cast<float2 *>(smem + C::RING + C::NX * C::XCH);  // [12 chunks][128 rows]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::DATA);
     uint64_t *empty = full + C::STAGES;
     uint64_t *accf = empty + C::STAGES;
@@ -934,8 +934,8 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
         mbar_wait(accf, 0, ep.status);
         __syncwarp();
         tc_fence_after();
-        // ---- pass 1: v = x + acc (+ bias) for this CTA's columns; moments over them
-        float cnt = 0.f;
+        // ---- pass 1: v = x + acc (+ bias) for this CTA's columns; each 32-column chunk's
+        //      (mean, M2) goes to slot [global chunk][row] of every CTA of the cluster
 #pragma unroll 1
         for (int c = 0; c < C::NX; ++c) {
             uint32_t a[32];
@@ -961,15 +961,14 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
             float cq = 0.f;
 #pragma unroll
             for (int j = 0; j < 32; ++j) cq += (v[j] - cm) * (v[j] - cm);
-            if (c == 0) {
-                mean = cm;
-                m2 = cq;
-                cnt = 32.f;
-            } else {
-                const float tot = cnt + 32.f, dl = cm - mean;
-                mean += dl * (32.f / tot);
-                m2 += cq + dl * dl * (cnt * 32.f / tot);
-                cnt = tot;
+            {
+                const uint32_t local = smem_u32(&mom[((int)rank * C::NX + c) * 128 + r]);
+#pragma unroll
+                for (int j = 0; j < NS; ++j) {
+                    uint32_t remote;
+                    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(j));
+                    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(cm), "f"(cq) : "memory");
+                }
             }
 #pragma unroll
             for (int j4 = 0; j4 < 8; ++j4)
@@ -987,30 +986,29 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
             }
         }
         tmem_st_wait();
-        // this CTA's (mean, M2) of row r, to slot [rank][r] of every CTA of the cluster
-        const uint32_t local = smem_u32(&mom[rank * 128 + r]);
-#pragma unroll
-        for (int j = 0; j < NS; ++j) {
-            uint32_t remote;
-            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(j));
-            asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(mean), "f"(m2) : "memory");
-        }
     }
     __syncwarp();
     rs_cluster_sync();
     if (warp >= 2) {
-        // ---- merge the NS partial moments (equal counts NC) in rank order
-        float mu = 0.f;
-#pragma unroll
-        for (int j = 0; j < NS; ++j) mu += mom[j * 128 + r].x;
-        mu *= 1.0f / NS;
-        float tot = 0.f;
-#pragma unroll
-        for (int j = 0; j < NS; ++j) {
-            const float2 p = mom[j * 128 + r];
-            tot += p.y + (float)C::NC * (p.x - mu) * (p.x - mu);
+        // ---- the twelve chunks' moments merged in column order with k_gemm_rl's update, so the
+        //      row's mean and M2 -- and the outputs -- are bit-identical to the unsplit kernel's
+        float cnt = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 12; ++c) {
+            const float2 p = mom[c * 128 + r];
+            if (c == 0) {
+                mean = p.x;
+                m2 = p.y;
+                cnt = 32.f;
+            } else {
+                const float tot = cnt + 32.f, dl = p.x - mean;
+                mean += dl * (32.f / tot);
+                m2 += p.y + dl * dl * (cnt * 32.f / tot);
+                cnt = tot;
+            }
         }
-        const float rstd = 1.0f / sqrtf(tot * (1.0f / D) + ep.eps);
+        const float mu = mean;
+        const float rstd = 1.0f / sqrtf(m2 * (1.0f / D) + ep.eps);
         // ---- pass 2: LayerNorm of this CTA's columns from TMEM, stored from registers
         const int row = m0 + r;
 #pragma unroll 1
@@ -1088,7 +1086,7 @@ struct RpCfg {
     static constexpr int XCH = 128 * 32 * 4;       // residual chunk: 128 rows x 32 FP32
     static constexpr int NX = NC / 32;             // residual chunks per tile
     static constexpr int NXB = 4;                  // residual buffers
-    static constexpr int MOM = 2 * NS * 128 * 8;   // (mean, M2): [tile parity][rank][row]
+    static constexpr int MOM = 2 * 12 * 128 * 8;   // (mean, M2): [tile parity][32-column chunk][row]
     static constexpr int DATA = RING + NXB * XCH + MOM;
     static constexpr int NBAR = 2 * STAGES + 2 + 2 + NXB + 2;
     static constexpr int SMEM = DATA + NBAR * 8 + 8 + 1024;
@@ -1139,7 +1137,7 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *xbuf = smem + C::RING;
-    float2 *mom = reinterpret_cast<float2 *>(smem + C::RING + C::NXB * C::XCH);  // [2][NS][128]
+    float2 *mom = reinterpret_cast<float2 *>(smem + C::RING + C::NXB * C::XCH);  // [2][12][128]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::DATA);
     uint64_t *empty = full + C::STAGES;
     uint64_t *accf = empty + C::STAGES;  // [2]
@@ -1246,8 +1244,8 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
             mbar_wait(&accf[b], (tc >> 1) & 1, ep.status);
             __syncwarp();
             tc_fence_after();
-            float cnt = 0.f, mean = 0.f, m2 = 0.f;
-            // ---- pass 1: v = x + acc (+ bias) for this CTA's columns; moments over them
+            // ---- pass 1: v = x + acc (+ bias) for this CTA's columns; each 32-column chunk's
+            //      (mean, M2) goes to slot [tile parity][global chunk][row] of both CTAs
 #pragma unroll 1
             for (int c = 0; c < C::NX; ++c) {
                 const uint32_t g = tc * C::NX + c, xb_i = g % C::NXB;
@@ -1274,15 +1272,15 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
                 float cq = 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) cq += (v[j] - cm) * (v[j] - cm);
-                if (c == 0) {
-                    mean = cm;
-                    m2 = cq;
-                    cnt = 32.f;
-                } else {
-                    const float tot = cnt + 32.f, dl = cm - mean;
-                    mean += dl * (32.f / tot);
-                    m2 += cq + dl * dl * (cnt * 32.f / tot);
-                    cnt = tot;
+                {
+                    const uint32_t local = smem_u32(&mom[((int)b * 12 + (int)rank * C::NX + c) * 128 + r]);
+#pragma unroll
+                    for (int j = 0; j < NS; ++j) {
+                        uint32_t remote;
+                        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(j));
+                        asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(cm), "f"(cq)
+                                     : "memory");
+                    }
                 }
 #pragma unroll
                 for (int j4 = 0; j4 < 8; ++j4)
@@ -1312,29 +1310,29 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
                 }
             }
             tmem_st_wait();
-            // ---- moments of this CTA's half to both CTAs, then merge the halves in rank order
-            float2 *slot = mom + (size_t)(b * NS + rank) * 128 + r;
-#pragma unroll
-            for (int j = 0; j < NS; ++j) {
-                uint32_t remote;
-                asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(slot)), "r"(j));
-                asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(mean), "f"(m2) : "memory");
-            }
-            // each thread releases its own stores with its arrivals
+            // each thread releases its own stores with its arrivals on both CTAs' barriers
 #pragma unroll
             for (int j = 0; j < NS; ++j) mbar_arrive_remote(&momf[b], (uint32_t)j);
             mbar_wait_cluster(&momf[b], (tc >> 1) & 1, ep.status);
-            float mu = 0.f;
-#pragma unroll
-            for (int j = 0; j < NS; ++j) mu += mom[(size_t)(b * NS + j) * 128 + r].x;
-            mu *= 1.0f / NS;
-            float tot = 0.f;
-#pragma unroll
-            for (int j = 0; j < NS; ++j) {
-                const float2 p = mom[(size_t)(b * NS + j) * 128 + r];
-                tot += p.y + (float)C::NC * (p.x - mu) * (p.x - mu);
+            // ---- the twelve chunks' moments merged in column order with k_gemm_rl's update, so the
+            //      row's mean and M2 -- and the outputs -- are bit-identical to the unsplit kernel's
+            float cnt = 0.f, mean = 0.f, m2 = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < 12; ++c) {
+                const float2 p = mom[((int)b * 12 + c) * 128 + r];
+                if (c == 0) {
+                    mean = p.x;
+                    m2 = p.y;
+                    cnt = 32.f;
+                } else {
+                    const float tot = cnt + 32.f, dl = p.x - mean;
+                    mean += dl * (32.f / tot);
+                    m2 += p.y + dl * dl * (cnt * 32.f / tot);
+                    cnt = tot;
+                }
             }
-            const float rstd = 1.0f / sqrtf(tot * (1.0f / D) + ep.eps);
+            const float mu = mean;
+            const float rstd = 1.0f / sqrtf(m2 * (1.0f / D) + ep.eps);
             // ---- pass 2: LayerNorm of this CTA's columns from TMEM
             const int row = m0 + r;
 #pragma unroll 1

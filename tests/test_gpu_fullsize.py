@@ -84,6 +84,14 @@ def test_throughput_full_size(weights_file):
         r = om.forward_all(serialize_row(rows[i], eo))
         worst = max(worst, _check_row(hb, res, enc, i, r["logits"], r["marker_state"], r["encoder_out"]))
     print(f"throughput 1024 rows: sampled rows {sample}, max |delta logit| {worst:.2e}")
+    # a row's result does not depend on its batch: the sampled rows scored alone (a batch of a few
+    # row tiles, which takes the cluster-split residual GEMM) give the same logits bit for bit
+    small = jl.Model(weights_file, 8192, 8, 256)
+    for i in sample:
+        alone = small.jd_decide_host([rows[i]], jl.encode_opts(**opts))
+        a, b = hb.opt_off[i], hb.opt_off[i + 1]
+        assert np.array_equal(alone["logits"], res["logits"][a:b]), (i, alone["logits"] - res["logits"][a:b])
+    small.close()
     model.close()
 
 
@@ -129,7 +137,7 @@ def test_router_workload(weights_file):
     for r in (0, 137, 511):
         q = reqs[r]
         rows = [Row(state=q.state, question=q.question, options=q.labels[g:g + 20], qtype=0) for g in range(0, 72, 20)]
-        ho = model.jd_decide_host(rows, opts)
+        ho = model.jd_decide_host(rows, opts)  # a row's result does not depend on its batch
         off = np.cumsum([0] + [len(x.options) for x in rows])
         expect = []
         for gi, g in enumerate(range(0, 72, 20)):
