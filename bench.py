@@ -52,8 +52,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=3)
     ap.add_argument("--fp8-steps", type=int, default=3, help="profiled steps of the FP8-mode leg (0: skip)")
-    ap.add_argument("--long-rows", type=int, default=4,
-                    help="rows of the bounded long-context leg (8192 tokens each; 0: skip)")
+    ap.add_argument("--long-rows", type=int, default=16,
+                    help="rows of the long-context leg (8192 tokens each; 0: skip)")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
 

@@ -54,6 +54,14 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t 
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(addr));
 }
+// P (FP16) times V (FP16): the second product of every attention kernel here
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -182,8 +190,8 @@ __global__ void __launch_bounds__(128)
             const float p2 = exp2f(sc[j][2] - mu1), p3 = exp2f(sc[j][3] - mu1);
             rs0 += p0 + p1;
             rs1 += p2 + p3;
-            pa[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p0, p1);
-            pa[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+            pa[j >> 1][(j & 1) * 2 + 0] = pack_f16x2(p0, p1);
+            pa[j >> 1][(j & 1) * 2 + 1] = pack_f16x2(p2, p3);
         }
         l0 = l0 * c0 + rs0;
         l1 = l1 * c1 + rs1;
@@ -199,8 +207,8 @@ __global__ void __launch_bounds__(128)
             for (int dp = 0; dp < 4; ++dp) {
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4_t(vb + sw128(vr, dp * 2 + (lane >> 4)), b0, b1, b2, b3);
-                mma_bf16(o[2 * dp], pa[kk], b0, b1);
-                mma_bf16(o[2 * dp + 1], pa[kk], b2, b3);
+                mma_f16(o[2 * dp], pa[kk], b0, b1);
+                mma_f16(o[2 * dp + 1], pa[kk], b2, b3);
             }
         }
         __syncthreads();
@@ -244,10 +252,11 @@ __global__ void __launch_bounds__(128)
 // [q0 - 64, q0 + 128), loaded once by TMA (three 64 x 64 tiles of K and of V);
 // warp w's 16 queries need only the 144 keys [q0 + 16w - 64, q0 + 16w + 80),
 // i.e. nine 16-key chunks, so each warp visits just those and runs an exact
-// two-pass softmax over them in registers (no running rescale).  A CTA finds
-// its row in the prep kernel's table of the row of every 64-query block (tb_row)
-// with one load: the binary search over the row offsets it replaced cost about
-// a fifth of the kernel's time (a chain of dependent L2 loads per CTA).
+// two-pass softmax over them in registers (no running rescale).  A CTA reads
+// its row's span and first query from the prep kernel's table of every 64-query
+// block, independent loads in one round trip to L2: a binary search over the
+// row offsets (a chain of dependent loads per CTA) cost about a fifth of the
+// kernel's time, and a row lookup followed by the row's offsets a tenth.
 constexpr int LW_CHUNKS = 9;  // (16 + 2 * 64) / 16
 // Two heads per CTA (8 warps, 2 CTAs per SM): 16 resident warps per SM instead of 12.
 constexpr int LOC_HEADS = 2;
@@ -258,8 +267,7 @@ constexpr int LOC_SMEM = LOC_HEADS * LOC_HEAD_BYTES + 1024;
 
 __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
     k_attn_local_bf16(const __grid_constant__ CUtensorMap tm, __nv_bfloat16 *__restrict__ out,
-                      const int *__restrict__ cu, const int *__restrict__ qb_off, const int *__restrict__ tb_row,
-                      int n_rows, unsigned *status) {
+                      const int *__restrict__ qb_off, const int *__restrict__ span, int n_rows, unsigned *status) {
     extern __shared__ __align__(16) uint8_t sm_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 8 * LOC_HEADS + 1023) &
                                               ~uintptr_t(1023));
@@ -270,10 +278,11 @@ __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm_raw) + hh;
 
     const int tile = blockIdx.x, h = blockIdx.y * LOC_HEADS + hh;
-    if (tile >= qb_off[n_rows]) return;
-    const int row = tb_row[tile];
-    const int cs = cu[row], ce = cu[row + 1];
-    const int q0 = cs + (tile - qb_off[row]) * BQ;
+    // the block count and the block's span are independent loads (one round trip to L2); the
+    // span entries of blocks past the count exist (the table covers the grid) and are not used
+    const int n_blocks = qb_off[n_rows];
+    const int cs = span[3 * tile], ce = span[3 * tile + 1], q0 = span[3 * tile + 2];
+    if (tile >= n_blocks) return;
     const int kbase = q0 - 64;         // band start (may precede the row: masked)
     const int warp = (threadIdx.x >> 5) & 3, lane = threadIdx.x & 31;  // warp inside the head's group
 
@@ -366,18 +375,21 @@ __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
     const float mu0 = mx0 == -INFINITY ? 0.f : -mx0 * sl2, mu1 = mx1 == -INFINITY ? 0.f : -mx1 * sl2;
-    float lp0[2] = {0.f, 0.f}, lp1[2] = {0.f, 0.f};  // two interleaved partial sums per row
+    // P in FP16 pairs straight from the special-function unit (one ex2 for two keys), the row
+    // sums as FP16 pair sums (three interleaved per row, at most six adds each, values <= 1)
+    uint32_t hp0[3] = {0u, 0u, 0u}, hp1[3] = {0u, 0u, 0u};
     uint32_t pa[LW_CHUNKS][4];
 #pragma unroll
     for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
-        const float p0 = ex2_ftz(fmaf(sc[j][0], sl2, mu0)), p1 = ex2_ftz(fmaf(sc[j][1], sl2, mu0));
-        const float p2 = ex2_ftz(fmaf(sc[j][2], sl2, mu1)), p3 = ex2_ftz(fmaf(sc[j][3], sl2, mu1));
-        lp0[j & 1] += p0 + p1;
-        lp1[j & 1] += p2 + p3;
-        pa[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p0, p1);
-        pa[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+        const uint32_t h01 = ex2_f16x2(fmaf(sc[j][0], sl2, mu0), fmaf(sc[j][1], sl2, mu0));
+        const uint32_t h23 = ex2_f16x2(fmaf(sc[j][2], sl2, mu1), fmaf(sc[j][3], sl2, mu1));
+        hp0[j % 3] = hadd2_u32(hp0[j % 3], h01);
+        hp1[j % 3] = hadd2_u32(hp1[j % 3], h23);
+        pa[j >> 1][(j & 1) * 2 + 0] = h01;
+        pa[j >> 1][(j & 1) * 2 + 1] = h23;
     }
-    float l0 = lp0[0] + lp0[1], l1 = lp1[0] + lp1[1];
+    float l0 = hsum2_f32(hp0[0]) + hsum2_f32(hp0[1]) + hsum2_f32(hp0[2]);
+    float l1 = hsum2_f32(hp1[0]) + hsum2_f32(hp1[1]) + hsum2_f32(hp1[2]);
     float o[8][4];
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
@@ -390,8 +402,8 @@ __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
         for (int dp = 0; dp < 4; ++dp) {
             uint32_t b0, b1, b2, b3;
             ldsm_x4_t(vb + sw128(vr, dp * 2 + (lane >> 4)), b0, b1, b2, b3);
-            mma_bf16(o[2 * dp], pa[cc], b0, b1);
-            mma_bf16(o[2 * dp + 1], pa[cc], b2, b3);
+            mma_f16(o[2 * dp], pa[cc], b0, b1);
+            mma_f16(o[2 * dp + 1], pa[cc], b2, b3);
         }
     }
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -517,8 +529,8 @@ cudaError_t launch_attention(const AttnArgs &a, bool fp32, cudaStream_t st) {
         const int smem = 5 * 8192 + 64 + 1024;
         if (local && a.window == 64)
             k_attn_local_bf16<<<dim3(max_tiles, NH / LOC_HEADS), 128 * LOC_HEADS, LOC_SMEM, st>>>(
-                *a.tm_qkv, (__nv_bfloat16 *)a.o, a.cu_seqlens, a.qb_off,
-                a.qb_off + qb_row64_offset(a.n_rows, a.n_tokens), a.n_rows, a.status);
+                *a.tm_qkv, (__nv_bfloat16 *)a.o, a.qb_off, a.qb_off + qb_span_offset(a.n_rows, a.n_tokens), a.n_rows,
+                a.status);
         else if (local)
             k_attn_bf16<true><<<grid, 128, smem, st>>>(*a.tm_qkv, (__nv_bfloat16 *)a.o, a.cu_seqlens, a.qb_off,
                                                        a.n_rows, a.window, a.status);
@@ -740,8 +752,8 @@ __global__ void __launch_bounds__(64)
                     const float p2 = exp2f(sc[j][2] - mu1), p3 = exp2f(sc[j][3] - mu1);
                     rs0 += p0 + p1;
                     rs1 += p2 + p3;
-                    pa[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p0, p1);
-                    pa[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+                    pa[j >> 1][(j & 1) * 2 + 0] = pack_f16x2(p0, p1);
+                    pa[j >> 1][(j & 1) * 2 + 1] = pack_f16x2(p2, p3);
                 }
                 l0 = l0 * c0 + rs0;
                 l1 = l1 * c1 + rs1;
@@ -757,8 +769,8 @@ __global__ void __launch_bounds__(64)
                     for (int dp = 0; dp < 4; ++dp) {
                         uint32_t b0, b1, b2, b3;
                         ldsm_x4_t(vb + sw128(vr, dp * 2 + (lane >> 4)), b0, b1, b2, b3);
-                        mma_bf16(o[2 * dp], pa[kk], b0, b1);
-                        mma_bf16(o[2 * dp + 1], pa[kk], b2, b3);
+                        mma_f16(o[2 * dp], pa[kk], b0, b1);
+                        mma_f16(o[2 * dp + 1], pa[kk], b2, b3);
                     }
                 }
             }

@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -75,6 +76,28 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
     uint16_t d;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
     return d;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+// 2^x of a pair in FP16 on the special-function unit, one instruction for both (the arguments
+// are rounded to FP16 first; 2^-inf = 0).  The attention probabilities P go to the tensor cores
+// in FP16 (10 mantissa bits, against BF16's 7), multiplied by FP16 values V.
+__device__ __forceinline__ uint32_t ex2_f16x2(float x0, float x1) {
+    uint32_t r;
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(pack_f16x2(x0, x1)));
+    return r;
+}
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+    __half2 r = __hadd2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+// The sum of both halves of an FP16 pair, in FP32.
+__device__ __forceinline__ float hsum2_f32(uint32_t a) {
+    const float2 f = __half22float2(*reinterpret_cast<__half2 *>(&a));
+    return f.x + f.y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -285,6 +308,11 @@ __device__ __forceinline__ void tc_mma_e4m3(uint32_t d_tmem, uint64_t adesc, uin
 
 // Instruction descriptor for kind::f8f6f4: E4M3 A and B (format code 0), f32 D, K-major A and B, M = 128.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// Instruction descriptor for kind::f16 with FP16 A and B (format code 0), f32 D, K-major A and B, M = 128.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int n) {
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 

@@ -301,6 +301,7 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
             tmem_ld_wait();
             const int n = n0 + h;
             const bool rot = have_cs && n < ep.rope_cols;
+            const bool vcol = ep.out_col0 + n >= 2 * D;  // v: FP16 (the attention's P V products are FP16)
             float ba[32], bb[32];
 #pragma unroll
             for (int j4 = 0; j4 < 8; ++j4) {
@@ -312,19 +313,14 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
                 ba[4 * j4] = x.x; ba[4 * j4 + 1] = x.y; ba[4 * j4 + 2] = x.z; ba[4 * j4 + 3] = x.w;
                 bb[4 * j4] = y.x; bb[4 * j4 + 1] = y.y; bb[4 * j4 + 2] = y.z; bb[4 * j4 + 3] = y.w;
             }
-            if constexpr (F8) {  // E4M3 product: undo the activation and weight-row scales
+            float sa[32], sb[32];  // FP8: per-column scales of the E4M3 product (activation x weight row)
+            if constexpr (F8) {
 #pragma unroll
                 for (int j4 = 0; j4 < 8; ++j4) {
                     const float4 x = reinterpret_cast<const float4 *>(ep.col_scale + n)[j4];
                     const float4 y = reinterpret_cast<const float4 *>(ep.col_scale + n + 32)[j4];
-                    a[4 * j4] = __float_as_uint(__uint_as_float(a[4 * j4]) * x.x);
-                    a[4 * j4 + 1] = __float_as_uint(__uint_as_float(a[4 * j4 + 1]) * x.y);
-                    a[4 * j4 + 2] = __float_as_uint(__uint_as_float(a[4 * j4 + 2]) * x.z);
-                    a[4 * j4 + 3] = __float_as_uint(__uint_as_float(a[4 * j4 + 3]) * x.w);
-                    b[4 * j4] = __float_as_uint(__uint_as_float(b[4 * j4]) * y.x);
-                    b[4 * j4 + 1] = __float_as_uint(__uint_as_float(b[4 * j4 + 1]) * y.y);
-                    b[4 * j4 + 2] = __float_as_uint(__uint_as_float(b[4 * j4 + 2]) * y.z);
-                    b[4 * j4 + 3] = __float_as_uint(__uint_as_float(b[4 * j4 + 3]) * y.w);
+                    sa[4 * j4] = x.x; sa[4 * j4 + 1] = x.y; sa[4 * j4 + 2] = x.z; sa[4 * j4 + 3] = x.w;
+                    sb[4 * j4] = y.x; sb[4 * j4 + 1] = y.y; sb[4 * j4 + 2] = y.z; sb[4 * j4 + 3] = y.w;
                 }
             }
 #pragma unroll
@@ -333,8 +329,8 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
                     const int jj = j + t;
-                    const float x1 = __uint_as_float(a[jj]) + ba[jj];
-                    const float x2 = __uint_as_float(b[jj]) + bb[jj];
+                    const float x1 = F8 ? fmaf(__uint_as_float(a[jj]), sa[jj], ba[jj]) : __uint_as_float(a[jj]) + ba[jj];
+                    const float x2 = F8 ? fmaf(__uint_as_float(b[jj]), sb[jj], bb[jj]) : __uint_as_float(b[jj]) + bb[jj];
                     if (rot) {
                         r2[t] = x1 * cs[jj].x - x2 * cs[jj].y;
                         s2[t] = x2 * cs[jj].x + x1 * cs[jj].y;
@@ -343,8 +339,8 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
                         s2[t] = x2;
                     }
                 }
-                w1[j >> 1] = pack_bf16x2(r2[0], r2[1]);
-                w2[j >> 1] = pack_bf16x2(s2[0], s2[1]);
+                w1[j >> 1] = vcol ? pack_f16x2(r2[0], r2[1]) : pack_bf16x2(r2[0], r2[1]);
+                w2[j >> 1] = vcol ? pack_f16x2(s2[0], s2[1]) : pack_bf16x2(s2[0], s2[1]);
             }
             stage_row32(box, r, 0, w1);
             stage_row32(box, r, 4, w2);
@@ -537,8 +533,11 @@ struct RlCfg {
 #endif
 constexpr int RL_STAGES = JD_RL_STAGES, RL_NXB = JD_RL_NXB;
 using RlCur = RlCfg<RL_STAGES, RL_NXB>;
-#ifndef JD_RL_SPLIT_PERSISTENT
-#define JD_RL_SPLIT_PERSISTENT 0
+// The persistent split kernel measured faster than k_gemm_rl for K = 1152 (Wo2: 20.7 against
+// 21.6 ms per step at 1024 rows) and slower for K = 384 (Wo: 17.5 against 14.7 ms): with a short
+// K the extra A reads of the second CTA outweigh the overlap.
+#ifndef JD_RL_SPLIT_MIN_K
+#define JD_RL_SPLIT_MIN_K 768
 #endif
 constexpr int RS_NS = 3;  // CTAs per row tile of the split residual GEMM (128 columns each)
 constexpr int RP_NS = 2;  // CTAs per row tile of the persistent split residual GEMM (192 columns each)
@@ -1555,8 +1554,9 @@ cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st) {
                                                                                            op.K, op.ep);
             return cudaGetLastError();
         }
-#if JD_RL_SPLIT_PERSISTENT
-        if (op.tmA && op.tmBp && op.K % 64 == 0) {  // many row tiles: persistent, columns split over 2 CTAs
+        if (op.tmA && op.tmBp && op.K % 64 == 0 && op.K >= JD_RL_SPLIT_MIN_K) {
+            // many row tiles and a long K (Wo2, the head's second feed-forward GEMM): persistent,
+            // the columns split over 2 CTAs so that one tile's epilogue overlaps the next one's MMAs
             if (op.out8 && (op.ep.ln_b || op.ep.out8_inv_scale <= 0.f)) return cudaErrorInvalidValue;
             const int ncl = std::min(n_tiles, g_num_sms / RP_NS);
             if (op.out8)
@@ -1567,7 +1567,6 @@ cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st) {
                                                                                         n_tiles, op.ep);
             return cudaGetLastError();
         }
-#endif
         if (op.out8) {
             if (op.ep.ln_b || op.ep.out8_inv_scale <= 0.f) return cudaErrorInvalidValue;
             k_gemm_rl<RL_STAGES, RL_NXB, true><<<grid, 192, RlCur::SMEM, st>>>(*op.tmA64, *op.tmB64, *op.tmX,

@@ -39,10 +39,13 @@ cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st);
 // Per-token row index / position and per-row attention work-unit offsets
 // (qb_off holds 2 * (n_rows + 1) ints: 64-query then 256-query block offsets,
 // followed by the row of every 256-query block (n_tokens / 256 + n_rows ints)
-// and the row of every 64-query block (n_tokens / 64 + n_rows ints), in all
-// qb_ints(n_rows, n_tokens) ints).
-inline int qb_row64_offset(int n_rows, int n_tokens) { return 2 * (n_rows + 1) + n_tokens / 256 + n_rows; }
-inline size_t qb_ints(int n_rows, int n_tokens) { return (size_t)qb_row64_offset(n_rows, n_tokens) + n_tokens / 64 + n_rows; }
+// and, for every 64-query block, its row's first and end token and its first
+// query (3 ints each, (n_tokens + 63) / 64 + n_rows blocks: as many as the
+// sliding-window attention's grid), in all qb_ints(n_rows, n_tokens) ints).
+constexpr int qb_span_offset(int n_rows, int n_tokens) { return 2 * (n_rows + 1) + n_tokens / 256 + n_rows; }
+constexpr size_t qb_ints(int n_rows, int n_tokens) {
+    return (size_t)qb_span_offset(n_rows, n_tokens) + 3 * ((size_t)(n_tokens + 63) / 64 + n_rows);
+}
 cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
                         cudaStream_t st);
 

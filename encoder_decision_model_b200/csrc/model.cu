@@ -1075,8 +1075,7 @@ constexpr size_t NA_Y = NA_O + na_up((size_t)NA_TOKENS * D * 2);
 constexpr size_t NA_TOKROW = NA_Y + na_up((size_t)NA_TOKENS * HFF * 2);
 constexpr size_t NA_POS = NA_TOKROW + na_up((size_t)NA_TOKENS * 4);
 constexpr size_t NA_QBOFF = NA_POS + na_up((size_t)NA_TOKENS * 4);
-constexpr size_t NA_HM =
-    NA_QBOFF + na_up((size_t)(2 * (NA_ROWS + 1) + NA_TOKENS / 256 + NA_ROWS + NA_TOKENS / 64 + NA_ROWS) * 4);
+constexpr size_t NA_HM = NA_QBOFF + na_up(qb_ints(NA_ROWS, NA_TOKENS) * 4);
 constexpr size_t NA_XM = NA_HM + na_up((size_t)NA_MARKERS * D * 4);
 constexpr size_t NA_QM = NA_XM + na_up((size_t)NA_MARKERS * D * 2);
 constexpr size_t NA_OM = NA_QM + na_up((size_t)NA_MARKERS * D * 2);

@@ -58,10 +58,23 @@ __global__ void __launch_bounds__(1024) k_qblock_offsets(const int *__restrict__
     }
 }
 
-// row of every block: blk_row[off[r] .. off[r + 1]) = r (off: the 64- or 256-query block offsets)
+// row of every 256-query block: blk_row[off[r] .. off[r + 1]) = r
 __global__ void k_qblock_rows(const int *__restrict__ off, int n_rows, int *__restrict__ blk_row) {
     for (int r = blockIdx.x * blockDim.y + threadIdx.y; r < n_rows; r += gridDim.x * blockDim.y)
         for (int pb = off[r] + threadIdx.x; pb < off[r + 1]; pb += blockDim.x) blk_row[pb] = r;
+}
+
+// every 64-query block b of row r: span[3 b .. 3 b + 2] = (row start, row end, first query)
+__global__ void k_qblock_spans(const int *__restrict__ off, const int *__restrict__ cu, int n_rows,
+                               int *__restrict__ span) {
+    for (int r = blockIdx.x * blockDim.y + threadIdx.y; r < n_rows; r += gridDim.x * blockDim.y) {
+        const int cs = cu[r], ce = cu[r + 1], b0 = off[r];
+        for (int pb = b0 + threadIdx.x; pb < off[r + 1]; pb += blockDim.x) {
+            span[3 * pb] = cs;
+            span[3 * pb + 1] = ce;
+            span[3 * pb + 2] = cs + (pb - b0) * 64;
+        }
+    }
 }
 
 cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
@@ -71,8 +84,8 @@ cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *to
     k_qblock_offsets<<<1, 1024, 0, st>>>(cu_seqlens, n_rows, qb_off);
     k_qblock_rows<<<min((n_rows + 7) / 8, 1024), dim3(32, 8), 0, st>>>(qb_off + n_rows + 1, n_rows,
                                                                        qb_off + 2 * (n_rows + 1));
-    k_qblock_rows<<<min((n_rows + 7) / 8, 1024), dim3(32, 8), 0, st>>>(qb_off, n_rows,
-                                                                       qb_off + qb_row64_offset(n_rows, n_tokens));
+    k_qblock_spans<<<min((n_rows + 7) / 8, 1024), dim3(32, 8), 0, st>>>(qb_off, cu_seqlens, n_rows,
+                                                                        qb_off + qb_span_offset(n_rows, n_tokens));
     return cudaGetLastError();
 }
 
