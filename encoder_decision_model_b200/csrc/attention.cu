@@ -375,21 +375,21 @@ __global__ void __launch_bounds__(128 * LOC_HEADS, 2)
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
     const float mu0 = mx0 == -INFINITY ? 0.f : -mx0 * sl2, mu1 = mx1 == -INFINITY ? 0.f : -mx1 * sl2;
-    // P in FP16 pairs straight from the special-function unit (one ex2 for two keys), the row
-    // sums as FP16 pair sums (three interleaved per row, at most six adds each, values <= 1)
-    uint32_t hp0[3] = {0u, 0u, 0u}, hp1[3] = {0u, 0u, 0u};
+    // P = 2^x in FP32 (one ex2.approx.ftz per key), FP32 row sums, P packed to FP16 pairs for the
+    // P V products (V is FP16).  An FP16 ex2 for two keys measured slower: its conversions cost
+    // more instructions than it saved on the special-function unit.
+    float lp0[2] = {0.f, 0.f}, lp1[2] = {0.f, 0.f};  // two interleaved partial sums per row
     uint32_t pa[LW_CHUNKS][4];
 #pragma unroll
     for (int j = 0; j < 2 * LW_CHUNKS; ++j) {
-        const uint32_t h01 = ex2_f16x2(fmaf(sc[j][0], sl2, mu0), fmaf(sc[j][1], sl2, mu0));
-        const uint32_t h23 = ex2_f16x2(fmaf(sc[j][2], sl2, mu1), fmaf(sc[j][3], sl2, mu1));
-        hp0[j % 3] = hadd2_u32(hp0[j % 3], h01);
-        hp1[j % 3] = hadd2_u32(hp1[j % 3], h23);
-        pa[j >> 1][(j & 1) * 2 + 0] = h01;
-        pa[j >> 1][(j & 1) * 2 + 1] = h23;
+        const float p0 = ex2_ftz(fmaf(sc[j][0], sl2, mu0)), p1 = ex2_ftz(fmaf(sc[j][1], sl2, mu0));
+        const float p2 = ex2_ftz(fmaf(sc[j][2], sl2, mu1)), p3 = ex2_ftz(fmaf(sc[j][3], sl2, mu1));
+        lp0[j & 1] += p0 + p1;
+        lp1[j & 1] += p2 + p3;
+        pa[j >> 1][(j & 1) * 2 + 0] = pack_f16x2(p0, p1);
+        pa[j >> 1][(j & 1) * 2 + 1] = pack_f16x2(p2, p3);
     }
-    float l0 = hsum2_f32(hp0[0]) + hsum2_f32(hp0[1]) + hsum2_f32(hp0[2]);
-    float l1 = hsum2_f32(hp1[0]) + hsum2_f32(hp1[1]) + hsum2_f32(hp1[2]);
+    float l0 = lp0[0] + lp0[1], l1 = lp1[0] + lp1[1];
     float o[8][4];
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;

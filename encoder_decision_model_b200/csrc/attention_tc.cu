@@ -379,28 +379,27 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                         named_bar_sync(BAR_G0_DONE, 256);
                     }
                 }
-                float ls = 0.f;
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int hk = 0; hk < 2; ++hk) {  // 64 keys at a time; the first half's store overlaps the second
-                    // P in FP16 pairs (one ex2 for two keys); row sums as FP16 pair sums, eight pairs
-                    // each (P <= 2^8), added to the FP32 sum every 64 keys
-                    uint32_t pk[32], hs[4] = {0u, 0u, 0u, 0u};
+                    // P = 2^x in FP32, FP32 row sums, P packed to FP16 pairs (V is FP16).  An FP16 ex2
+                    // for two keys measured slower: the special-function unit stayed as busy and the
+                    // conversions added instructions.
+                    uint32_t pk[32];
 #pragma unroll
                     for (int e = 0; e < 64; e += 2) {
                         const float2 xv = fma2(make_float2(__uint_as_float(sv[64 * hk + e]), __uint_as_float(sv[64 * hk + e + 1])),
                                                make_float2(sl2, sl2), make_float2(-m, -m));
-                        uint32_t hp;
+                        float p0, p1;
                         if (((e >> 1) & 7) < JD_EX2_POLY_OF8) {
-                            float p0, p1;
                             ex2_poly2(xv.x, xv.y, p0, p1);
-                            hp = pack_f16x2(p0, p1);
                         } else {
-                            hp = ex2_f16x2(xv.x, xv.y);
+                            p0 = ex2_approx(xv.x);
+                            p1 = ex2_approx(xv.y);
                         }
-                        hs[(e >> 1) & 3] = hadd2_u32(hs[(e >> 1) & 3], hp);
-                        pk[e >> 1] = hp;
+                        ls[(e >> 1) & 3] += p0 + p1;
+                        pk[e >> 1] = pack_f16x2(p0, p1);
                     }
-                    ls += (hsum2_f32(hs[0]) + hsum2_f32(hs[1])) + (hsum2_f32(hs[2]) + hsum2_f32(hs[3]));
                     if (hk == 0) {
                         if (j != 0) mbar_wait(&pvdone[x], (c - 1) & 1, status);  // P_x consumed by the last product
                         __syncwarp();
@@ -412,7 +411,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     if (x == 0) named_bar_arrive(BAR_G0_DONE, 256);
                     else if (j != t.nt - 1) named_bar_arrive(BAR_G1_DONE, 256);
                 }
-                l += ls;
+                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();

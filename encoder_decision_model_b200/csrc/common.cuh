@@ -78,28 +78,11 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
     return d;
 }
 
+// Two floats to an FP16 pair (the attention probabilities P, multiplied by FP16 values V).
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
 }
-// 2^x of a pair in FP16 on the special-function unit, one instruction for both (the arguments
-// are rounded to FP16 first; 2^-inf = 0).  The attention probabilities P go to the tensor cores
-// in FP16 (10 mantissa bits, against BF16's 7), multiplied by FP16 values V.
-__device__ __forceinline__ uint32_t ex2_f16x2(float x0, float x1) {
-    uint32_t r;
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(pack_f16x2(x0, x1)));
-    return r;
-}
-__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
-    __half2 r = __hadd2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
-    return *reinterpret_cast<uint32_t *>(&r);
-}
-// The sum of both halves of an FP16 pair, in FP32.
-__device__ __forceinline__ float hsum2_f32(uint32_t a) {
-    const float2 f = __half22float2(*reinterpret_cast<__half2 *>(&a));
-    return f.x + f.y;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);

@@ -539,7 +539,8 @@ using RlCur = RlCfg<RL_STAGES, RL_NXB>;
 #ifndef JD_RL_SPLIT_MIN_K
 #define JD_RL_SPLIT_MIN_K 768
 #endif
-constexpr int RS_NS = 3;  // CTAs per row tile of the split residual GEMM (128 columns each)
+// CTAs per row tile of the split residual GEMM: six (64 columns each) when the grid fits the SMs,
+// else three (128 columns each)
 constexpr int RP_NS = 2;  // CTAs per row tile of the persistent split residual GEMM (192 columns each)
 
 // OUT8: the LayerNorm output goes out as E4M3 bytes, y * ep.out8_inv_scale, rows of 384 bytes
@@ -815,7 +816,8 @@ __global__ void __launch_bounds__(192, 1)
 // distributed shared memory; after a cluster barrier each CTA merges the NS
 // partial moments in rank order (equal counts: the mean of the means, M2 plus
 // the spread of the means) and writes the LayerNorm output of its columns.
-//   warp 0 lane 0  TMA producer: A box 128 x 64 and W box NC x 64 (128-byte swizzle) per stage
+//   warp 0 lane 0  TMA producer: A box 128 x 64 and NC / 64 W boxes of 64 x 64 (128-byte swizzle)
+//                  per stage
 //   warp 1         TMEM allocation; lane 0 issues the N = NC MMAs
 //   warps 2..5     epilogue, one row per thread; the NC / 32 residual chunks (FP32,
 //                  128 x 32) are loaded by TMA at the start, under the mainloop
@@ -825,16 +827,17 @@ struct RsCfg {
     static constexpr int A_BYTES = 128 * 128;    // 128 rows x 64 bf16
     static constexpr int B_BYTES = NC * 128;     // NC rows x 64 bf16
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int STAGES = NS == 2 ? 3 : 4;
+    static constexpr int STAGES = NS >= 6 ? 6 : 4;
     static constexpr int RING = STAGES * STAGE;
+    static constexpr int NWL = NC / 64;          // W boxes of 64 rows per stage
     static constexpr int XCH = 128 * 32 * 4;     // residual chunk: 128 rows x 32 FP32
     static constexpr int NX = NC / 32;
     static constexpr int MOM = 12 * 128 * 8;     // (mean, M2) of every row's twelve 32-column chunks
     static constexpr int DATA = RING + NX * XCH + MOM;
     static constexpr int BAR_BYTES = (2 * STAGES + 1 + NX) * 8 + 8;
     static constexpr int SMEM = DATA + BAR_BYTES + 1024;
-    static constexpr uint32_t TMEM_COLS = NC <= 128 ? 128 : 256;
-    static_assert(NC % 32 == 0 && NC % 16 == 0 && NC <= 256, "column share");
+    static constexpr uint32_t TMEM_COLS = NC <= 64 ? 64 : (NC <= 128 ? 128 : 256);
+    static_assert(NC % 64 == 0 && NC <= 256, "column share: whole 64-row W boxes");
     static_assert(SMEM <= 227 * 1024, "split residual GEMM shared memory");
 };
 
@@ -899,7 +902,9 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
                 uint8_t *sa = smem + s * C::STAGE;
                 mbar_arrive_expect_tx(&full[s], C::STAGE);
                 tma_load_2d(sa, &tmA, &full[s], kb * 64, m0);
-                tma_load_2d(sa + C::A_BYTES, &tmB, &full[s], kb * 64, c0);
+#pragma unroll
+                for (int w = 0; w < C::NWL; ++w)
+                    tma_load_2d(sa + C::A_BYTES + w * 64 * 128, &tmB, &full[s], kb * 64, c0 + 64 * w);
             }
         }
     } else if (warp == 1) {
@@ -1483,11 +1488,17 @@ cudaError_t gemm_init_attributes() {
     if ((e = cudaFuncSetAttribute(k_gemm_rlp<RP_NS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   RpCfg<RP_NS>::SMEM)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(k_gemm_rls<RS_NS, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  RsCfg<RS_NS>::SMEM)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(k_gemm_rls<3, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  RsCfg<3>::SMEM)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(k_gemm_rls<RS_NS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  RsCfg<RS_NS>::SMEM)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(k_gemm_rls<3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  RsCfg<3>::SMEM)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_gemm_rls<6, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  RsCfg<6>::SMEM)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_gemm_rls<6, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  RsCfg<6>::SMEM)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 192, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<192>::SMEM)) != cudaSuccess)
@@ -1543,15 +1554,20 @@ cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st) {
         op.N == D && op.K % 32 == 0) {
         const int n_tiles = (op.ep.rows + 127) / 128;
         const int grid = n_tiles < g_num_sms ? n_tiles : g_num_sms;
-        if (op.tmA && op.tmBs && op.K % 64 == 0 && RS_NS * n_tiles <= g_num_sms) {
-            // few row tiles: split each tile's columns over a cluster, so RS_NS SMs share it
+        if (op.tmA && op.tmBs && op.K % 64 == 0 && 3 * n_tiles <= g_num_sms) {
+            // few row tiles: split each tile's columns over a cluster, so six or three SMs share it
             if (op.out8 && (op.ep.ln_b || op.ep.out8_inv_scale <= 0.f)) return cudaErrorInvalidValue;
-            if (op.out8)
-                k_gemm_rls<RS_NS, true><<<RS_NS * n_tiles, 192, RsCfg<RS_NS>::SMEM, st>>>(*op.tmA, *op.tmBs, *op.tmX,
-                                                                                          op.K, op.ep);
-            else
-                k_gemm_rls<RS_NS, false><<<RS_NS * n_tiles, 192, RsCfg<RS_NS>::SMEM, st>>>(*op.tmA, *op.tmBs, *op.tmX,
-                                                                                           op.K, op.ep);
+            if (6 * n_tiles <= g_num_sms) {
+                if (op.out8)
+                    k_gemm_rls<6, true><<<6 * n_tiles, 192, RsCfg<6>::SMEM, st>>>(*op.tmA, *op.tmBs, *op.tmX, op.K, op.ep);
+                else
+                    k_gemm_rls<6, false><<<6 * n_tiles, 192, RsCfg<6>::SMEM, st>>>(*op.tmA, *op.tmBs, *op.tmX, op.K, op.ep);
+            } else {
+                if (op.out8)
+                    k_gemm_rls<3, true><<<3 * n_tiles, 192, RsCfg<3>::SMEM, st>>>(*op.tmA, *op.tmBs, *op.tmX, op.K, op.ep);
+                else
+                    k_gemm_rls<3, false><<<3 * n_tiles, 192, RsCfg<3>::SMEM, st>>>(*op.tmA, *op.tmBs, *op.tmX, op.K, op.ep);
+            }
             return cudaGetLastError();
         }
         if (op.tmA && op.tmBp && op.K % 64 == 0 && op.K >= JD_RL_SPLIT_MIN_K) {

@@ -25,7 +25,7 @@ struct GemmOp {
     const CUtensorMap *tmXN;  // BF16 residual epilogue: LayerNorm output, box 64 x 128, 128-byte swizzle
     const CUtensorMap *tmA64; // BF16 residual GEMM: A box 32 x 128, 64-byte swizzle
     const CUtensorMap *tmB64; // BF16 residual GEMM: W box 32 x 192, 64-byte swizzle
-    const CUtensorMap *tmBs;  // BF16 residual GEMM split over a cluster: W box 64 x 128, 128-byte swizzle
+    const CUtensorMap *tmBs;  // BF16 residual GEMM split over a cluster: W box 64 x 64, 128-byte swizzle
     const CUtensorMap *tmBp;  // BF16 persistent split residual GEMM: W box 64 x 192, 128-byte swizzle
     const float *A32;         // FP32 path: A [rows, lda]
     int lda;

@@ -157,7 +157,7 @@ struct ProjW {            // one projection weight [N, K]
     void *w = nullptr;    // bf16 or f32 on device
     CUtensorMap tm{};     // BF16 mode only
     CUtensorMap tm64{};   // BF16 mode, 384-wide tiles: box 32 x 192, 64-byte swizzle (residual GEMM)
-    CUtensorMap tm128{};  // BF16 mode, 384-wide tiles: box 64 x 128 (residual GEMM split over a cluster)
+    CUtensorMap tms{};    // BF16 mode, 384-wide tiles: box 64 x 64 (residual GEMM split over a cluster)
     int N = 0, K = 0;
     // FP8 mode, encoder QKV: E4M3 codes of W[n, :] / s_n (s_n = max_k |W[n, k]| / 448), box 128 x 192,
     // and per output column the product of the input's activation scale and s_n
@@ -294,7 +294,7 @@ jd_status upload_proj(jd_model *m, const std::vector<float> &h, int r0, int N, i
         TRY(make_map(&p.tm, d, K, N, K, 64, box_rows));
         if (bn == 384) {
             TRY(make_map(&p.tm64, d, K, N, K, 32, 192, false, true));
-            TRY(make_map(&p.tm128, d, K, N, K, 64, 128));
+            TRY(make_map(&p.tms, d, K, N, K, 64, 64));
         }
     }
     return JD_OK;
@@ -537,7 +537,7 @@ GemmOp make_op(int epi, int bn, const ProjW &w, const CUtensorMap *tmA, const vo
     op.tmXN = tmXN;
     op.tmA64 = tmA64;
     op.tmB64 = tmA64 ? &w.tm64 : nullptr;
-    op.tmBs = tmA64 ? &w.tm128 : nullptr;
+    op.tmBs = tmA64 ? &w.tms : nullptr;
     op.tmBp = tmA64 ? &w.tm : nullptr;  // box 64 x 192 of the 384-wide weights
     op.epi = epi;
     op.bn = bn;

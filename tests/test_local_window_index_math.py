@@ -63,3 +63,22 @@ def test_warp_keys_cover_each_query_window_and_stay_in_the_band():
             qi = q0 + 16 * warp + r
             need = set(range(qi - WINDOW, qi + WINDOW + 1))
             assert need <= keys, (warp, r)
+
+
+def test_interior_warps_skip_row_tests_only_when_every_key_is_in_the_row():
+    """The kernel takes the copy of the mask loop without per-key row tests when the warp's
+    first key kw and its last key kw + 16 * LW_CHUNKS - 1 lie in [cs, ce); brute force over
+    rows of every length up to 400 and every warp position: then every key the warp reads
+    is in the row, and a warp that fails the test does read a key outside it."""
+    src = open(SRC).read()
+    assert "if (kw >= cs && kw + 16 * LW_CHUNKS <= ce) {" in src
+    chunks, _, _ = _kernel_constants()
+    cs = 1000
+    for L in range(1, 400):
+        ce = cs + L
+        for q0 in range(cs, ce, BQ):
+            for warp in range(4):
+                kw = q0 - WINDOW + 16 * warp
+                keys = range(kw, kw + 16 * chunks)
+                interior = kw >= cs and kw + 16 * chunks <= ce
+                assert interior == all(cs <= k < ce for k in keys), (L, q0, warp)
