@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                         named_bar_sync(BAR_G0_DONE, 256);
                     }
                 }
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                float2 ls[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};  // pair sums: one add.f32x2 per pair
 #pragma unroll
                 for (int hk = 0; hk < 2; ++hk) {  // 64 keys at a time; the first half's store overlaps the second
                     // P = 2^x in FP32, FP32 row sums, P packed to FP16 pairs (V is FP16).  An FP16 ex2
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                             p0 = ex2_approx(xv.x);
                             p1 = ex2_approx(xv.y);
                         }
-                        ls[(e >> 1) & 3] += p0 + p1;
+                        ls[(e >> 1) & 3] = add2(ls[(e >> 1) & 3], make_float2(p0, p1));
                         pk[e >> 1] = pack_f16x2(p0, p1);
                     }
                     if (hk == 0) {
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     if (x == 0) named_bar_arrive(BAR_G0_DONE, 256);
                     else if (j != t.nt - 1) named_bar_arrive(BAR_G1_DONE, 256);
                 }
-                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                l += ((ls[0].x + ls[0].y) + (ls[1].x + ls[1].y)) + ((ls[2].x + ls[2].y) + (ls[3].x + ls[3].y));
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();

@@ -1506,6 +1506,9 @@ cudaError_t gemm_init_attributes() {
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 192, 4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<192>::SMEM)) != cudaSuccess)
         return e;
+    if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 64, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  PcCfg<64>::SMEM)) != cudaSuccess)
+        return e;
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_GEGLU, 256, GEGLU_EW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<256>::SMEM)) != cudaSuccess)
         return e;
@@ -1595,7 +1598,17 @@ cudaError_t launch_gemm(const GemmOp &op, bool fp32, cudaStream_t st) {
     }
     if (op.out8 || (op.f8 && (fp32 || op.epi != EPI_QKV))) return cudaErrorInvalidValue;
     if (!fp32) {  // persistent tcgen05 kernels for the column-split epilogues
-        if (op.epi == EPI_QKV) return op.f8 ? launch_pc<EPI_QKV, 192, true>(op, st) : launch_pc<EPI_QKV, 192>(op, st);
+        if (op.epi == EPI_QKV) {
+            if (op.f8) return launch_pc<EPI_QKV, 192, true>(op, st);
+            // few row tiles: one 64-column head per tile, so up to three times as many SMs share the product
+            const int row_tiles = (op.ep.rows + 127) / 128;
+            if (op.tmBs && op.N % 64 == 0 && row_tiles * (op.N / 64) <= g_num_sms) {
+                GemmOp o = op;
+                o.tmB = op.tmBs;
+                return launch_pc<EPI_QKV, 64>(o, st);
+            }
+            return launch_pc<EPI_QKV, 192>(op, st);
+        }
         if (op.epi == EPI_GEGLU) return launch_pc<EPI_GEGLU, 256>(op, st);
         if (op.epi == EPI_BIAS_ACT) return launch_pc<EPI_BIAS_ACT, 256>(op, st);
     }

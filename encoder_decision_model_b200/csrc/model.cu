@@ -157,7 +157,8 @@ struct ProjW {            // one projection weight [N, K]
     void *w = nullptr;    // bf16 or f32 on device
     CUtensorMap tm{};     // BF16 mode only
     CUtensorMap tm64{};   // BF16 mode, 384-wide tiles: box 32 x 192, 64-byte swizzle (residual GEMM)
-    CUtensorMap tms{};    // BF16 mode, 384-wide tiles: box 64 x 64 (residual GEMM split over a cluster)
+    CUtensorMap tms{};    // BF16 mode, 384-wide tiles: box 64 x 64 (split residual GEMM, one-head QKV tiles)
+    bool has_tms = false;
     int N = 0, K = 0;
     // FP8 mode, encoder QKV: E4M3 codes of W[n, :] / s_n (s_n = max_k |W[n, k]| / 448), box 128 x 192,
     // and per output column the product of the input's activation scale and s_n
@@ -295,6 +296,7 @@ jd_status upload_proj(jd_model *m, const std::vector<float> &h, int r0, int N, i
         if (bn == 384) {
             TRY(make_map(&p.tm64, d, K, N, K, 32, 192, false, true));
             TRY(make_map(&p.tms, d, K, N, K, 64, 64));
+            p.has_tms = true;
         }
     }
     return JD_OK;
@@ -537,7 +539,7 @@ GemmOp make_op(int epi, int bn, const ProjW &w, const CUtensorMap *tmA, const vo
     op.tmXN = tmXN;
     op.tmA64 = tmA64;
     op.tmB64 = tmA64 ? &w.tm64 : nullptr;
-    op.tmBs = tmA64 ? &w.tms : nullptr;
+    op.tmBs = w.N % 64 == 0 && w.has_tms ? &w.tms : nullptr;  // W box 64 x 64 (split residual, small-batch QKV)
     op.tmBp = tmA64 ? &w.tm : nullptr;  // box 64 x 192 of the 384-wide weights
     op.epi = epi;
     op.bn = bn;
@@ -582,7 +584,7 @@ jd_status enqueue_forward(jd_model *m, const jd_batch *b, const jd_outputs *out,
     m->n_ev = 0;
     const int T = b->n_tokens, B = b->n_rows, M = b->n_markers;
     LK(cudaMemsetAsync(m->status, 0, sizeof(unsigned), st));
-    KL("prep", 3, launch_prep(b->cu_seqlens, B, T, m->tok_row, m->pos, m->qb_off, st));
+    KL("prep", 2, launch_prep(b->cu_seqlens, B, T, m->tok_row, m->pos, m->qb_off, st));
     const bool f8 = m->fp8;
     KL("embed_ln", 1, launch_embed_ln(b->tokens, T, m->E, VOCAB, m->emb_g, EPS, m->x, f8 ? (void *)m->xn8 : m->xn, f32,
                                       m->status, st, f8 ? m->inv8[0] : 0.f));

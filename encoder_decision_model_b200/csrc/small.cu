@@ -18,10 +18,13 @@ __global__ void k_token_meta(const int *__restrict__ cu, int n_rows, int *__rest
     }
 }
 
-// Attention work-unit offsets, one CTA of 1024 threads:
-//   qb_off[r]             = sum over rows < r of ceil(len / 64)   (64-query blocks)
+// Attention work units, one CTA of 1024 threads:
+//   qb_off[r]              = sum over rows < r of ceil(len / 64)   (64-query blocks)
 //   qb_off[n_rows + 1 + r] = sum over rows < r of ceil(len / 256)  (256-query blocks)
-__global__ void __launch_bounds__(1024) k_qblock_offsets(const int *__restrict__ cu, int n_rows, int *__restrict__ qb_off) {
+// then, by the thread that owns row r, the row of each of its 256-query blocks (pb_row) and
+// each of its 64-query blocks' row start, row end and first query (span[3 b .. 3 b + 2]).
+__global__ void __launch_bounds__(1024) k_qblock_meta(const int *__restrict__ cu, int n_rows, int *__restrict__ qb_off,
+                                                      int *__restrict__ pb_row, int *__restrict__ span) {
     __shared__ int part[2][1024];
     const int tid = threadIdx.x;
     const int per = (n_rows + 1023) / 1024;
@@ -46,11 +49,19 @@ __global__ void __launch_bounds__(1024) k_qblock_offsets(const int *__restrict__
     int run64 = tid ? part[0][tid - 1] : 0, run256 = tid ? part[1][tid - 1] : 0;
     int *q256 = qb_off + n_rows + 1;
     for (int r = r0; r < r1; ++r) {
-        const int len = cu[r + 1] - cu[r];
+        const int cs = cu[r], ce = cu[r + 1], len = ce - cs;
+        const int n64 = (len + 63) / 64, n256 = (len + 255) / 256;
         qb_off[r] = run64;
         q256[r] = run256;
-        run64 += (len + 63) / 64;
-        run256 += (len + 255) / 256;
+        for (int b = 0; b < n256; ++b) pb_row[run256 + b] = r;
+        for (int b = 0; b < n64; ++b) {
+            int *sp = span + 3 * (run64 + b);
+            sp[0] = cs;
+            sp[1] = ce;
+            sp[2] = cs + b * 64;
+        }
+        run64 += n64;
+        run256 += n256;
     }
     if (tid == 1023) {
         qb_off[n_rows] = part[0][1023];
@@ -58,34 +69,12 @@ __global__ void __launch_bounds__(1024) k_qblock_offsets(const int *__restrict__
     }
 }
 
-// row of every 256-query block: blk_row[off[r] .. off[r + 1]) = r
-__global__ void k_qblock_rows(const int *__restrict__ off, int n_rows, int *__restrict__ blk_row) {
-    for (int r = blockIdx.x * blockDim.y + threadIdx.y; r < n_rows; r += gridDim.x * blockDim.y)
-        for (int pb = off[r] + threadIdx.x; pb < off[r + 1]; pb += blockDim.x) blk_row[pb] = r;
-}
-
-// every 64-query block b of row r: span[3 b .. 3 b + 2] = (row start, row end, first query)
-__global__ void k_qblock_spans(const int *__restrict__ off, const int *__restrict__ cu, int n_rows,
-                               int *__restrict__ span) {
-    for (int r = blockIdx.x * blockDim.y + threadIdx.y; r < n_rows; r += gridDim.x * blockDim.y) {
-        const int cs = cu[r], ce = cu[r + 1], b0 = off[r];
-        for (int pb = b0 + threadIdx.x; pb < off[r + 1]; pb += blockDim.x) {
-            span[3 * pb] = cs;
-            span[3 * pb + 1] = ce;
-            span[3 * pb + 2] = cs + (pb - b0) * 64;
-        }
-    }
-}
-
 cudaError_t launch_prep(const int *cu_seqlens, int n_rows, int n_tokens, int *tok_row, int *pos, int *qb_off,
                         cudaStream_t st) {
     if (n_rows <= 0) return cudaSuccess;
     k_token_meta<<<min(n_rows, 4096), 256, 0, st>>>(cu_seqlens, n_rows, tok_row, pos);
-    k_qblock_offsets<<<1, 1024, 0, st>>>(cu_seqlens, n_rows, qb_off);
-    k_qblock_rows<<<min((n_rows + 7) / 8, 1024), dim3(32, 8), 0, st>>>(qb_off + n_rows + 1, n_rows,
-                                                                       qb_off + 2 * (n_rows + 1));
-    k_qblock_spans<<<min((n_rows + 7) / 8, 1024), dim3(32, 8), 0, st>>>(qb_off, cu_seqlens, n_rows,
-                                                                        qb_off + qb_span_offset(n_rows, n_tokens));
+    k_qblock_meta<<<1, 1024, 0, st>>>(cu_seqlens, n_rows, qb_off, qb_off + 2 * (n_rows + 1),
+                                      qb_off + qb_span_offset(n_rows, n_tokens));
     return cudaGetLastError();
 }
 
