@@ -450,8 +450,10 @@ def measure_latency(jl, wpath, local, calls, n_distinct=128):
     200-token state) through jd_decide_host, host serialisation and copies included.
     `distinct`: a pool of `n_distinct` seeded requests of that recipe (questions
     8..24 ids, options 3..20 ids, so each has its own length), called in turn;
-    eager launches and CUDA-graph mode side by side.  `repeated`: one request
-    called over and over in graph mode (every call replays the same graph)."""
+    eager launches and CUDA-graph mode side by side.  Graph mode keeps one graph
+    per bucket of padded shapes; one untimed pass over the pool captures them, so
+    the timed calls only replay (their capture count is reported).  `repeated`: one
+    request called over and over in graph mode."""
     from workloads import rows_config1
     o1 = jl.encode_opts(1024, 512, True)
     pool = [rows_config1(seed=101 + k) for k in range(n_distinct)]
@@ -459,14 +461,19 @@ def measure_latency(jl, wpath, local, calls, n_distinct=128):
 
     def run(graph, reqs):
         lm.jd_set_graph_mode(graph)
-        for k in range(20):
+        for k in range(max(20, len(reqs))):  # graph mode: every bucket of the pool captured before timing
             lm.jd_decide_host(reqs[k % len(reqs)], o1)
+        c0, r0, _ = lm.jd_graph_stats()
         ts = []
         for k in range(calls):
             t = time.perf_counter()
             lm.jd_decide_host(reqs[k % len(reqs)], o1)
             ts.append(1000 * (time.perf_counter() - t))
-        return {"p50_ms": _r(float(np.percentile(ts, 50))), "p99_ms": _r(float(np.percentile(ts, 99)))}
+        c1, r1, nb = lm.jd_graph_stats()
+        out = {"p50_ms": _r(float(np.percentile(ts, 50))), "p99_ms": _r(float(np.percentile(ts, 99)))}
+        if graph:
+            out.update(captures_in_timed_calls=c1 - c0, replays_in_timed_calls=r1 - r0, buckets=nb)
+        return out
 
     out = {"distinct_eager": run(False, pool), "distinct_graph": run(True, pool),
            "repeated_graph": run(True, pool[:1])}

@@ -117,6 +117,7 @@ def lib():
     L.jd_decide_packed_host.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.POINTER(jd_host_outputs), C.c_void_p]
     L.jd_check_status.argtypes = [C.c_void_p]
     L.jd_set_graph_mode.argtypes = [C.c_void_p, C.c_int]
+    L.jd_graph_stats.argtypes = [C.c_void_p, C.POINTER(C.c_int64), C.POINTER(C.c_int64), C.POINTER(C.c_int32)]
     L.jd_route_host.argtypes = [C.c_void_p, C.POINTER(jd_route_request), C.c_int32, C.POINTER(jd_encode_opts),
                                 C.c_int32, C.c_int32, C.c_int32, C.POINTER(jd_route_outputs), C.c_void_p]
     L.jd_route_host.restype = C.c_int
@@ -129,7 +130,7 @@ def lib():
     L.jd_set_profiling.argtypes = [C.c_void_p, C.c_int]
     L.jd_profile_report.argtypes = [C.c_void_p, C.c_char_p, C.c_size_t]
     for name in ("jd_serialize", "jd_model_create", "jd_model_create_shared", "jd_decide", "jd_forward", "jd_decide_host",
-                 "jd_decide_packed_host", "jd_check_status", "jd_set_graph_mode", "jd_set_profiling",
+                 "jd_decide_packed_host", "jd_check_status", "jd_set_graph_mode", "jd_graph_stats", "jd_set_profiling",
                  "jd_profile_report"):
         getattr(L, name).restype = C.c_int
     _lib = L
@@ -445,6 +446,12 @@ class Model:
 
     def jd_set_graph_mode(self, enable):
         _check(lib().jd_set_graph_mode(self.h, int(bool(enable))))
+
+    def jd_graph_stats(self):
+        """(graphs captured, calls served by replaying an earlier capture, buckets held)."""
+        c, r, b = C.c_int64(), C.c_int64(), C.c_int32()
+        _check(lib().jd_graph_stats(self.h, C.byref(c), C.byref(r), C.byref(b)))
+        return c.value, r.value, b.value
 
     def jd_last_launch_count(self):
         return lib().jd_last_launch_count(self.h)

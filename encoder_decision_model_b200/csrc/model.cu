@@ -17,6 +17,7 @@
 // mode).  Wi rows are interleaved in blocks of 128 ([u_j | g_j]) so that one
 // 256-wide GEMM tile holds both halves of 128 GEGLU outputs.
 
+#include <array>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -227,9 +228,20 @@ struct jd_model {
     int n_ev = 0;
     std::map<std::string, std::pair<long, double>> prof_acc;
 
-    // CUDA graph cache (one entry)
+    // CUDA graphs: one per bucket of padded batch shapes (tokens, rows, markers, longest row),
+    // least recently used dropped beyond GRAPH_BUCKETS_MAX, plus one exact-shape entry for the
+    // calls that no bucket serves (taps requested, or a bucket beyond the capacity)
     bool graph_mode = false;
+    struct Bucket {
+        cudaGraphExec_t exec = nullptr;
+        int launches = 0;
+        long last_use = 0;
+    };
+    std::map<std::array<int, 4>, Bucket> gbuckets;
+    long gclock = 0;
+    long g_captures = 0, g_replays = 0;
     cudaGraphExec_t gexec = nullptr;
+    int gexec_launches = 0;
     std::vector<uintptr_t> gkey;
 
     template <class T>
@@ -783,6 +795,84 @@ jd_status check_batch(jd_model *m, const jd_batch *b) {
     return JD_OK;
 }
 
+// Capture the launch sequence of one call on `st` (a private stream when st is the legacy
+// stream, which cannot be captured) and instantiate it.
+jd_status capture_forward(jd_model *m, const jd_batch *b, const jd_outputs *out, const jd_taps *taps,
+                          cudaStream_t st, cudaGraphExec_t *exec) {
+    cudaStream_t cap = st;
+    bool own = false;
+    if (cap == nullptr) {
+        CK(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
+        own = true;
+    }
+    CK(cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal));
+    jd_status s = enqueue_forward(m, b, out, taps, cap);
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamEndCapture(cap, &g);
+    if (own) cudaStreamDestroy(cap);
+    if (s != JD_OK) {
+        if (g) cudaGraphDestroy(g);
+        return s;
+    }
+    if (e != cudaSuccess) return fail(JD_ERR_CUDA, "graph capture: %s", cudaGetErrorString(e));
+    e = cudaGraphInstantiate(exec, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) return fail(JD_ERR_CUDA, "graph instantiate: %s", cudaGetErrorString(e));
+    ++m->g_captures;
+    return JD_OK;
+}
+
+constexpr size_t GRAPH_BUCKETS_MAX = 64;
+
+// The bucket of a batch in graph mode: its padded shape (pad_shape) and the longest row of the
+// padded batch as the graph sees it.  That is 1024 for batches whose rows all fit in 1024 tokens,
+// else the longest row rounded up to a multiple of 1024, so that the marker attention splits the
+// keys of every row as it does for the unpadded batch.  False when the padded batch exceeds the
+// model's capacity.
+bool graph_bucket(const jd_model *m, const jd_batch *b, PadShape *s, int *Lb) {
+    *s = pad_shape(b->n_tokens, b->n_rows, b->n_markers);
+    const int L = std::max(b->max_row_len, s->Tb - s->T);
+    *Lb = L <= 1024 ? 1024 : std::min(MAX_POS, (L + 1023) / 1024 * 1024);
+    return s->Tb <= m->T_cap && s->Bb <= m->B_cap && s->Mb <= m->M_cap;
+}
+
+// Replay (capturing on first use) the graph of a bucket.  Its batch is the padded one in the
+// model's device staging (d_tokens ...), its outputs the model's internal output arrays.
+jd_status bucket_replay(jd_model *m, const PadShape &s, int Lb, cudaStream_t st) {
+    const std::array<int, 4> key{s.Tb, s.Bb, s.Mb, Lb};
+    auto it = m->gbuckets.find(key);
+    if (it == m->gbuckets.end()) {
+        if (m->gbuckets.size() >= GRAPH_BUCKETS_MAX) {
+            auto lru = m->gbuckets.begin();
+            for (auto j = m->gbuckets.begin(); j != m->gbuckets.end(); ++j)
+                if (j->second.last_use < lru->second.last_use) lru = j;
+            cudaGraphExecDestroy(lru->second.exec);
+            m->gbuckets.erase(lru);
+        }
+        jd_batch db{};
+        db.n_rows = s.Bb;
+        db.n_tokens = s.Tb;
+        db.n_markers = s.Mb;
+        db.max_row_len = Lb;
+        db.tokens = m->d_tokens;
+        db.cu_seqlens = m->d_cu;
+        db.mask_pos = m->d_mask;
+        db.opt_off = m->d_opt;
+        db.row_type = m->d_type;
+        jd_outputs o{m->i_logits, m->i_probs, m->i_choice, m->i_score, m->i_noul, m->i_maxp};
+        jd_model::Bucket bk;
+        TRY(capture_forward(m, &db, &o, nullptr, st, &bk.exec));
+        bk.launches = m->launches;
+        it = m->gbuckets.emplace(key, bk).first;
+    } else {
+        ++m->g_replays;
+    }
+    it->second.last_use = ++m->gclock;
+    CK(cudaGraphLaunch(it->second.exec, st));
+    m->launches = it->second.launches;
+    return JD_OK;
+}
+
 // Resolves the no-allocation path's static array on `dev` (defined with it below).
 jd_status noalloc_prepare(int dev);
 
@@ -874,6 +964,7 @@ extern "C" void jd_model_destroy(jd_model *m) {
     if (!m) return;
     cudaSetDevice(m->device);
     if (m->gexec) cudaGraphExecDestroy(m->gexec);
+    for (auto &kv : m->gbuckets) cudaGraphExecDestroy(kv.second.exec);
     for (cudaEvent_t e : m->ev) cudaEventDestroy(e);
     for (void *p : m->allocs) cudaFree(p);
     for (void *p : m->hallocs) cudaFreeHost(p);
@@ -886,6 +977,15 @@ extern "C" jd_status jd_set_graph_mode(jd_model *m, int enable) {
     clear_error();
     if (!m) return fail(JD_ERR_INVALID_ARG, "model is NULL");
     m->graph_mode = enable != 0;
+    return JD_OK;
+}
+
+extern "C" jd_status jd_graph_stats(const jd_model *m, int64_t *captures, int64_t *replays, int32_t *buckets) {
+    clear_error();
+    if (!m) return fail(JD_ERR_INVALID_ARG, "model is NULL");
+    if (captures) *captures = m->g_captures;
+    if (replays) *replays = m->g_replays;
+    if (buckets) *buckets = (int32_t)m->gbuckets.size();
     return JD_OK;
 }
 
@@ -905,11 +1005,26 @@ extern "C" jd_status jd_decide(jd_model *m, const jd_batch *b, const jd_outputs 
     }
     if (!m->graph_mode) return enqueue_forward(m, b, out, taps, st);
 
+    PadShape ps;
+    int Lb = 0;
+    if (!taps && graph_bucket(m, b, &ps, &Lb)) {
+        // the padded batch into the model's staging, the bucket's graph, the real rows out
+        LK(launch_pad_batch(ps, b->tokens, b->cu_seqlens, b->mask_pos, b->opt_off, b->row_type, m->d_tokens,
+                            m->d_cu, m->d_mask, m->d_opt, m->d_type, st));
+        TRY(bucket_replay(m, ps, Lb, st));
+        LK(launch_unpad_outputs(b->n_markers, b->n_rows, m->i_logits, m->i_probs, m->i_choice, m->i_score,
+                                m->i_noul, m->i_maxp, out->logits, out->probs, out->choice, out->score, out->noul,
+                                out->max_p, st));
+        m->launches += 2;
+        return JD_OK;
+    }
+
     std::vector<uintptr_t> key = {(uintptr_t)b->n_tokens,  (uintptr_t)b->n_rows,     (uintptr_t)b->n_markers,
                                   (uintptr_t)b->tokens,    (uintptr_t)b->cu_seqlens, (uintptr_t)b->mask_pos,
                                   (uintptr_t)b->opt_off,   (uintptr_t)b->row_type,   (uintptr_t)out->logits,
                                   (uintptr_t)out->probs,   (uintptr_t)out->choice,   (uintptr_t)out->score,
                                   (uintptr_t)out->noul,    (uintptr_t)out->max_p,
+                                  (uintptr_t)b->max_row_len,
                                   (uintptr_t)(taps ? taps->encoder_out : nullptr),
                                   (uintptr_t)(taps ? taps->marker_state : nullptr)};
     if (!m->gexec || key != m->gkey) {
@@ -917,28 +1032,14 @@ extern "C" jd_status jd_decide(jd_model *m, const jd_batch *b, const jd_outputs 
             cudaGraphExecDestroy(m->gexec);
             m->gexec = nullptr;
         }
-        cudaStream_t cap = st;
-        bool own = false;
-        if (cap == nullptr) {  // the legacy stream cannot be captured: capture on a private one
-            CK(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
-            own = true;
-        }
-        CK(cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal));
-        jd_status s = enqueue_forward(m, b, out, taps, cap);
-        cudaGraph_t g = nullptr;
-        cudaError_t e = cudaStreamEndCapture(cap, &g);
-        if (own) cudaStreamDestroy(cap);
-        if (s != JD_OK) {
-            if (g) cudaGraphDestroy(g);
-            return s;
-        }
-        if (e != cudaSuccess) return fail(JD_ERR_CUDA, "graph capture: %s", cudaGetErrorString(e));
-        e = cudaGraphInstantiate(&m->gexec, g, 0);
-        cudaGraphDestroy(g);
-        if (e != cudaSuccess) return fail(JD_ERR_CUDA, "graph instantiate: %s", cudaGetErrorString(e));
+        TRY(capture_forward(m, b, out, taps, st, &m->gexec));
+        m->gexec_launches = m->launches;
         m->gkey = key;
+    } else {
+        ++m->g_replays;
     }
     CK(cudaGraphLaunch(m->gexec, st));
+    m->launches = m->gexec_launches;
     return JD_OK;
 }
 
@@ -957,26 +1058,44 @@ extern "C" jd_status jd_decide_packed_host(jd_model *m, const jd_batch *hb, jd_h
     CK(cudaSetDevice(m->device));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int T = hb->n_tokens, B = hb->n_rows, M = hb->n_markers;
+    // graph mode: the batch padded to its bucket on the host, so that its graph reads it from the
+    // staging arrays and writes the internal outputs directly
+    PadShape ps = pad_shape(T, B, M);
+    int Lb = 0;
+    const bool bucket = m->graph_mode && !m->prof && graph_bucket(m, hb, &ps, &Lb);
+    if (!bucket) ps = PadShape{T, B, M, T, B, M};
     memcpy(m->h_tokens, hb->tokens, sizeof(int) * T);
     memcpy(m->h_cu, hb->cu_seqlens, sizeof(int) * (B + 1));
     memcpy(m->h_mask, hb->mask_pos, sizeof(int) * M);
     memcpy(m->h_opt, hb->opt_off, sizeof(int) * (B + 1));
     memcpy(m->h_type, hb->row_type, sizeof(int) * B);
-    CK(cudaMemcpyAsync(m->d_tokens, m->h_tokens, sizeof(int) * T, cudaMemcpyHostToDevice, st));
-    CK(cudaMemcpyAsync(m->d_cu, m->h_cu, sizeof(int) * (B + 1), cudaMemcpyHostToDevice, st));
-    CK(cudaMemcpyAsync(m->d_mask, m->h_mask, sizeof(int) * M, cudaMemcpyHostToDevice, st));
-    CK(cudaMemcpyAsync(m->d_opt, m->h_opt, sizeof(int) * (B + 1), cudaMemcpyHostToDevice, st));
-    CK(cudaMemcpyAsync(m->d_type, m->h_type, sizeof(int) * B, cudaMemcpyHostToDevice, st));
-    jd_batch db = *hb;
-    db.tokens = m->d_tokens;
-    db.cu_seqlens = m->d_cu;
-    db.mask_pos = m->d_mask;
-    db.opt_off = m->d_opt;
-    db.row_type = m->d_type;
-    db.head_len = nullptr;
-    db.trunc = nullptr;
-    jd_outputs o{m->i_logits, m->i_probs, m->i_choice, m->i_score, m->i_noul, m->i_maxp};
-    TRY(jd_decide(m, &db, &o, nullptr, stream));
+    for (int i = T; i < ps.Tb; ++i) m->h_tokens[i] = pad_token_at(ps, hb->tokens, i);
+    for (int i = B + 1; i <= ps.Bb; ++i) {
+        m->h_cu[i] = pad_cu_at(ps, hb->cu_seqlens, i);
+        m->h_opt[i] = pad_opt_at(ps, hb->opt_off, i);
+    }
+    for (int i = M; i < ps.Mb; ++i) m->h_mask[i] = pad_mask_at(ps, hb->mask_pos, i);
+    for (int i = B; i < ps.Bb; ++i) m->h_type[i] = pad_type_at(ps, hb->row_type, i);
+    CK(cudaMemcpyAsync(m->d_tokens, m->h_tokens, sizeof(int) * ps.Tb, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_cu, m->h_cu, sizeof(int) * (ps.Bb + 1), cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_mask, m->h_mask, sizeof(int) * ps.Mb, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_opt, m->h_opt, sizeof(int) * (ps.Bb + 1), cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_type, m->h_type, sizeof(int) * ps.Bb, cudaMemcpyHostToDevice, st));
+    if (bucket) {
+        m->last_stream = st;
+        TRY(bucket_replay(m, ps, Lb, st));
+    } else {
+        jd_batch db = *hb;
+        db.tokens = m->d_tokens;
+        db.cu_seqlens = m->d_cu;
+        db.mask_pos = m->d_mask;
+        db.opt_off = m->d_opt;
+        db.row_type = m->d_type;
+        db.head_len = nullptr;
+        db.trunc = nullptr;
+        jd_outputs o{m->i_logits, m->i_probs, m->i_choice, m->i_score, m->i_noul, m->i_maxp};
+        TRY(jd_decide(m, &db, &o, nullptr, stream));
+    }
     CK(cudaMemcpyAsync(m->h_logits, m->i_logits, sizeof(float) * M, cudaMemcpyDeviceToHost, st));
     CK(cudaMemcpyAsync(m->h_probs, m->i_probs, sizeof(float) * M, cudaMemcpyDeviceToHost, st));
     CK(cudaMemcpyAsync(m->h_choice, m->i_choice, sizeof(int) * B, cudaMemcpyDeviceToHost, st));

@@ -180,6 +180,63 @@ cudaError_t launch_gather_markers(const int *mask_pos, int n_markers, int n_toke
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ bucket padding
+
+__global__ void __launch_bounds__(256)
+    k_pad_batch(PadShape s, const int *tokens, const int *cu, const int *mask, const int *opt, const int *type,
+                int *dtokens, int *dcu, int *dmask, int *dopt, int *dtype) {
+    const int stride = gridDim.x * blockDim.x;
+    const int n = max(s.Tb, max(s.Mb, s.Bb + 1));
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        if (i < s.Tb) dtokens[i] = pad_token_at(s, tokens, i);
+        if (i < s.Mb) dmask[i] = pad_mask_at(s, mask, i);
+        if (i <= s.Bb) {
+            dcu[i] = pad_cu_at(s, cu, i);
+            dopt[i] = pad_opt_at(s, opt, i);
+        }
+        if (i < s.Bb) dtype[i] = pad_type_at(s, type, i);
+    }
+}
+
+cudaError_t launch_pad_batch(const PadShape &s, const int *tokens, const int *cu, const int *mask, const int *opt,
+                             const int *type, int *dtokens, int *dcu, int *dmask, int *dopt, int *dtype,
+                             cudaStream_t st) {
+    const int n = max(s.Tb, max(s.Mb, s.Bb + 1));
+    k_pad_batch<<<min((n + 255) / 256, 1184), 256, 0, st>>>(s, tokens, cu, mask, opt, type, dtokens, dcu, dmask,
+                                                             dopt, dtype);
+    return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256)
+    k_unpad_outputs(int M, int B, const float *logits, const float *probs, const int *choice, const float *score,
+                    const float *noul, const float *max_p, float *o_logits, float *o_probs, int *o_choice,
+                    float *o_score, float *o_noul, float *o_max_p) {
+    const int stride = gridDim.x * blockDim.x;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < max(M, B); i += stride) {
+        if (i < M) {
+            o_logits[i] = logits[i];
+            o_probs[i] = probs[i];
+        }
+        if (i < B) {
+            o_choice[i] = choice[i];
+            o_score[i] = score[i];
+            o_noul[i] = noul[i];
+            o_max_p[i] = max_p[i];
+        }
+    }
+}
+
+cudaError_t launch_unpad_outputs(int M, int B, const float *logits, const float *probs, const int *choice,
+                                 const float *score, const float *noul, const float *max_p, float *o_logits,
+                                 float *o_probs, int *o_choice, float *o_score, float *o_noul, float *o_max_p,
+                                 cudaStream_t st) {
+    const int n = max(M, B);
+    if (n <= 0) return cudaSuccess;
+    k_unpad_outputs<<<min((n + 255) / 256, 148), 256, 0, st>>>(M, B, logits, probs, choice, score, noul, max_p,
+                                                              o_logits, o_probs, o_choice, o_score, o_noul, o_max_p);
+    return cudaGetLastError();
+}
+
 cudaError_t gemm_init_attributes();
 cudaError_t attn_init_attributes();
 cudaError_t head_init_attributes();

@@ -315,11 +315,30 @@ jd_status jd_route_scored(const jd_route_request *requests, int32_t n_requests, 
  * JD_ERR_DEVICE_STATUS with a message if a kernel recorded a failure. */
 jd_status jd_check_status(jd_model *model);
 
-/* CUDA-graph replay for repeated calls of one batch shape: the first call
- * with a given (n_tokens, n_rows, n_markers, batch pointers, outputs)
- * captures the whole jd_decide launch sequence on `stream`; later calls with
- * the same key replay it.  enable = 0 turns capture off (the default). */
+/* CUDA-graph mode ("Julia-1 MLX", "Performance": batch-1 requests, where the
+ * fixed cost of each call decides the latency).  enable = 0 turns it off (the
+ * default: every call launches its kernels).  In graph mode a call runs its
+ * batch padded to a bucket: n_tokens rounded up from n_tokens + 8 to a
+ * multiple of 128, n_rows + 1 rows and n_markers rounded up from n_markers + 1
+ * to a multiple of 8; the added last row holds the extra tokens (id 0) and
+ * markers.  Each bucket's launch sequence is captured once, into a graph that
+ * reads the padded batch from the model's own staging arrays; every later
+ * call of that bucket, whatever its exact shape and pointers, copies its
+ * batch there (jd_decide: one small kernel; jd_decide_packed_host /
+ * jd_decide_host: the host-to-device copies it makes anyway), replays the
+ * graph and copies its rows' outputs out.  No row's result depends on the
+ * rest of its batch, so the outputs equal those of eager launches bit for bit
+ * (the marker attention's key split, which depends on the longest row, is kept
+ * by bucketing that length too).  At most 64 buckets are kept, the least
+ * recently used dropped first.  Calls whose padded batch exceeds the model's
+ * capacity, and jd_decide calls with taps, use one graph keyed on their exact
+ * shape and pointers instead, captured again whenever those change. */
 jd_status jd_set_graph_mode(jd_model *model, int enable);
+
+/* Graph-mode counters of this handle since it was created: graphs captured,
+ * calls served by replaying a graph captured earlier, buckets held now.  Any
+ * pointer may be NULL. */
+jd_status jd_graph_stats(const jd_model *model, int64_t *captures, int64_t *replays, int32_t *buckets);
 
 /* Number of kernels the last jd_decide / jd_forward call launched (the same
  * sequence whether replayed from a graph or launched eagerly). */

@@ -112,19 +112,58 @@ def test_decide_host_equals_device(bf16_model):
     np.testing.assert_array_equal(ho["choice"], res["choice"])
 
 
+def _same_bucket_pair(opts):
+    """Two seeded 3-question requests whose packed batches differ in length but share a graph
+    bucket (tokens rounded up from T + 8 to a multiple of 128, markers from M + 1 to a multiple of 8)."""
+    seen = {}
+    for seed in range(101, 400):
+        rows = rows_config1(seed=seed)
+        hb = jl.jd_serialize(rows, jl.encode_opts(**opts))
+        key = ((hb.n_tokens + 8 + 127) // 128, hb.n_rows, (hb.n_markers + 8) // 8)
+        if key in seen and seen[key][1] != hb.n_tokens:
+            return seen[key][0], rows
+        seen.setdefault(key, (rows, hb.n_tokens))
+    raise AssertionError("no two requests share a bucket")
+
+
 def test_graph_replay_equals_eager(bf16_model):
+    """Graph mode against eager launches, bit for bit, on two request shapes of one bucket: the
+    first call captures the bucket's graph, the second (another length, other device buffers)
+    replays it; then the same two through the host entry point, and the exact-shape graph that a
+    call with taps takes."""
     import torch
-    rows = rows_config1()
-    hb, res = device_run(bf16_model, rows, OPT1)
+    ra, rb = _same_bucket_pair(OPT1)
+    eager = [device_run(bf16_model, r, OPT1)[1] for r in (ra, rb)]
+    eager_host = [bf16_model.jd_decide_host(r, jl.encode_opts(**OPT1)) for r in (ra, rb)]
+    keys = ("logits", "probs", "choice", "score", "noul", "max_p")
+    c0, r0, _ = bf16_model.jd_graph_stats()
     bf16_model.jd_set_graph_mode(True)
     try:
         s = torch.cuda.Stream()
         with torch.cuda.stream(s):
-            for _ in range(2):
-                hb2, res2 = device_run(bf16_model, rows, OPT1, stream=s)
-                np.testing.assert_array_equal(res2["logits"], res["logits"])
+            for i, r in enumerate((ra, rb, ra)):
+                _, res = device_run(bf16_model, r, OPT1, stream=s)
+                for k in keys:
+                    np.testing.assert_array_equal(res[k], eager[i % 2][k], err_msg=f"request {i % 2}: {k}")
+            c1, r1, _ = bf16_model.jd_graph_stats()
+            assert (c1 - c0, r1 - r0) == (1, 2), (c1 - c0, r1 - r0)
+            for i, r in enumerate((ra, rb)):
+                o = bf16_model.jd_decide_host(r, jl.encode_opts(**OPT1), stream=s)
+                for k in keys:
+                    np.testing.assert_array_equal(o[k], eager_host[i][k], err_msg=f"host request {i}: {k}")
+            c2, r2, _ = bf16_model.jd_graph_stats()
+            assert (c2 - c1, r2 - r1) == (0, 2), (c2 - c1, r2 - r1)
+            # taps: the exact-shape graph
+            tap_graph = [device_run(bf16_model, ra, OPT1, taps=True, stream=s)[1]]
+            c3, _, _ = bf16_model.jd_graph_stats()
+            assert c3 - c2 == 1
     finally:
         bf16_model.jd_set_graph_mode(False)
+    tap_eager = device_run(bf16_model, ra, OPT1, taps=True)[1]
+    for k in keys + ("encoder_out", "marker_state"):
+        np.testing.assert_array_equal(tap_graph[0][k], tap_eager[k], err_msg=f"taps: {k}")
+    for k in keys:
+        np.testing.assert_array_equal(tap_eager[k], eager[0][k], err_msg=f"taps against no taps: {k}")
 
 
 def test_capacity_and_status_errors(bf16_model):
