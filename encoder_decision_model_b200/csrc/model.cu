@@ -30,6 +30,7 @@
 #include "e4m3.h"
 #include "host_common.h"
 #include "kernels.h"
+#include "batch_pad.h"
 
 using namespace jd;
 

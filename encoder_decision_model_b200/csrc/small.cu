@@ -3,6 +3,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "batch_pad.h"
 
 namespace jd {
 
