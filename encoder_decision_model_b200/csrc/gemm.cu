@@ -218,6 +218,56 @@ struct OutStage {
 };
 
 // Write 4 x 16 bytes (32 bf16) of row r into 16-byte chunks c0..c0+3 of a swizzled box.
+// GELU(u) * g for a pair of columns, FP32, on packed f32x2 FMAs and one ex2 per value.
+// GELU(x) = x Phi(x) = max(x, 0) - |x| Phi(-|x|), and the normal tail is written as
+// Phi(-a) = 2^(P(a / 6) - a^2 log2(e) / 2), P the degree-7 polynomial of least maximum error
+// against log2 Phi(-6 s) + 18 s^2 log2(e) on s in [0, 1] (Remez exchange; |error| <= 4.8e-6 in
+// log2, a relative error of 3.3e-6 in the tail, so |GELU error| < 1e-6).  Past |x| = 6 the
+// polynomial is held at s = 1 while the Gaussian factor keeps falling; the tail there is below
+// 1e-9.  erf's rational form (gelu_as) needs a reciprocal and an ex2 per value: the special-
+// function unit then worked as long as the tile's MMAs.
+constexpr float GT_C0 = -0.9999952912330627f, GT_C1 = -6.907506465911865f, GT_C2 = 9.46379280090332f,
+                GT_C3 = -11.655374526977539f, GT_C4 = 11.026226043701172f, GT_C5 = -7.235760688781738f,
+                GT_C6 = 2.873929500579834f, GT_C7 = -0.5136296153068542f;
+constexpr float GT_G = -25.968510341644287f;  // -36 log2(e) / 2: the Gaussian factor in s
+__device__ __forceinline__ float2 f2mul(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 f2c(float v) { return make_float2(v, v); }
+__device__ __forceinline__ float2 geglu_pair(float2 x, float2 g) {
+    const float2 na = make_float2(-fabsf(x.x), -fabsf(x.y));
+    const float2 s = f2mul(na, f2c(-1.0f / 6.0f));
+    const float2 sc = make_float2(fminf(s.x, 1.0f), fminf(s.y, 1.0f));
+    float2 p = f2fma(sc, f2c(GT_C7), f2c(GT_C6));
+    p = f2fma(p, sc, f2c(GT_C5));
+    p = f2fma(p, sc, f2c(GT_C4));
+    p = f2fma(p, sc, f2c(GT_C3));
+    p = f2fma(p, sc, f2c(GT_C2));
+    p = f2fma(p, sc, f2c(GT_C1));
+    p = f2fma(p, sc, f2c(GT_C0));
+    const float2 arg = f2fma(f2mul(s, s), f2c(GT_G), p);
+    float2 t;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(t.x) : "f"(arg.x));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(t.y) : "f"(arg.y));
+    const float2 y = f2fma(na, t, make_float2(fmaxf(x.x, 0.0f), fmaxf(x.y, 0.0f)));
+    return f2mul(y, g);
+}
+
 __device__ __forceinline__ void stage_row32(uint8_t *box, int r, int c0, const uint32_t (&w)[16]) {
 #pragma unroll
     for (int q = 0; q < 4; ++q)
@@ -233,8 +283,8 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
         // stored straight from registers: a shared-memory staging pass here
         // competes with the 256-wide MMAs for shared-memory bandwidth; with
         // NPART warps per TMEM lane quarter each takes G / NPART output columns.
-        // GELU uses the rational erf approximation (gelu_as, |error| < 5e-7):
-        // with erff this epilogue was slower than the tile's MMAs.
+        // GELU by geglu_pair (one ex2 per value): with erff, and then with erf's rational
+        // form, this epilogue kept the special-function unit as busy as the tile's MMAs.
         constexpr int G = BN / 2;
         constexpr int GP = G / NPART;
         static_assert(GP == 64, "two 32-column chunks per warp");
@@ -249,8 +299,9 @@ __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0,
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = q * 16 + e * 2;
-                        w[e] = pack_bf16x2(gelu_as(__uint_as_float(u[j])) * __uint_as_float(g[j]),
-                                           gelu_as(__uint_as_float(u[j + 1])) * __uint_as_float(g[j + 1]));
+                        const float2 y = geglu_pair(make_float2(__uint_as_float(u[j]), __uint_as_float(u[j + 1])),
+                                                    make_float2(__uint_as_float(g[j]), __uint_as_float(g[j + 1])));
+                        w[e] = pack_bf16x2(y.x, y.y);
                     }
                     st_global_v8(dst + 32 * q, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
                 }
@@ -1509,6 +1560,7 @@ cudaError_t gemm_init_attributes() {
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_QKV, 64, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<64>::SMEM)) != cudaSuccess)
         return e;
+
     if ((e = cudaFuncSetAttribute(k_gemm_pc<EPI_GEGLU, 256, GEGLU_EW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   PcCfg<256>::SMEM)) != cudaSuccess)
         return e;
