@@ -50,27 +50,6 @@ __device__ __forceinline__ void st_global_v8(void *p, uint32_t a0, uint32_t a1, 
 
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
 
-// GELU(x) = x Phi(x), Phi(x) = (1 + erf(x / sqrt 2)) / 2, with erf from the rational
-// approximation of Abramowitz and Stegun, Handbook of Mathematical Functions,
-// eq. 7.1.26 (|error| <= 1.5e-7 for z >= 0; odd symmetry for z < 0):
-//   erf(z) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),  t = 1 / (1 + p z).
-// With z = |x| / sqrt 2 the 1 / sqrt 2 is folded into p, the 1/2 of Phi into a1..a5,
-// and x (1 - erf(z)) / 2 = xh gives GELU = x - xh (x >= 0) or xh (x < 0): one
-// reciprocal and one exp2 on the special-function unit and eleven FMA-pipe
-// operations (|GELU error| <= 3.4e-7 against the erf form in fp32).
-__device__ __forceinline__ float gelu_as(float x) {
-    float t;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.23164188861846924f, fabsf(x), 1.0f)));
-    float p = fmaf(0.5307027101516724f, t, -0.726576030254364f);
-    p = fmaf(p, t, 0.710706889629364f);
-    p = fmaf(p, t, -0.14224836230278015f);
-    p = fmaf(p, t, 0.1274147927761078f);
-    float e;  // exp(-x^2 / 2) = 2^(-x^2 log2(e) / 2)
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x * (x * -0.7213475108146667f)));
-    const float xh = x * ((p * t) * e);
-    return x >= 0.f ? x - xh : xh;
-}
-
 // Two floats to FP8 E4M3 bytes (round to nearest even, saturating at +-448): lo in the low byte.
 __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
     uint16_t d;

@@ -224,8 +224,8 @@ struct OutStage {
 // against log2 Phi(-6 s) + 18 s^2 log2(e) on s in [0, 1] (Remez exchange; |error| <= 4.8e-6 in
 // log2, a relative error of 3.3e-6 in the tail, so |GELU error| < 1e-6).  Past |x| = 6 the
 // polynomial is held at s = 1 while the Gaussian factor keeps falling; the tail there is below
-// 1e-9.  erf's rational form (gelu_as) needs a reciprocal and an ex2 per value: the special-
-// function unit then worked as long as the tile's MMAs.
+// 1e-9.  erf's rational form (Abramowitz and Stegun 7.1.26) needs a reciprocal and an ex2 per
+// value: the special-function unit then worked as long as the tile's MMAs.
 constexpr float GT_C0 = -0.9999952912330627f, GT_C1 = -6.907506465911865f, GT_C2 = 9.46379280090332f,
                 GT_C3 = -11.655374526977539f, GT_C4 = 11.026226043701172f, GT_C5 = -7.235760688781738f,
                 GT_C6 = 2.873929500579834f, GT_C7 = -0.5136296153068542f;
