@@ -554,20 +554,29 @@ def measure_router(jl, wpath, local, rank, ranks, reps, peaks):
     """Router workload: 512 independent requests, each a 256-id state, a question
     and 72 labels; round 1 scores groups of <=20 labels (4 rows per request), the
     survivors go to one final row per request.  decisions/s = requests / wall time
-    of jd_route_host (serialisation, both forward rounds, survivor rule, copies).
+    of jd_route_device (rows of both rounds formed and packed on the device, forward
+    rounds, survivor rule, copies), with jd_route_host (host serialisation per round)
+    timed beside it and its outputs compared.
     Round 1 is also run alone with per-kernel events to give the HBM fraction of
     the attention, norm and gather kernels at this shape."""
     from workloads import Row, requests_config4
     reqs = requests_config4(512, seed=104 + 1000 * rank)
     opts = jl.encode_opts(1024, 512, True)
     m = jl.Model(wpath, 1 << 20, 2048, 2048 * 20, precision=jl.JD_PREC_BF16, device=local)
-    for _ in range(2):
-        out = m.jd_route_host(reqs, opts)
-    ranks.barrier()
-    t0 = time.perf_counter()
-    for _ in range(reps):
-        out = m.jd_route_host(reqs, opts)
-    el = ranks.max(time.perf_counter() - t0)
+
+    def timed(call):
+        for _ in range(2):
+            o = call(reqs, opts)
+        ranks.barrier()
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            o = call(reqs, opts)
+        return o, ranks.max(time.perf_counter() - t0)
+
+    out_h, el_h = timed(m.jd_route_host)
+    out, el = timed(m.jd_route_device)
+    same = all(np.array_equal(np.asarray(out[k]), np.asarray(out_h[k]))
+               for k in ("winner", "winner_p", "final_candidates", "final_probs", "rows_per_round"))
     total = ranks.sum(float(len(reqs) * reps))
     m.jd_check_status()
     m.close()
@@ -579,6 +588,11 @@ def measure_router(jl, wpath, local, rank, ranks, reps, peaks):
     return {"workload": "512 requests x 72 labels of 3..12 ids on a 256-id state; groups of <=20, then one "
                         "final row of the survivors; head budget 512, max_length 1024, strict",
             "value": _r(total / el), "unit": "requests/s", "ms_per_call": _r(1000 * el / reps),
+            "call": "jd_route_device (rounds formed, encoded and narrowed on the device; four counters read "
+                    "back per round)",
+            "host_rounds": {"value": _r(total / el_h), "ms_per_call": _r(1000 * el_h / reps),
+                            "call": "jd_route_host (each round serialised on the host)",
+                            "outputs_identical": bool(same)},
             "rows_per_round": [int(x) for x in out["rows_per_round"]],
             "round1": {"rows": int(hb.n_rows), "tokens": int(hb.n_tokens), "markers": int(hb.n_markers),
                        "ms_forward": _r(ms),

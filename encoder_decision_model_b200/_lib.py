@@ -121,6 +121,9 @@ def lib():
     L.jd_route_host.argtypes = [C.c_void_p, C.POINTER(jd_route_request), C.c_int32, C.POINTER(jd_encode_opts),
                                 C.c_int32, C.c_int32, C.c_int32, C.POINTER(jd_route_outputs), C.c_void_p]
     L.jd_route_host.restype = C.c_int
+    L.jd_route_device.argtypes = [C.c_void_p, C.POINTER(jd_route_request), C.c_int32, C.POINTER(jd_encode_opts),
+                                  C.POINTER(jd_route_outputs), C.c_void_p]
+    L.jd_route_device.restype = C.c_int
     L.jd_forward_noalloc.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.c_void_p, C.c_void_p]
     L.jd_forward_noalloc.restype = C.c_int
     L.jd_noalloc_check_status.argtypes = [C.c_void_p, C.c_void_p]
@@ -429,6 +432,12 @@ class Model:
         _check(lib().jd_route_host(self.h, arr, len(requests), C.byref(opts), int(max_tokens or c.max_tokens),
                                    int(max_rows or c.max_rows), int(max_markers or c.max_markers), C.byref(s),
                                    _stream(stream)))
+        return _route_result(o, s)
+
+    def jd_route_device(self, requests, opts: jd_encode_opts, stream=None):
+        """jd_route_host with the rounds on the device; the same dict."""
+        arr, keep, o, s = _route_marshal(requests)
+        _check(lib().jd_route_device(self.h, arr, len(requests), C.byref(opts), C.byref(s), _stream(stream)))
         return _route_result(o, s)
 
     def jd_forward_noalloc(self, batch: jd_batch, logits, stream=None):

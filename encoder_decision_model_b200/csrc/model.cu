@@ -17,6 +17,7 @@
 // mode).  Wi rows are interleaved in blocks of 128 ([u_j | g_j]) so that one
 // 256-wide GEMM tile holds both halves of 128 GEGLU outputs.
 
+#include <algorithm>
 #include <array>
 #include <cmath>
 #include <cstdio>
@@ -31,6 +32,7 @@
 #include "host_common.h"
 #include "kernels.h"
 #include "batch_pad.h"
+#include "route_kernels.h"
 
 using namespace jd;
 
@@ -220,6 +222,11 @@ struct jd_model {
     int *h_choice = nullptr;
 
     cudaStream_t last_stream = nullptr;
+
+    // device-side router (jd_route_device): workspace grown on demand, pinned read-back slots
+    void *route_buf = nullptr;
+    size_t route_bytes = 0;
+    int *h_route = nullptr;  // [16]: the round's counters, then the status word
     int launches = 0;
 
     // per-kernel event timing (profiling mode)
@@ -509,6 +516,7 @@ jd_status alloc_workspace(jd_model *m) {
     TRY(m->halloc(&m->h_score, B));
     TRY(m->halloc(&m->h_noul, B));
     TRY(m->halloc(&m->h_maxp, B));
+    TRY(m->halloc(&m->h_route, 16));
     if (!m->fp32) {
         TRY(make_map(&m->tm_xn, m->xn, D, T, D, 64, 128));
         TRY(make_map(&m->tm_o, m->o, D, T, D, 64, 128));
@@ -968,6 +976,7 @@ extern "C" void jd_model_destroy(jd_model *m) {
     for (auto &kv : m->gbuckets) cudaGraphExecDestroy(kv.second.exec);
     for (cudaEvent_t e : m->ev) cudaEventDestroy(e);
     for (void *p : m->allocs) cudaFree(p);
+    if (m->route_buf) cudaFree(m->route_buf);
     for (void *p : m->hallocs) cudaFreeHost(p);
     delete m;
 }
@@ -1127,6 +1136,197 @@ extern "C" jd_status jd_decide_host(jd_model *m, const jd_row *rows, int32_t n_r
     s = jd_decide_packed_host(m, hb, ho, stream);
     jd_batch_free(hb);
     return s;
+}
+
+// ================================================================== router rounds on the device
+//
+// The same tournament as jd_route_host with the candidates, the rows of every round and the
+// survivor rule on the device: the requests are uploaded once; per round the host reads back
+// four counters (rows, tokens, markers, longest row) to size the forward pass's launches, and
+// nothing else crosses until the final outputs.
+
+namespace {
+
+struct RouteLayout {
+    size_t off[16] = {};
+    size_t bytes = 0;
+    size_t add(size_t n) {
+        const size_t o = bytes;
+        bytes += (n + 63) / 64 * 64;  // 64-byte aligned pieces
+        return o;
+    }
+};
+
+}  // namespace
+
+extern "C" jd_status jd_route_device(jd_model *m, const jd_route_request *reqs, int32_t n_requests,
+                                     const jd_encode_opts *opts, jd_route_outputs *out, void *stream) {
+    clear_error();
+    if (!m || !opts || !out || (n_requests > 0 && !reqs) || n_requests < 0)
+        return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    if (n_requests > 0 && !out->winner) return fail(JD_ERR_INVALID_ARG, "out->winner is NULL");
+    if (out->rows_per_round && out->max_rounds < 0) return fail(JD_ERR_INVALID_ARG, "max_rounds < 0");
+    if (opts->max_length < 1 || opts->max_length > MAX_POS || opts->head_budget < 1 || opts->vocab < 1)
+        return fail(JD_ERR_INVALID_ARG, "max_length must be in [1, 8192] and head_budget >= 1");
+    auto in_vocab = [&](const int32_t *p, int n) {
+        for (int i = 0; i < n; ++i)
+            if (p[i] < 0 || p[i] >= opts->vocab) return false;
+        return true;
+    };
+    const int32_t special[3] = {opts->bos, opts->eos, opts->mask};
+    if (!in_vocab(special, 3)) return fail(JD_ERR_TOKEN_RANGE, "bos/eos/mask id outside [0, %d)", opts->vocab);
+    out->n_rounds = 0;
+    if (n_requests == 0) return JD_OK;
+
+    // the request pool: req[6] per request, lab[2] per label, then every id
+    std::vector<int32_t> req((size_t)n_requests * 6), lab, ids;
+    for (int r = 0; r < n_requests; ++r) {
+        const jd_route_request &q = reqs[r];
+        if (q.n_labels < 1 || q.n_labels > 4096 || !q.labels || !q.n_label_ids)
+            return fail(JD_ERR_INVALID_ARG, "request %d: 1..4096 labels required", r);
+        if (q.n_question < 0 || q.n_state < 0 || (q.n_question && !q.question) || (q.n_state && !q.state))
+            return fail(JD_ERR_INVALID_ARG, "request %d has a null array or a negative length", r);
+        if (!in_vocab(q.question, q.n_question) || !in_vocab(q.state, q.n_state))
+            return fail(JD_ERR_TOKEN_RANGE, "request %d: token id outside [0, %d)", r, opts->vocab);
+        int32_t *rq = req.data() + (size_t)r * 6;
+        rq[0] = (int32_t)ids.size();
+        rq[1] = q.n_question;
+        ids.insert(ids.end(), q.question, q.question + q.n_question);
+        rq[2] = (int32_t)ids.size();
+        rq[3] = q.n_state;
+        ids.insert(ids.end(), q.state, q.state + q.n_state);
+        rq[4] = (int32_t)(lab.size() / 2);
+        rq[5] = q.n_labels;
+        for (int i = 0; i < q.n_labels; ++i) {
+            const int n = q.n_label_ids[i];
+            if (n < 0 || (n && !q.labels[i])) return fail(JD_ERR_INVALID_ARG, "request %d label %d is invalid", r, i);
+            if (!in_vocab(q.labels[i], n))
+                return fail(JD_ERR_TOKEN_RANGE, "request %d label %d: token id outside [0, %d)", r, i, opts->vocab);
+            lab.push_back((int32_t)ids.size());
+            lab.push_back(n);
+            ids.insert(ids.end(), q.labels[i], q.labels[i] + n);
+        }
+        if (ids.size() > 0x7fffffffu) return fail(JD_ERR_INVALID_ARG, "requests too large");
+    }
+    const size_t n_req = (size_t)n_requests, n_lab = lab.size() / 2;
+    const int bound = (int)std::max(n_lab / 2, n_req) + 1;  // rows of any round: two candidates or more each
+
+    RouteLayout ly;
+    const size_t o_pool = ly.add((req.size() + lab.size() + ids.size()) * 4);
+    const size_t o_cand0 = ly.add(n_lab * 4), o_cand1 = ly.add(n_lab * 4);
+    const size_t o_nc0 = ly.add(n_req * 4), o_nc1 = ly.add(n_req * 4);
+    const size_t o_rowoff = ly.add((n_req + 1) * 4), o_desc = ly.add((size_t)bound * 12);
+    const size_t o_plan = ly.add((size_t)bound * sizeof(RoutePlan));
+    const size_t o_cu = ly.add(((size_t)bound + 1) * 4), o_opt = ly.add(((size_t)bound + 1) * 4);
+    const size_t o_cnt = ly.add(RC_COUNT * 4);
+    const size_t o_win = ly.add(n_req * 4), o_winp = ly.add(n_req * 4);
+    const size_t o_finc = ly.add(n_req * 20 * 4), o_finp = ly.add(n_req * 20 * 4);
+    CK(cudaSetDevice(m->device));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    m->last_stream = st;
+    if (ly.bytes > m->route_bytes) {
+        CK(cudaStreamSynchronize(st));
+        if (m->route_buf) cudaFree(m->route_buf);
+        m->route_buf = nullptr;
+        m->route_bytes = 0;
+        void *p = nullptr;
+        cudaError_t e = cudaMalloc(&p, ly.bytes);
+        if (e != cudaSuccess) return fail(JD_ERR_CUDA, "router workspace (%zu bytes): %s", ly.bytes, cudaGetErrorString(e));
+        m->route_buf = p;
+        m->route_bytes = ly.bytes;
+    }
+    uint8_t *base = static_cast<uint8_t *>(m->route_buf);
+    auto I = [&](size_t o) { return reinterpret_cast<int *>(base + o); };
+    std::vector<int32_t> pool;
+    pool.reserve(req.size() + lab.size() + ids.size());
+    pool.insert(pool.end(), req.begin(), req.end());
+    pool.insert(pool.end(), lab.begin(), lab.end());
+    pool.insert(pool.end(), ids.begin(), ids.end());
+    CK(cudaMemcpyAsync(base + o_pool, pool.data(), pool.size() * 4, cudaMemcpyHostToDevice, st));
+
+    RouteArgs a;
+    a.n_req = n_requests;
+    a.req = I(o_pool);
+    a.lab = a.req + req.size();
+    a.ids = a.lab + lab.size();
+    a.strict = opts->strict != 0;
+    a.head_budget = opts->head_budget;
+    a.max_length = opts->max_length;
+    a.bos = opts->bos;
+    a.eos = opts->eos;
+    a.mask = opts->mask;
+    int *cand[2] = {I(o_cand0), I(o_cand1)}, *nc[2] = {I(o_nc0), I(o_nc1)};
+    int *cnt = I(o_cnt), *cu = I(o_cu), *opt = I(o_opt), *row_off = I(o_rowoff), *desc = I(o_desc);
+    RoutePlan *plan = reinterpret_cast<RoutePlan *>(base + o_plan);
+    LK(launch_route_init(a, cand[0], nc[0], st));
+
+    int cur = 0, round = 0;
+    bool final_round = false;
+    for (;;) {
+        LK(cudaMemsetAsync(cnt, 0, RC_COUNT * 4, st));
+        LK(launch_route_plan_round(a, cand[cur], nc[cur], final_round ? 1 : 0, bound, row_off, desc, plan, cu, opt,
+                                   cnt, st));
+        CK(cudaMemcpyAsync(m->h_route, cnt, RC_COUNT * 4, cudaMemcpyDeviceToHost, st));
+        CK(cudaMemcpyAsync(m->h_route + RC_COUNT, m->status, 4, cudaMemcpyDeviceToHost, st));
+        CK(cudaStreamSynchronize(st));
+        const int B = m->h_route[RC_ROWS], T = m->h_route[RC_TOKENS], M = m->h_route[RC_MARKERS];
+        const int L = m->h_route[RC_LONGEST], err = m->h_route[RC_ERR];
+        if (m->h_route[RC_COUNT])
+            return fail(JD_ERR_DEVICE_STATUS, "device status 0x%x (1: wait timeout, 2: token id range, 4: index)",
+                        (unsigned)m->h_route[RC_COUNT]);
+        if (err & RE_OPTION_48) return fail(JD_ERR_OVERFLOW, "round %d: an option is longer than 48 tokens", round + 1);
+        if (err & RE_HEAD_BUDGET)
+            return fail(JD_ERR_OVERFLOW, "round %d: question plus options over the head budget %d", round + 1,
+                        opts->head_budget);
+        if (err & RE_MAX_LENGTH) return fail(JD_ERR_OVERFLOW, "round %d: a row is longer than max_length", round + 1);
+        if (B == 0 && !final_round) {
+            final_round = true;
+            continue;
+        }
+        if (B > 0) {
+            if (T > m->cfg.max_tokens || B > m->cfg.max_rows || M > m->cfg.max_markers || L > MAX_POS)
+                return fail(JD_ERR_CAPACITY, "round %d (%d tokens, %d rows, %d markers) exceeds the capacity (%d, %d, %d)",
+                            round + 1, T, B, M, m->cfg.max_tokens, m->cfg.max_rows, m->cfg.max_markers);
+            LK(launch_route_write(a, cand[cur], desc, plan, cu, opt, B, m->d_tokens, m->d_mask, m->d_type, st));
+            jd_batch db{};
+            db.n_rows = B;
+            db.n_tokens = T;
+            db.n_markers = M;
+            db.max_row_len = L;
+            db.tokens = m->d_tokens;
+            db.cu_seqlens = cu;
+            db.mask_pos = m->d_mask;
+            db.opt_off = opt;
+            db.row_type = m->d_type;
+            jd_outputs o{m->i_logits, m->i_probs, m->i_choice, m->i_score, m->i_noul, m->i_maxp};
+            TRY(enqueue_forward(m, &db, &o, nullptr, st));
+            if (out->rows_per_round && round < out->max_rounds) out->rows_per_round[round] = B;
+            ++round;
+        }
+        if (final_round) break;
+        LK(launch_route_survive(a, cand[cur], nc[cur], cand[cur ^ 1], nc[cur ^ 1], row_off, opt, m->i_probs, st));
+        cur ^= 1;
+    }
+    LK(launch_route_final(a, cand[cur], nc[cur], row_off, opt, m->i_probs, I(o_win),
+                          reinterpret_cast<float *>(base + o_winp), I(o_finc), reinterpret_cast<float *>(base + o_finp),
+                          st));
+    std::vector<int32_t> win(n_req), finc(n_req * 20);
+    std::vector<float> winp(n_req), finp(n_req * 20);
+    CK(cudaMemcpyAsync(win.data(), base + o_win, n_req * 4, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(winp.data(), base + o_winp, n_req * 4, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(finc.data(), base + o_finc, n_req * 80, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(finp.data(), base + o_finp, n_req * 80, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(m->h_route + RC_COUNT, m->status, 4, cudaMemcpyDeviceToHost, st));
+    CK(cudaStreamSynchronize(st));
+    if (m->h_route[RC_COUNT])
+        return fail(JD_ERR_DEVICE_STATUS, "device status 0x%x (1: wait timeout, 2: token id range, 4: index)",
+                    (unsigned)m->h_route[RC_COUNT]);
+    std::copy(win.begin(), win.end(), out->winner);
+    if (out->winner_p) std::copy(winp.begin(), winp.end(), out->winner_p);
+    if (out->final_candidates) std::copy(finc.begin(), finc.end(), out->final_candidates);
+    if (out->final_probs) std::copy(finp.begin(), finp.end(), out->final_probs);
+    out->n_rounds = round;
+    return JD_OK;
 }
 
 extern "C" jd_status jd_check_status(jd_model *m) {

@@ -297,6 +297,25 @@ jd_status jd_route_host(jd_model *model, const jd_route_request *requests, int32
                         const jd_encode_opts *opts, int32_t max_tokens, int32_t max_rows, int32_t max_markers,
                         jd_route_outputs *out, void *stream);
 
+/* jd_route_host with the tournament on the device ("Julia-1: one score per
+ * mask token", "More than 20 options: the Router"; no counterpart API on the
+ * pages): the requests are copied to the device once; every round's rows are
+ * then formed, encoded with `opts` (the serializer's layout and budget rules,
+ * strict or not) and packed by kernels, scored by the forward pass, and
+ * narrowed by the same survivor rule, with no host serialisation between
+ * rounds.  Per round the host reads back only the round's row, token and
+ * marker counts and longest row (four ints) to size the next launches; the
+ * outputs come back once at the end.  Outputs equal jd_route_host's on the
+ * same model (no row's result depends on the rest of its batch).
+ * Differences: every id of every request is checked against opts->vocab up
+ * front (JD_ERR_TOKEN_RANGE), and a round must fit the model's capacity in
+ * one batch (JD_ERR_CAPACITY; jd_route_host splits rounds into chunks).
+ * Strict overflow in a round gives JD_ERR_OVERFLOW.  The device workspace
+ * grows on first use (one allocation, kept by the model).  `stream` may be
+ * NULL; the call synchronizes it once per round. */
+jd_status jd_route_device(jd_model *model, const jd_route_request *requests, int32_t n_requests,
+                          const jd_encode_opts *opts, jd_route_outputs *out, void *stream);
+
 /* Scoring callback of jd_route_scored: score n_rows choice rows (host memory,
  * valid during the call) and write the probabilities of every option of every
  * row, in row order, into probs (host memory, one entry per option of the
