@@ -179,6 +179,9 @@ __global__ void __launch_bounds__(256, 1)
 //                  store each (double-buffered); GEGLU outputs go straight
 //                  from registers to global memory.
 constexpr int GEGLU_EW = 8;  // GEGLU epilogue warps (16 measured no faster)
+#ifndef JD_PC_NBUF
+#define JD_PC_NBUF 3
+#endif
 
 template <int BN>
 struct PcCfg {
@@ -188,23 +191,27 @@ struct PcCfg {
     static constexpr int STAGES = 4;
     static constexpr int RING = STAGES * STAGE;
     static constexpr int OUT_BOX = 32 * 128;           // 32 rows x 64 bf16
-    static constexpr int OUT = 4 * 2 * OUT_BOX;        // 4 warps x 2 buffers
+    // staging buffers per epilogue warp: three where the shared memory allows (a 192-wide tile
+    // has three boxes per warp, so none waits on the store of the same tile)
+    static constexpr int NBUF = BN <= 192 ? JD_PC_NBUF : 2;
+    static constexpr int OUT = 4 * NBUF * OUT_BOX;     // 4 warps x NBUF buffers
     static constexpr int DATA = RING + OUT;
     static constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 8;
     static constexpr int SMEM = DATA + BAR_BYTES + 1024;
     static constexpr uint32_t BUF_COLS = 256;          // column stride of the two accumulators
 };
 
-// Per-warp double-buffered staging of 32 x 64 bf16 boxes for TMA stores.
+// Per-warp staging of 32 x 64 bf16 boxes for TMA stores, NB buffers used in turn.
+template <int NB>
 struct OutStage {
-    uint8_t *base;   // this warp's two 4 KB buffers
+    uint8_t *base;   // this warp's NB 4 KB buffers
     uint32_t count;  // boxes issued so far
     __device__ __forceinline__ uint8_t *begin(int lane) {
-        if (count >= 2) {
-            if (lane == 0) bulk_wait_read<1>();  // the store that used this buffer has read it
+        if (count >= NB) {
+            if (lane == 0) bulk_wait_read<NB - 1>();  // the store that used this buffer has read it
             __syncwarp();
         }
-        return base + (count & 1) * 4096;
+        return base + (count % NB) * 4096;
     }
     __device__ __forceinline__ void commit(uint8_t *buf, const CUtensorMap *map, int x, int y, int lane) {
         fence_proxy_async_smem();
@@ -277,7 +284,7 @@ __device__ __forceinline__ void stage_row32(uint8_t *box, int r, int c0, const u
 
 template <int EPI, int BN, int NPART, bool F8 = false>
 __device__ __forceinline__ void pc_epilogue_rows(uint32_t tacc, int r, int row0, int n0, const EpiParams &ep,
-                                                 const CUtensorMap *tmO, OutStage &os, int lane,
+                                                 const CUtensorMap *tmO, OutStage<PcCfg<BN>::NBUF> &os, int lane,
                                                  const float2 (&cs)[32], bool have_cs, int part) {
     if constexpr (EPI == EPI_GEGLU) {
         // stored straight from registers: a shared-memory staging pass here
@@ -497,7 +504,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
     } else {
         const int q = warp & 3;           // TMEM lane quarter of this warp
         const int part = (warp - 2) >> 2;  // which share of the tile's columns (EW / 4 shares)
-        OutStage os{smem + C::RING + ((warp - 2) & 3) * 2 * C::OUT_BOX, 0u};
+        OutStage<C::NBUF> os{smem + C::RING + ((warp - 2) & 3) * C::NBUF * C::OUT_BOX, 0u};
         uint32_t tc = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tc) {
             const int m0 = (t / nblk) * 128, n0 = (t % nblk) * BN;
