@@ -115,6 +115,11 @@ def lib():
     L.jd_decide_host.argtypes = [C.c_void_p, C.POINTER(jd_row), C.c_int32, C.POINTER(jd_encode_opts),
                                  C.POINTER(jd_host_outputs), C.c_void_p]
     L.jd_decide_packed_host.argtypes = [C.c_void_p, C.POINTER(jd_batch), C.POINTER(jd_host_outputs), C.c_void_p]
+    L.jd_decide_host_submit.argtypes = [C.c_void_p, C.POINTER(jd_row), C.c_int32, C.POINTER(jd_encode_opts),
+                                        C.c_void_p, C.POINTER(C.c_int64)]
+    L.jd_decide_host_submit.restype = C.c_int
+    L.jd_decide_host_collect.argtypes = [C.c_void_p, C.c_int64, C.POINTER(jd_host_outputs)]
+    L.jd_decide_host_collect.restype = C.c_int
     L.jd_check_status.argtypes = [C.c_void_p]
     L.jd_set_graph_mode.argtypes = [C.c_void_p, C.c_int]
     L.jd_graph_stats.argtypes = [C.c_void_p, C.POINTER(C.c_int64), C.POINTER(C.c_int64), C.POINTER(C.c_int32)]
@@ -492,6 +497,22 @@ class Model:
         n_m = sum(len(r.options) for r in rows)
         o, s = self._host_out(len(rows), n_m)
         _check(lib().jd_decide_host(self.h, keep.arr, len(rows), C.byref(opts), C.byref(s), _stream(stream)))
+        return o
+
+    def jd_decide_host_submit(self, rows, opts: jd_encode_opts, stream=None):
+        """Queue one host batch (at most two in flight); returns its ticket."""
+        keep = _RowKeep(rows)
+        t = C.c_int64()
+        _check(lib().jd_decide_host_submit(self.h, keep.arr, len(rows), C.byref(opts), _stream(stream), C.byref(t)))
+        self._inflight = getattr(self, "_inflight", {})
+        self._inflight[t.value] = (len(rows), sum(len(r.options) for r in rows))
+        return t.value
+
+    def jd_decide_host_collect(self, ticket):
+        """Outputs of the oldest call in flight (the dict of jd_decide_host)."""
+        n_rows, n_m = self._inflight.pop(ticket)
+        o, s = self._host_out(n_rows, n_m)
+        _check(lib().jd_decide_host_collect(self.h, ticket, C.byref(s)))
         return o
 
     def jd_decide_packed_host(self, hb: HostBatch, stream=None):

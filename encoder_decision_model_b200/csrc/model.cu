@@ -217,9 +217,19 @@ struct jd_model {
     int *i_choice = nullptr;
     int *d_tokens = nullptr, *d_cu = nullptr, *d_mask = nullptr, *d_opt = nullptr, *d_type = nullptr;
     // pinned host staging
-    int *h_tokens = nullptr, *h_cu = nullptr, *h_mask = nullptr, *h_opt = nullptr, *h_type = nullptr;
-    float *h_logits = nullptr, *h_probs = nullptr, *h_score = nullptr, *h_noul = nullptr, *h_maxp = nullptr;
-    int *h_choice = nullptr;
+    // pinned host staging of the host entry points: two slots, so that one call can be prepared
+    // while the previous one runs (jd_decide_host_submit / jd_decide_host_collect); slot 1 is
+    // allocated on first use
+    struct HostSlot {
+        int *h_tokens = nullptr, *h_cu = nullptr, *h_mask = nullptr, *h_opt = nullptr, *h_type = nullptr;
+        float *h_logits = nullptr, *h_probs = nullptr, *h_score = nullptr, *h_noul = nullptr, *h_maxp = nullptr;
+        int *h_choice = nullptr;
+        unsigned *h_status = nullptr;
+        cudaEvent_t done = nullptr;  // recorded after the slot's outputs are copied back
+        int B = 0, M = 0;
+    };
+    HostSlot hs[2];
+    int64_t submitted = 0, collected = 0;
 
     cudaStream_t last_stream = nullptr;
 
@@ -469,6 +479,24 @@ jd_status load_weights(jd_model *m, const char *path) {
     return JD_OK;
 }
 
+jd_status alloc_host_slot(jd_model *m, jd_model::HostSlot &h) {
+    const size_t T = m->T_cap, M = m->M_cap, B = m->B_cap;
+    TRY(m->halloc(&h.h_tokens, T));
+    TRY(m->halloc(&h.h_cu, B + 1));
+    TRY(m->halloc(&h.h_mask, M));
+    TRY(m->halloc(&h.h_opt, B + 1));
+    TRY(m->halloc(&h.h_type, B));
+    TRY(m->halloc(&h.h_logits, M));
+    TRY(m->halloc(&h.h_probs, M));
+    TRY(m->halloc(&h.h_choice, B));
+    TRY(m->halloc(&h.h_score, B));
+    TRY(m->halloc(&h.h_noul, B));
+    TRY(m->halloc(&h.h_maxp, B));
+    TRY(m->halloc(&h.h_status, 1));
+    CK(cudaEventCreateWithFlags(&h.done, cudaEventDisableTiming));
+    return JD_OK;
+}
+
 jd_status alloc_workspace(jd_model *m) {
     const size_t T = m->T_cap, M = m->M_cap, B = m->B_cap;
     const size_t es = m->fp32 ? 4 : 2;
@@ -505,17 +533,7 @@ jd_status alloc_workspace(jd_model *m) {
     TRY(m->dalloc(&m->d_mask, M));
     TRY(m->dalloc(&m->d_opt, B + 1));
     TRY(m->dalloc(&m->d_type, B));
-    TRY(m->halloc(&m->h_tokens, T));
-    TRY(m->halloc(&m->h_cu, B + 1));
-    TRY(m->halloc(&m->h_mask, M));
-    TRY(m->halloc(&m->h_opt, B + 1));
-    TRY(m->halloc(&m->h_type, B));
-    TRY(m->halloc(&m->h_logits, M));
-    TRY(m->halloc(&m->h_probs, M));
-    TRY(m->halloc(&m->h_choice, B));
-    TRY(m->halloc(&m->h_score, B));
-    TRY(m->halloc(&m->h_noul, B));
-    TRY(m->halloc(&m->h_maxp, B));
+    TRY(alloc_host_slot(m, m->hs[0]));
     TRY(m->halloc(&m->h_route, 16));
     if (!m->fp32) {
         TRY(make_map(&m->tm_xn, m->xn, D, T, D, 64, 128));
@@ -973,6 +991,8 @@ extern "C" void jd_model_destroy(jd_model *m) {
     if (!m) return;
     cudaSetDevice(m->device);
     if (m->gexec) cudaGraphExecDestroy(m->gexec);
+    for (auto &h : m->hs)
+        if (h.done) cudaEventDestroy(h.done);
     for (auto &kv : m->gbuckets) cudaGraphExecDestroy(kv.second.exec);
     for (cudaEvent_t e : m->ev) cudaEventDestroy(e);
     for (void *p : m->allocs) cudaFree(p);
@@ -1061,12 +1081,11 @@ extern "C" jd_status jd_forward(jd_model *m, const jd_batch *b, float *logits, v
     return jd_decide(m, b, &o, nullptr, stream);
 }
 
-extern "C" jd_status jd_decide_packed_host(jd_model *m, const jd_batch *hb, jd_host_outputs *ho, void *stream) {
-    clear_error();
-    if (!m || !hb || !ho) return fail(JD_ERR_INVALID_ARG, "NULL argument");
-    TRY(check_batch(m, hb));
-    CK(cudaSetDevice(m->device));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
+namespace {
+
+// Queue one host batch on `st` through the pinned slot h: copies in, forward pass (a bucket's
+// graph in graph mode), outputs and the status word copied back, h.done recorded.
+jd_status host_enqueue(jd_model *m, const jd_batch *hb, jd_model::HostSlot &h, cudaStream_t st) {
     const int T = hb->n_tokens, B = hb->n_rows, M = hb->n_markers;
     // graph mode: the batch padded to its bucket on the host, so that its graph reads it from the
     // staging arrays and writes the internal outputs directly
@@ -1074,23 +1093,23 @@ extern "C" jd_status jd_decide_packed_host(jd_model *m, const jd_batch *hb, jd_h
     int Lb = 0;
     const bool bucket = m->graph_mode && !m->prof && graph_bucket(m, hb, &ps, &Lb);
     if (!bucket) ps = PadShape{T, B, M, T, B, M};
-    memcpy(m->h_tokens, hb->tokens, sizeof(int) * T);
-    memcpy(m->h_cu, hb->cu_seqlens, sizeof(int) * (B + 1));
-    memcpy(m->h_mask, hb->mask_pos, sizeof(int) * M);
-    memcpy(m->h_opt, hb->opt_off, sizeof(int) * (B + 1));
-    memcpy(m->h_type, hb->row_type, sizeof(int) * B);
-    for (int i = T; i < ps.Tb; ++i) m->h_tokens[i] = pad_token_at(ps, hb->tokens, i);
+    memcpy(h.h_tokens, hb->tokens, sizeof(int) * T);
+    memcpy(h.h_cu, hb->cu_seqlens, sizeof(int) * (B + 1));
+    memcpy(h.h_mask, hb->mask_pos, sizeof(int) * M);
+    memcpy(h.h_opt, hb->opt_off, sizeof(int) * (B + 1));
+    memcpy(h.h_type, hb->row_type, sizeof(int) * B);
+    for (int i = T; i < ps.Tb; ++i) h.h_tokens[i] = pad_token_at(ps, hb->tokens, i);
     for (int i = B + 1; i <= ps.Bb; ++i) {
-        m->h_cu[i] = pad_cu_at(ps, hb->cu_seqlens, i);
-        m->h_opt[i] = pad_opt_at(ps, hb->opt_off, i);
+        h.h_cu[i] = pad_cu_at(ps, hb->cu_seqlens, i);
+        h.h_opt[i] = pad_opt_at(ps, hb->opt_off, i);
     }
-    for (int i = M; i < ps.Mb; ++i) m->h_mask[i] = pad_mask_at(ps, hb->mask_pos, i);
-    for (int i = B; i < ps.Bb; ++i) m->h_type[i] = pad_type_at(ps, hb->row_type, i);
-    CK(cudaMemcpyAsync(m->d_tokens, m->h_tokens, sizeof(int) * ps.Tb, cudaMemcpyHostToDevice, st));
-    CK(cudaMemcpyAsync(m->d_cu, m->h_cu, sizeof(int) * (ps.Bb + 1), cudaMemcpyHostToDevice, st));
-    CK(cudaMemcpyAsync(m->d_mask, m->h_mask, sizeof(int) * ps.Mb, cudaMemcpyHostToDevice, st));
-    CK(cudaMemcpyAsync(m->d_opt, m->h_opt, sizeof(int) * (ps.Bb + 1), cudaMemcpyHostToDevice, st));
-    CK(cudaMemcpyAsync(m->d_type, m->h_type, sizeof(int) * ps.Bb, cudaMemcpyHostToDevice, st));
+    for (int i = M; i < ps.Mb; ++i) h.h_mask[i] = pad_mask_at(ps, hb->mask_pos, i);
+    for (int i = B; i < ps.Bb; ++i) h.h_type[i] = pad_type_at(ps, hb->row_type, i);
+    CK(cudaMemcpyAsync(m->d_tokens, h.h_tokens, sizeof(int) * ps.Tb, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_cu, h.h_cu, sizeof(int) * (ps.Bb + 1), cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_mask, h.h_mask, sizeof(int) * ps.Mb, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_opt, h.h_opt, sizeof(int) * (ps.Bb + 1), cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(m->d_type, h.h_type, sizeof(int) * ps.Bb, cudaMemcpyHostToDevice, st));
     if (bucket) {
         m->last_stream = st;
         TRY(bucket_replay(m, ps, Lb, st));
@@ -1104,27 +1123,82 @@ extern "C" jd_status jd_decide_packed_host(jd_model *m, const jd_batch *hb, jd_h
         db.head_len = nullptr;
         db.trunc = nullptr;
         jd_outputs o{m->i_logits, m->i_probs, m->i_choice, m->i_score, m->i_noul, m->i_maxp};
-        TRY(jd_decide(m, &db, &o, nullptr, stream));
+        TRY(jd_decide(m, &db, &o, nullptr, st));
     }
-    CK(cudaMemcpyAsync(m->h_logits, m->i_logits, sizeof(float) * M, cudaMemcpyDeviceToHost, st));
-    CK(cudaMemcpyAsync(m->h_probs, m->i_probs, sizeof(float) * M, cudaMemcpyDeviceToHost, st));
-    CK(cudaMemcpyAsync(m->h_choice, m->i_choice, sizeof(int) * B, cudaMemcpyDeviceToHost, st));
-    CK(cudaMemcpyAsync(m->h_score, m->i_score, sizeof(float) * B, cudaMemcpyDeviceToHost, st));
-    CK(cudaMemcpyAsync(m->h_noul, m->i_noul, sizeof(float) * B, cudaMemcpyDeviceToHost, st));
-    CK(cudaMemcpyAsync(m->h_maxp, m->i_maxp, sizeof(float) * B, cudaMemcpyDeviceToHost, st));
-    CK(cudaStreamSynchronize(st));
-    unsigned stv = 0;
-    CK(cudaMemcpy(&stv, m->status, sizeof(unsigned), cudaMemcpyDeviceToHost));
-    if (stv) return fail(JD_ERR_DEVICE_STATUS, "device status 0x%x (1: wait timeout, 2: token id range, 4: index)", stv);
-    if (ho->logits) memcpy(ho->logits, m->h_logits, sizeof(float) * M);
-    if (ho->probs) memcpy(ho->probs, m->h_probs, sizeof(float) * M);
-    if (ho->choice) memcpy(ho->choice, m->h_choice, sizeof(int) * B);
-    if (ho->score) memcpy(ho->score, m->h_score, sizeof(float) * B);
-    if (ho->noul) memcpy(ho->noul, m->h_noul, sizeof(float) * B);
-    if (ho->max_p) memcpy(ho->max_p, m->h_maxp, sizeof(float) * B);
+    CK(cudaMemcpyAsync(h.h_logits, m->i_logits, sizeof(float) * M, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(h.h_probs, m->i_probs, sizeof(float) * M, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(h.h_choice, m->i_choice, sizeof(int) * B, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(h.h_score, m->i_score, sizeof(float) * B, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(h.h_noul, m->i_noul, sizeof(float) * B, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(h.h_maxp, m->i_maxp, sizeof(float) * B, cudaMemcpyDeviceToHost, st));
+    CK(cudaMemcpyAsync(h.h_status, m->status, sizeof(unsigned), cudaMemcpyDeviceToHost, st));
+    CK(cudaEventRecord(h.done, st));
+    h.B = B;
+    h.M = M;
+    return JD_OK;
+}
+
+// Wait for slot h's call and copy its outputs out (its own copy of the status word decides).
+jd_status host_finish(jd_model::HostSlot &h, jd_host_outputs *ho) {
+    CK(cudaEventSynchronize(h.done));
+    const int B = h.B, M = h.M;
+    if (*h.h_status)
+        return fail(JD_ERR_DEVICE_STATUS, "device status 0x%x (1: wait timeout, 2: token id range, 4: index)",
+                    *h.h_status);
+    if (ho->logits) memcpy(ho->logits, h.h_logits, sizeof(float) * M);
+    if (ho->probs) memcpy(ho->probs, h.h_probs, sizeof(float) * M);
+    if (ho->choice) memcpy(ho->choice, h.h_choice, sizeof(int) * B);
+    if (ho->score) memcpy(ho->score, h.h_score, sizeof(float) * B);
+    if (ho->noul) memcpy(ho->noul, h.h_noul, sizeof(float) * B);
+    if (ho->max_p) memcpy(ho->max_p, h.h_maxp, sizeof(float) * B);
     ho->n_rows = B;
     ho->n_markers = M;
     return JD_OK;
+}
+
+}  // namespace
+
+extern "C" jd_status jd_decide_packed_host(jd_model *m, const jd_batch *hb, jd_host_outputs *ho, void *stream) {
+    clear_error();
+    if (!m || !hb || !ho) return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    TRY(check_batch(m, hb));
+    if (m->submitted != m->collected)
+        return fail(JD_ERR_INVALID_ARG, "collect the submitted calls (jd_decide_host_collect) first");
+    CK(cudaSetDevice(m->device));
+    TRY(host_enqueue(m, hb, m->hs[0], static_cast<cudaStream_t>(stream)));
+    return host_finish(m->hs[0], ho);
+}
+
+extern "C" jd_status jd_decide_host_submit(jd_model *m, const jd_row *rows, int32_t n_rows, const jd_encode_opts *opts,
+                                           void *stream, int64_t *ticket) {
+    clear_error();
+    if (!m || !ticket) return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    if (m->submitted - m->collected >= 2)
+        return fail(JD_ERR_INVALID_ARG, "two calls in flight: collect one (jd_decide_host_collect) first");
+    CK(cudaSetDevice(m->device));
+    jd_model::HostSlot &h = m->hs[m->submitted % 2];
+    if (!h.h_tokens) TRY(alloc_host_slot(m, h));
+    jd_batch *hb = nullptr;
+    int32_t bad = -1;
+    jd_status s = jd_serialize(rows, n_rows, opts, &hb, &bad);
+    if (s != JD_OK) return s;
+    s = check_batch(m, hb);
+    if (s == JD_OK) s = host_enqueue(m, hb, h, static_cast<cudaStream_t>(stream));
+    jd_batch_free(hb);
+    if (s != JD_OK) return s;
+    *ticket = m->submitted++;
+    return JD_OK;
+}
+
+extern "C" jd_status jd_decide_host_collect(jd_model *m, int64_t ticket, jd_host_outputs *ho) {
+    clear_error();
+    if (!m || !ho) return fail(JD_ERR_INVALID_ARG, "NULL argument");
+    if (ticket != m->collected || m->collected >= m->submitted)
+        return fail(JD_ERR_INVALID_ARG, "ticket %lld is not the oldest call in flight", (long long)ticket);
+    CK(cudaSetDevice(m->device));
+    jd_status s = host_finish(m->hs[ticket % 2], ho);
+    ++m->collected;  // a failed call is collected too: its slot is free again
+    return s;
 }
 
 extern "C" jd_status jd_decide_host(jd_model *m, const jd_row *rows, int32_t n_rows, const jd_encode_opts *opts,

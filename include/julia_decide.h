@@ -258,9 +258,26 @@ typedef struct {
 jd_status jd_decide_host(jd_model *model, const jd_row *rows, int32_t n_rows,
                          const jd_encode_opts *opts, jd_host_outputs *out, void *stream);
 
-/* Same as jd_decide_host, starting from an already serialized host batch. */
+/* Same as jd_decide_host, starting from an already serialized host batch.
+ * JD_ERR_INVALID_ARG while calls of jd_decide_host_submit are uncollected. */
 jd_status jd_decide_packed_host(jd_model *model, const jd_batch *host_batch,
                                 jd_host_outputs *out, void *stream);
+
+/* jd_decide_host in two halves, so that the host prepares one call while the
+ * device runs the previous one (the serving loop of a stream of batches):
+ * submit serialises the rows, queues the copies in, the forward pass and the
+ * copies back on `stream` through one of two pinned staging slots (the second
+ * is allocated on first use), and returns at once with a ticket (0, 1, 2 ...
+ * per handle); collect waits for the oldest call in flight and copies its
+ * outputs into `out` (host memory; the same outputs as jd_decide_host, and
+ * JD_ERR_DEVICE_STATUS if that call's kernels recorded a failure).  At most
+ * two calls are in flight (a third submit gives JD_ERR_INVALID_ARG), tickets
+ * are collected in order, and the synchronous host calls refuse to run while
+ * any is in flight.  The rows need not outlive submit.  Both calls of a
+ * handle come from one host thread at a time. */
+jd_status jd_decide_host_submit(jd_model *model, const jd_row *rows, int32_t n_rows,
+                                const jd_encode_opts *opts, void *stream, int64_t *ticket);
+jd_status jd_decide_host_collect(jd_model *model, int64_t ticket, jd_host_outputs *out);
 
 /* A choice question over up to 4096 candidate labels (host memory). */
 typedef struct {
