@@ -1222,7 +1222,7 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], 4);
-            mbar_init(&momf[b], NS * 128);  // one arrival per epilogue thread of every CTA
+            mbar_init(&momf[b], 1);  // the leader's arrival with the tile's expected moment bytes
         }
         for (int b = 0; b < C::NXB; ++b) mbar_init(&xfull[b], 1);
         fence_barrier_init();
@@ -1306,6 +1306,8 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
             mbar_wait(&accf[b], (tc >> 1) & 1, ep.status);
             __syncwarp();
             tc_fence_after();
+            // the moments of this tile arrive as NS x NX x 128 asynchronous 8-byte stores
+            if (leader) mbar_arrive_expect_tx(&momf[b], NS * C::NX * 128 * 8);
             // ---- pass 1: v = x + acc (+ bias) for this CTA's columns; each 32-column chunk's
             //      (mean, M2) goes to slot [tile parity][global chunk][row] of both CTAs
 #pragma unroll 1
@@ -1335,13 +1337,20 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) cq += (v[j] - cm) * (v[j] - cm);
                 {
+                    // asynchronous stores that complete their bytes on the receiving CTA's moment
+                    // barrier: no release of this thread's other (global) stores is waited for
                     const uint32_t local = smem_u32(&mom[((int)b * 12 + (int)rank * C::NX + c) * 128 + r]);
+                    const uint32_t lbar = smem_u32(&momf[b]);
 #pragma unroll
                     for (int j = 0; j < NS; ++j) {
-                        uint32_t remote;
+                        uint32_t remote, rbar;
                         asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(j));
-                        asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(cm), "f"(cq)
-                                     : "memory");
+                        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(lbar), "r"(j));
+                        asm volatile(
+                            "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+                                remote),
+                            "f"(cm), "f"(cq), "r"(rbar)
+                            : "memory");
                     }
                 }
 #pragma unroll
@@ -1372,9 +1381,6 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
                 }
             }
             tmem_st_wait();
-            // each thread releases its own stores with its arrivals on both CTAs' barriers
-#pragma unroll
-            for (int j = 0; j < NS; ++j) mbar_arrive_remote(&momf[b], (uint32_t)j);
             mbar_wait_cluster(&momf[b], (tc >> 1) & 1, ep.status);
             // ---- the twelve chunks' moments merged in column order with k_gemm_rl's update, so the
             //      row's mean and M2 -- and the outputs -- are bit-identical to the unsplit kernel's
