@@ -862,6 +862,41 @@ __global__ void __launch_bounds__(192, 1)
     }
 }
 
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (the arrivals come from the other CTAs of the cluster).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, unsigned *status) {
+    const uint32_t addr = smem_u32(bar);
+    uint64_t t0 = 0;
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_cluster(addr, parity)) return true;
+        if ((it & 255u) == 0) {
+            if (status && (*reinterpret_cast<volatile unsigned *>(status) & ST_WAIT_TIMEOUT)) return false;
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > 2000000000ull) {
+                if (status) atomicOr(status, ST_WAIT_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+// Arrive on the barrier at the address of `local_bar` in CTA `rank` of this cluster.
+__device__ __forceinline__ void mbar_arrive_remote(const uint64_t *local_bar, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local_bar)), "r"(rank));
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+}
+
 // ---------------------------------------------------------------- residual + LayerNorm GEMM, split over a cluster
 //
 // For batches of a few row tiles (a single request of some hundred tokens makes
@@ -892,7 +927,7 @@ struct RsCfg {
     static constexpr int NX = NC / 32;
     static constexpr int MOM = 12 * 128 * 8;     // (mean, M2) of every row's twelve 32-column chunks
     static constexpr int DATA = RING + NX * XCH + MOM;
-    static constexpr int BAR_BYTES = (2 * STAGES + 1 + NX) * 8 + 8;
+    static constexpr int BAR_BYTES = (2 * STAGES + 2 + NX) * 8 + 8;
     static constexpr int SMEM = DATA + BAR_BYTES + 1024;
     static constexpr uint32_t TMEM_COLS = NC <= 64 ? 64 : (NC <= 128 ? 128 : 256);
     static_assert(NC % 64 == 0 && NC <= 256, "column share: whole 64-row W boxes");
@@ -921,7 +956,8 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
     uint64_t *empty = full + C::STAGES;
     uint64_t *accf = empty + C::STAGES;
     uint64_t *xfull = accf + 1;  // [NX]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xfull + C::NX);
+    uint64_t *momf = xfull + C::NX;  // every CTA's moments of this CTA's rows have arrived
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(momf + 1);
 
     const uint32_t rank = rs_cluster_rank();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -936,6 +972,7 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
         }
         mbar_init(accf, 1);
         for (int c = 0; c < C::NX; ++c) mbar_init(&xfull[c], 1);
+        mbar_init(momf, 1);  // one arrival with the expected moment bytes
         fence_barrier_init();
         fence_proxy_async_smem();
         prefetch_tmap(&tmA);
@@ -948,6 +985,7 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
     }
     tc_fence_before();
     __syncthreads();
+    rs_cluster_sync();  // every CTA's moment barrier exists before the first remote store
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const bool leader = threadIdx.x == 64;
@@ -993,6 +1031,7 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     float mean = 0.f, m2 = 0.f;
     if (warp >= 2) {
+        if (leader) mbar_arrive_expect_tx(momf, NS * C::NX * 128 * 8);
         mbar_wait(accf, 0, ep.status);
         __syncwarp();
         tc_fence_after();
@@ -1024,12 +1063,18 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) cq += (v[j] - cm) * (v[j] - cm);
             {
+                // asynchronous stores that complete their bytes on each receiving CTA's moment barrier
                 const uint32_t local = smem_u32(&mom[((int)rank * C::NX + c) * 128 + r]);
+                const uint32_t lbar = smem_u32(momf);
 #pragma unroll
                 for (int j = 0; j < NS; ++j) {
-                    uint32_t remote;
+                    uint32_t remote, rbar;
                     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(j));
-                    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(cm), "f"(cq) : "memory");
+                    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(lbar), "r"(j));
+                    asm volatile(
+                        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(remote),
+                        "f"(cm), "f"(cq), "r"(rbar)
+                        : "memory");
                 }
             }
 #pragma unroll
@@ -1048,9 +1093,9 @@ __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
             }
         }
         tmem_st_wait();
+        // every CTA's moments of these rows; a CTA leaves only after all stores into it landed
+        mbar_wait_cluster(momf, 0, ep.status);
     }
-    __syncwarp();
-    rs_cluster_sync();
     if (warp >= 2) {
         // ---- the twelve chunks' moments merged in column order with k_gemm_rl's update, so the
         //      row's mean and M2 -- and the outputs -- are bit-identical to the unsplit kernel's
@@ -1155,41 +1200,6 @@ struct RpCfg {
     static constexpr uint32_t ACC_STRIDE = 256;    // TMEM columns between the two accumulators
     static_assert(NC % 32 == 0 && NC <= 256 && SMEM <= 227 * 1024, "persistent split residual GEMM");
 };
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t addr, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait with cluster-scope acquire (the arrivals come from the other CTAs of the cluster).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, unsigned *status) {
-    const uint32_t addr = smem_u32(bar);
-    uint64_t t0 = 0;
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait_cluster(addr, parity)) return true;
-        if ((it & 255u) == 0) {
-            if (status && (*reinterpret_cast<volatile unsigned *>(status) & ST_WAIT_TIMEOUT)) return false;
-            const uint64_t now = globaltimer_ns();
-            if (t0 == 0) t0 = now;
-            else if (now - t0 > 2000000000ull) {
-                if (status) atomicOr(status, ST_WAIT_TIMEOUT);
-                return false;
-            }
-        }
-    }
-}
-// Arrive on the barrier at the address of `local_bar` in CTA `rank` of this cluster.
-__device__ __forceinline__ void mbar_arrive_remote(const uint64_t *local_bar, uint32_t rank) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local_bar)), "r"(rank));
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
-}
 
 template <int NS, bool OUT8>
 __global__ void __cluster_dims__(NS, 1, 1) __launch_bounds__(192, 1)
