@@ -343,11 +343,11 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     for (int e = 0; e < TK; ++e)
                         if (k0 + e >= t.ce) sv[e] = __float_as_uint(-INFINITY);
                 }
-                float m4[4];
+                float m4[4];  // four independent chains over keys 8 i + 2 a, 8 i + 2 a + 1
 #pragma unroll
-                for (int e = 0; e < 4; ++e) m4[e] = __uint_as_float(sv[e]);
+                for (int a = 0; a < 4; ++a) m4[a] = fmaxf(__uint_as_float(sv[2 * a]), __uint_as_float(sv[2 * a + 1]));
 #pragma unroll
-                for (int e = 4; e < TK; e += 8)
+                for (int e = 8; e < TK; e += 8)
 #pragma unroll
                     for (int a = 0; a < 4; ++a)
                         m4[a] = fmax3(m4[a], __uint_as_float(sv[e + 2 * a]), __uint_as_float(sv[e + 2 * a + 1]));
