@@ -56,7 +56,7 @@ constexpr uint32_t T_S = 0, T_O = 256, T_P = 384;
 constexpr float kLazy = 8.0f;    // log2 headroom before the running max is moved
 constexpr int V_WARP = 10;
 constexpr int ATC_THREADS = 11 * 32;
-constexpr int BAR_G0_DONE = 1, BAR_G1_DONE = 2, BAR_ITEM = 3;  // named barriers of the softmax groups
+constexpr int BAR_G0_DONE = 1, BAR_G1_DONE = 2;  // named barriers of the softmax groups' hand-off
 }  // namespace
 
 // max(a, b, c) in one instruction
@@ -237,29 +237,38 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             uint32_t J = 0, it = 0;
             uint32_t cnt[2] = {0, 0};   // S tiles issued per Q tile, over all items
             uint32_t uses[2] = {0, 0};  // items that used each Q tile
+            // O_x += P_x V for the K tile at ring position Jp: cx[x] is that tile's S count of Q tile
+            // x, `first` marks an item's first tile (O_x overwritten once the last item's O_x is read
+            // out: us[x] items had used it before)
+            auto issue_pv = [&](uint32_t Jp, int nx, const uint32_t (&cx)[2], bool first, const uint32_t (&us)[2]) {
+                const uint32_t s = Jp % NV;
+                mbar_wait(&vfull[s], (Jp / NV) & 1, status);
+                const uint32_t v_base = smem_u32(smem + OFF_V + s * KT_BYTES);
+                for (int x = 0; x < nx; ++x) {
+                    mbar_wait(&pready[x], cx[x] & 1, status);
+                    if (first && us[x] >= 1) mbar_wait(&ofree[x], (us[x] - 1) & 1, status);
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < TK / 16; ++ks)
+                        tc_mma_bf16_ts(tmem + T_O + 64 * x, tmem + T_P + 64 * x + 8 * ks,
+                                       sdesc_sw128(v_base + ks * 16 * 128), idesc_pv, (!first || ks != 0) ? 1u : 0u);
+                    tc_commit(&pvdone[x]);
+                }
+                tc_commit(&vfree[s]);
+            };
+            // The PV products of an item's last K tile are issued after the next item's first S
+            // products, so that the softmax groups find their next S tile ready when they finish
+            // the item, instead of after both groups' last exponentials.
+            bool pend = false;
+            uint32_t pJ = 0, pc[2] = {0, 0}, pu[2] = {0, 0};
+            int pnx = 0;
+            bool pfirst = false;
             for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++it) {
                 const AtcItem t = atc_item(q256, pb_row, cu, w);
                 const uint32_t qbuf = it & 1;
                 mbar_wait(&qfull[qbuf], (it >> 1) & 1, status);
                 tc_fence_after();
-                const uint32_t J0 = J, c0[2] = {cnt[0], cnt[1]};
-                auto issue_pv = [&](int j) {
-                    const uint32_t Jp = J0 + j, s = Jp % NV;
-                    mbar_wait(&vfull[s], (Jp / NV) & 1, status);
-                    const uint32_t v_base = smem_u32(smem + OFF_V + s * KT_BYTES);
-                    for (int x = 0; x < t.nx; ++x) {
-                        const uint32_t c = c0[x] + j;
-                        mbar_wait(&pready[x], c & 1, status);
-                        if (j == 0 && uses[x] >= 1) mbar_wait(&ofree[x], (uses[x] - 1) & 1, status);
-                        tc_fence_after();
-#pragma unroll
-                        for (int ks = 0; ks < TK / 16; ++ks)
-                            tc_mma_bf16_ts(tmem + T_O + 64 * x, tmem + T_P + 64 * x + 8 * ks,
-                                           sdesc_sw128(v_base + ks * 16 * 128), idesc_pv, (j != 0 || ks != 0) ? 1u : 0u);
-                        tc_commit(&pvdone[x]);
-                    }
-                    tc_commit(&vfree[s]);
-                };
+                const uint32_t J0 = J, c0[2] = {cnt[0], cnt[1]}, u0[2] = {uses[0], uses[1]};
                 for (int j = 0; j < t.nt; ++j, ++J) {
                     const uint32_t s = J % NK;
                     mbar_wait(&kfull[s], (J / NK) & 1, status);
@@ -277,11 +286,26 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     }
                     tc_commit(&kfree[s]);
                     if (j == t.nt - 1) tc_commit(&qfree[qbuf]);
-                    if (j >= 1) issue_pv(j - 1);
+                    if (j == 0 && pend) {
+                        issue_pv(pJ, pnx, pc, pfirst, pu);
+                        pend = false;
+                    }
+                    if (j >= 1) {
+                        const uint32_t cx[2] = {c0[0] + j - 1, c0[1] + j - 1};
+                        issue_pv(J0 + j - 1, t.nx, cx, j == 1, u0);
+                    }
                 }
-                issue_pv(t.nt - 1);
+                pend = true;
+                pJ = J0 + t.nt - 1;
+                pnx = t.nx;
+                pc[0] = c0[0] + t.nt - 1;
+                pc[1] = c0[1] + t.nt - 1;
+                pfirst = t.nt == 1;
+                pu[0] = u0[0];
+                pu[1] = u0[1];
                 for (int x = 0; x < t.nx; ++x) ++uses[x];
             }
+            if (pend) issue_pv(pJ, pnx, pc, pfirst, pu);
         }
     } else {
         const int x = (warp - 2) >> 2;         // Q tile of this warp group
@@ -289,12 +313,20 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float sl2 = 0.125f * 1.4426950408889634f;
         uint32_t c = 0;
+        bool prev_pp = false;  // the CTA's previous item had two Q tiles
         for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
             const AtcItem t = atc_item(q256, pb_row, cu, w);
-            if (x >= t.nx) continue;
-            const int qi = t.q0 + x * TQ + r;
             const bool pp = t.nx == 2;  // both groups busy: alternate the exponential phases
-            if (pp) named_bar_sync(BAR_ITEM, 256);
+            // The hand-off runs on from one two-tile item into the next: group 0 starts an item's
+            // exponentials after group 1's last ones of the previous item, group 1 hands over its
+            // last tile only when the next item has two tiles too.  Either way every arrival on a
+            // hand-off barrier meets exactly one wait.
+            const bool g0_wait_first = pp && prev_pp;
+            prev_pp = pp;
+            if (x >= t.nx) continue;
+            const bool g1_hand_last =
+                pp && x == 1 && w + (int)gridDim.x < n_items && atc_item(q256, pb_row, cu, w + gridDim.x).nx == 2;
+            const int qi = t.q0 + x * TQ + r;
             // A warp whose 32 query rows all lie past the row's end (the tail of a short row's
             // last tile) reads nothing of S, P or O: it keeps every wait and arrival of the
             // pipeline, so the barrier phases stay those of the other warps, and skips the math.
@@ -305,7 +337,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     if (lane == 0) mbar_arrive(&sfree[x]);
                     if (pp) {
                         if (x == 0) {
-                            if (j != 0) named_bar_sync(BAR_G1_DONE, 256);
+                            if (j != 0 || g0_wait_first) named_bar_sync(BAR_G1_DONE, 256);
                         } else {
                             named_bar_sync(BAR_G0_DONE, 256);
                         }
@@ -313,7 +345,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     if (j != 0) mbar_wait(&pvdone[x], (c - 1) & 1, status);
                     if (pp) {
                         if (x == 0) named_bar_arrive(BAR_G0_DONE, 256);
-                        else if (j != t.nt - 1) named_bar_arrive(BAR_G1_DONE, 256);
+                        else if (j != t.nt - 1 || g1_hand_last) named_bar_arrive(BAR_G1_DONE, 256);
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pready[x]);
@@ -374,7 +406,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                 }
                 if (pp) {
                     if (x == 0) {
-                        if (j != 0) named_bar_sync(BAR_G1_DONE, 256);
+                        if (j != 0 || g0_wait_first) named_bar_sync(BAR_G1_DONE, 256);
                     } else {
                         named_bar_sync(BAR_G0_DONE, 256);
                     }
@@ -409,7 +441,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                 }
                 if (pp) {
                     if (x == 0) named_bar_arrive(BAR_G0_DONE, 256);
-                    else if (j != t.nt - 1) named_bar_arrive(BAR_G1_DONE, 256);
+                    else if (j != t.nt - 1 || g1_hand_last) named_bar_arrive(BAR_G1_DONE, 256);
                 }
                 l += ((ls[0].x + ls[0].y) + (ls[1].x + ls[1].y)) + ((ls[2].x + ls[2].y) + (ls[3].x + ls[3].y));
                 tmem_st_wait();
