@@ -314,6 +314,39 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         const float sl2 = 0.125f * 1.4426950408889634f;
         uint32_t c = 0;
         bool prev_pp = false;  // the CTA's previous item had two Q tiles
+        // An item's O_x is read out once its last PV product has landed, which this thread waits
+        // for anyway before storing the next item's first P tile: the readout follows that store,
+        // so the wait for the last product hides behind the next item's first exponentials.
+        // rd_dst: the pending row's output (null for a row past the end)
+        bool rd_pend = false;
+        __nv_bfloat16 *rd_dst = nullptr;
+        float rd_inv = 0.f;
+        auto readout = [&]() {
+            __syncwarp();
+            tc_fence_after();
+#pragma unroll 1
+            for (int hc = 0; hc < 64; hc += 32) {
+                uint32_t o[32];
+                tmem_ld32(tl + T_O + 64 * x + hc, o);
+                tmem_ld_wait();
+                if (rd_dst) {  // 32-byte stores: a warp instruction fills whole sectors
+                    uint8_t *dst = reinterpret_cast<uint8_t *>(rd_dst + hc);
+#pragma unroll
+                    for (int k8 = 0; k8 < 2; ++k8) {
+                        uint32_t wv[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            wv[e] = pack_bf16x2(__uint_as_float(o[16 * k8 + 2 * e]) * rd_inv,
+                                                __uint_as_float(o[16 * k8 + 2 * e + 1]) * rd_inv);
+                        st_global_v8(dst + 32 * k8, wv[0], wv[1], wv[2], wv[3], wv[4], wv[5], wv[6], wv[7]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ofree[x]);
+            rd_pend = false;
+        };
         for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
             const AtcItem t = atc_item(q256, pb_row, cu, w);
             const bool pp = t.nx == 2;  // both groups busy: alternate the exponential phases
@@ -331,6 +364,10 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             // last tile) reads nothing of S, P or O: it keeps every wait and arrival of the
             // pipeline, so the barrier phases stay those of the other warps, and skips the math.
             if (t.q0 + x * TQ + (warp & 3) * 32 >= t.ce) {
+                if (rd_pend) {
+                    mbar_wait(&pvdone[x], (c - 1) & 1, status);
+                    readout();
+                }
                 for (int j = 0; j < t.nt; ++j, ++c) {
                     mbar_wait(&sfull[x], c & 1, status);
                     __syncwarp();
@@ -433,7 +470,8 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                         pk[e >> 1] = pack_f16x2(p0, p1);
                     }
                     if (hk == 0) {
-                        if (j != 0) mbar_wait(&pvdone[x], (c - 1) & 1, status);  // P_x consumed by the last product
+                        // P_x consumed by the last product (the previous item's, then also its O_x final)
+                        if (j != 0 || rd_pend) mbar_wait(&pvdone[x], (c - 1) & 1, status);
                         __syncwarp();
                         tc_fence_after();
                     }
@@ -444,35 +482,20 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     else if (j != t.nt - 1 || g1_hand_last) named_bar_arrive(BAR_G1_DONE, 256);
                 }
                 l += ((ls[0].x + ls[0].y) + (ls[1].x + ls[1].y)) + ((ls[2].x + ls[2].y) + (ls[3].x + ls[3].y));
+                if (rd_pend) readout();
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&pready[x]);
             }
-            // O / l for this item's query rows
+            // O / l for this item's query rows, read out after the next item's first P store
+            rd_pend = true;
+            rd_dst = qi < t.ce ? out + (size_t)qi * D + t.h * DH : nullptr;
+            rd_inv = 1.0f / l;
+        }
+        if (rd_pend) {
             mbar_wait(&pvdone[x], (c - 1) & 1, status);
-            __syncwarp();
-            tc_fence_after();
-            uint32_t o[64];
-            tmem_ld32(tl + T_O + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-            tmem_ld32(tl + T_O + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
-            tmem_ld_wait();
-            if (qi < t.ce) {  // 32-byte stores: a warp instruction fills whole sectors
-                const float inv = 1.0f / l;
-                uint8_t *dst = reinterpret_cast<uint8_t *>(out + (size_t)qi * D + t.h * DH);
-#pragma unroll
-                for (int k8 = 0; k8 < 4; ++k8) {
-                    uint32_t wv[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        wv[e] = pack_bf16x2(__uint_as_float(o[16 * k8 + 2 * e]) * inv,
-                                            __uint_as_float(o[16 * k8 + 2 * e + 1]) * inv);
-                    st_global_v8(dst + 32 * k8, wv[0], wv[1], wv[2], wv[3], wv[4], wv[5], wv[6], wv[7]);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ofree[x]);
+            readout();
         }
     }
     __syncthreads();
