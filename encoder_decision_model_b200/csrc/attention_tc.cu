@@ -15,12 +15,12 @@
 //                   once per item into one of two buffers; K tiles (128 keys x
 //                   64) into a four-stage ring, each stage released when its
 //                   S products complete
-//   warp 10 lane 0  TMA producer of the V tiles: a four-stage ring, each stage
+//   warp 2 lane 0   TMA producer of the V tiles: a four-stage ring, each stage
 //                   released when its PV products complete
 //   warp 1          TMEM allocation; lane 0 issues tcgen05.mma:
 //                     S_x = Q_x K_j^T  (M 128, N 128, K 64; A, B from shared memory)
 //                     O_x += P_x V_j   (M 128, N 64, K 128; P from TMEM, V read MN-major)
-//   warps 2..5      softmax of Q tile 0, warps 6..9 of Q tile 1: one query
+//   warps 4..7      softmax of Q tile 0, warps 8..11 of Q tile 1: one query
 //                   row per thread (warp w reads TMEM lane quarter w % 4), all
 //                   128 keys of every tile.  The running max is kept lazily: O
 //                   and the row sum are rescaled only when the max grows by
@@ -30,7 +30,8 @@
 //                   2), so that the special-function unit, which bounds that
 //                   phase, is busy with one group while the other loads S,
 //                   takes the row max and hands P over.
-// TMEM columns: S_x at 128 x, O_x at 256 + 64 x, P_x at 384 + 64 x.
+// Warp group 0 (warps 0..3, warp 3 idle) hands registers to the two softmax warp groups
+// (setmaxnreg).  TMEM columns: S_x at 128 x, O_x at 256 + 64 x, P_x at 384 + 64 x.
 
 #include "common.cuh"
 #include "kernels.h"
@@ -54,8 +55,13 @@ constexpr int ATC_SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
 static_assert(ATC_SMEM <= 227 * 1024, "attention shared memory");
 constexpr uint32_t T_S = 0, T_O = 256, T_P = 384;
 constexpr float kLazy = 8.0f;    // log2 headroom before the running max is moved
-constexpr int V_WARP = 10;
-constexpr int ATC_THREADS = 11 * 32;
+constexpr int V_WARP = 2;
+constexpr int ATC_THREADS = 12 * 32;
+// Registers: the launch gives every thread ATC_REGS (the compiled count, checked on the host
+// before the first launch); warp group 0 (producers, MMA issue) gives up all but ATC_REGS_LOW and
+// the two softmax warp groups take ATC_REGS_HIGH, 128 x LOW + 256 x HIGH <= 384 x ATC_REGS.
+constexpr int ATC_REGS = 168, ATC_REGS_LOW = 120, ATC_REGS_HIGH = 192;
+static_assert(128 * ATC_REGS_LOW + 256 * ATC_REGS_HIGH <= ATC_THREADS * ATC_REGS, "register split");
 constexpr int BAR_G0_DONE = 1, BAR_G1_DONE = 2;  // named barriers of the softmax groups' hand-off
 }  // namespace
 
@@ -198,117 +204,120 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            uint32_t J = 0, it = 0;
-            for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++it) {
-                const AtcItem t = atc_item(q256, pb_row, cu, w);
-                const uint32_t qbuf = it & 1;
-                if (it >= 2) mbar_wait(&qfree[qbuf], ((it - 2) >> 1) & 1, status);
-                mbar_arrive_expect_tx(&qfull[qbuf], t.nx * Q_BYTES);
-                for (int x = 0; x < t.nx; ++x)
-                    tma_load_2d(smem + OFF_Q + (qbuf * 2 + x) * Q_BYTES, &tm, &qfull[qbuf], t.h * DH, t.q0 + x * TQ);
-                for (int j = 0; j < t.nt; ++j, ++J) {
-                    const uint32_t s = J % NK;
-                    if (J >= NK) mbar_wait(&kfree[s], ((J - NK) / NK) & 1, status);
-                    mbar_arrive_expect_tx(&kfull[s], KT_BYTES);
-                    tma_load_2d(smem + OFF_K + s * KT_BYTES, &tm, &kfull[s], D + t.h * DH, t.cs + j * TK);
+    if (warp < 4) {  // warp group 0: the TMA producers and the MMA issue
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(ATC_REGS_LOW));
+        if (warp == 0) {
+            if (lane == 0) {
+                uint32_t J = 0, it = 0;
+                for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++it) {
+                    const AtcItem t = atc_item(q256, pb_row, cu, w);
+                    const uint32_t qbuf = it & 1;
+                    if (it >= 2) mbar_wait(&qfree[qbuf], ((it - 2) >> 1) & 1, status);
+                    mbar_arrive_expect_tx(&qfull[qbuf], t.nx * Q_BYTES);
+                    for (int x = 0; x < t.nx; ++x)
+                        tma_load_2d(smem + OFF_Q + (qbuf * 2 + x) * Q_BYTES, &tm, &qfull[qbuf], t.h * DH, t.q0 + x * TQ);
+                    for (int j = 0; j < t.nt; ++j, ++J) {
+                        const uint32_t s = J % NK;
+                        if (J >= NK) mbar_wait(&kfree[s], ((J - NK) / NK) & 1, status);
+                        mbar_arrive_expect_tx(&kfull[s], KT_BYTES);
+                        tma_load_2d(smem + OFF_K + s * KT_BYTES, &tm, &kfull[s], D + t.h * DH, t.cs + j * TK);
+                    }
                 }
             }
-        }
-    } else if (warp == V_WARP) {
-        if (lane == 0) {
-            uint32_t J = 0;
-            for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
-                const AtcItem t = atc_item(q256, pb_row, cu, w);
-                for (int j = 0; j < t.nt; ++j, ++J) {
-                    const uint32_t s = J % NV;
-                    if (J >= NV) mbar_wait(&vfree[s], ((J - NV) / NV) & 1, status);
-                    mbar_arrive_expect_tx(&vfull[s], KT_BYTES);
-                    tma_load_2d(smem + OFF_V + s * KT_BYTES, &tm, &vfull[s], 2 * D + t.h * DH, t.cs + j * TK);
+        } else if (warp == V_WARP) {
+            if (lane == 0) {
+                uint32_t J = 0;
+                for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
+                    const AtcItem t = atc_item(q256, pb_row, cu, w);
+                    for (int j = 0; j < t.nt; ++j, ++J) {
+                        const uint32_t s = J % NV;
+                        if (J >= NV) mbar_wait(&vfree[s], ((J - NV) / NV) & 1, status);
+                        mbar_arrive_expect_tx(&vfull[s], KT_BYTES);
+                        tma_load_2d(smem + OFF_V + s * KT_BYTES, &tm, &vfull[s], 2 * D + t.h * DH, t.cs + j * TK);
+                    }
                 }
             }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(TK);
-            constexpr uint32_t idesc_pv = idesc_f16_f32(DH) | (1u << 16);  // P and V FP16; B (V) is MN-major
-            uint32_t J = 0, it = 0;
-            uint32_t cnt[2] = {0, 0};   // S tiles issued per Q tile, over all items
-            uint32_t uses[2] = {0, 0};  // items that used each Q tile
-            // O_x += P_x V for the K tile at ring position Jp: cx[x] is that tile's S count of Q tile
-            // x, `first` marks an item's first tile (O_x overwritten once the last item's O_x is read
-            // out: us[x] items had used it before)
-            auto issue_pv = [&](uint32_t Jp, int nx, const uint32_t (&cx)[2], bool first, const uint32_t (&us)[2]) {
-                const uint32_t s = Jp % NV;
-                mbar_wait(&vfull[s], (Jp / NV) & 1, status);
-                const uint32_t v_base = smem_u32(smem + OFF_V + s * KT_BYTES);
-                for (int x = 0; x < nx; ++x) {
-                    mbar_wait(&pready[x], cx[x] & 1, status);
-                    if (first && us[x] >= 1) mbar_wait(&ofree[x], (us[x] - 1) & 1, status);
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < TK / 16; ++ks)
-                        tc_mma_bf16_ts(tmem + T_O + 64 * x, tmem + T_P + 64 * x + 8 * ks,
-                                       sdesc_sw128(v_base + ks * 16 * 128), idesc_pv, (!first || ks != 0) ? 1u : 0u);
-                    tc_commit(&pvdone[x]);
-                }
-                tc_commit(&vfree[s]);
-            };
-            // The PV products of an item's last K tile are issued after the next item's first S
-            // products, so that the softmax groups find their next S tile ready when they finish
-            // the item, instead of after both groups' last exponentials.
-            bool pend = false;
-            uint32_t pJ = 0, pc[2] = {0, 0}, pu[2] = {0, 0};
-            int pnx = 0;
-            bool pfirst = false;
-            for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++it) {
-                const AtcItem t = atc_item(q256, pb_row, cu, w);
-                const uint32_t qbuf = it & 1;
-                mbar_wait(&qfull[qbuf], (it >> 1) & 1, status);
-                tc_fence_after();
-                const uint32_t J0 = J, c0[2] = {cnt[0], cnt[1]}, u0[2] = {uses[0], uses[1]};
-                for (int j = 0; j < t.nt; ++j, ++J) {
-                    const uint32_t s = J % NK;
-                    mbar_wait(&kfull[s], (J / NK) & 1, status);
-                    const uint32_t k_base = smem_u32(smem + OFF_K + s * KT_BYTES);
-                    for (int x = 0; x < t.nx; ++x) {
-                        const uint32_t c = cnt[x]++;
-                        if (c >= 1) mbar_wait(&sfree[x], (c - 1) & 1, status);  // S_x read out
+        } else if (warp == 1) {
+            if (lane == 0) {
+                constexpr uint32_t idesc_s = idesc_bf16_f32(TK);
+                constexpr uint32_t idesc_pv = idesc_f16_f32(DH) | (1u << 16);  // P and V FP16; B (V) is MN-major
+                uint32_t J = 0, it = 0;
+                uint32_t cnt[2] = {0, 0};   // S tiles issued per Q tile, over all items
+                uint32_t uses[2] = {0, 0};  // items that used each Q tile
+                // O_x += P_x V for the K tile at ring position Jp: cx[x] is that tile's S count of Q tile
+                // x, `first` marks an item's first tile (O_x overwritten once the last item's O_x is read
+                // out: us[x] items had used it before)
+                auto issue_pv = [&](uint32_t Jp, int nx, const uint32_t (&cx)[2], bool first, const uint32_t (&us)[2]) {
+                    const uint32_t s = Jp % NV;
+                    mbar_wait(&vfull[s], (Jp / NV) & 1, status);
+                    const uint32_t v_base = smem_u32(smem + OFF_V + s * KT_BYTES);
+                    for (int x = 0; x < nx; ++x) {
+                        mbar_wait(&pready[x], cx[x] & 1, status);
+                        if (first && us[x] >= 1) mbar_wait(&ofree[x], (us[x] - 1) & 1, status);
                         tc_fence_after();
-                        const uint32_t q_base = smem_u32(smem + OFF_Q + (qbuf * 2 + x) * Q_BYTES);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_mma_bf16(tmem + T_S + TK * x, sdesc_sw128(q_base + kk * 32),
-                                        sdesc_sw128(k_base + kk * 32), idesc_s, kk != 0);
-                        tc_commit(&sfull[x]);
+    #pragma unroll
+                        for (int ks = 0; ks < TK / 16; ++ks)
+                            tc_mma_bf16_ts(tmem + T_O + 64 * x, tmem + T_P + 64 * x + 8 * ks,
+                                           sdesc_sw128(v_base + ks * 16 * 128), idesc_pv, (!first || ks != 0) ? 1u : 0u);
+                        tc_commit(&pvdone[x]);
                     }
-                    tc_commit(&kfree[s]);
-                    if (j == t.nt - 1) tc_commit(&qfree[qbuf]);
-                    if (j == 0 && pend) {
-                        issue_pv(pJ, pnx, pc, pfirst, pu);
-                        pend = false;
+                    tc_commit(&vfree[s]);
+                };
+                // The PV products of an item's last K tile are issued after the next item's first S
+                // products, so that the softmax groups find their next S tile ready when they finish
+                // the item, instead of after both groups' last exponentials.
+                bool pend = false;
+                uint32_t pJ = 0, pc[2] = {0, 0}, pu[2] = {0, 0};
+                int pnx = 0;
+                bool pfirst = false;
+                for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++it) {
+                    const AtcItem t = atc_item(q256, pb_row, cu, w);
+                    const uint32_t qbuf = it & 1;
+                    mbar_wait(&qfull[qbuf], (it >> 1) & 1, status);
+                    tc_fence_after();
+                    const uint32_t J0 = J, c0[2] = {cnt[0], cnt[1]}, u0[2] = {uses[0], uses[1]};
+                    for (int j = 0; j < t.nt; ++j, ++J) {
+                        const uint32_t s = J % NK;
+                        mbar_wait(&kfull[s], (J / NK) & 1, status);
+                        const uint32_t k_base = smem_u32(smem + OFF_K + s * KT_BYTES);
+                        for (int x = 0; x < t.nx; ++x) {
+                            const uint32_t c = cnt[x]++;
+                            if (c >= 1) mbar_wait(&sfree[x], (c - 1) & 1, status);  // S_x read out
+                            tc_fence_after();
+                            const uint32_t q_base = smem_u32(smem + OFF_Q + (qbuf * 2 + x) * Q_BYTES);
+    #pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                tc_mma_bf16(tmem + T_S + TK * x, sdesc_sw128(q_base + kk * 32),
+                                            sdesc_sw128(k_base + kk * 32), idesc_s, kk != 0);
+                            tc_commit(&sfull[x]);
+                        }
+                        tc_commit(&kfree[s]);
+                        if (j == t.nt - 1) tc_commit(&qfree[qbuf]);
+                        if (j == 0 && pend) {
+                            issue_pv(pJ, pnx, pc, pfirst, pu);
+                            pend = false;
+                        }
+                        if (j >= 1) {
+                            const uint32_t cx[2] = {c0[0] + j - 1, c0[1] + j - 1};
+                            issue_pv(J0 + j - 1, t.nx, cx, j == 1, u0);
+                        }
                     }
-                    if (j >= 1) {
-                        const uint32_t cx[2] = {c0[0] + j - 1, c0[1] + j - 1};
-                        issue_pv(J0 + j - 1, t.nx, cx, j == 1, u0);
-                    }
+                    pend = true;
+                    pJ = J0 + t.nt - 1;
+                    pnx = t.nx;
+                    pc[0] = c0[0] + t.nt - 1;
+                    pc[1] = c0[1] + t.nt - 1;
+                    pfirst = t.nt == 1;
+                    pu[0] = u0[0];
+                    pu[1] = u0[1];
+                    for (int x = 0; x < t.nx; ++x) ++uses[x];
                 }
-                pend = true;
-                pJ = J0 + t.nt - 1;
-                pnx = t.nx;
-                pc[0] = c0[0] + t.nt - 1;
-                pc[1] = c0[1] + t.nt - 1;
-                pfirst = t.nt == 1;
-                pu[0] = u0[0];
-                pu[1] = u0[1];
-                for (int x = 0; x < t.nx; ++x) ++uses[x];
+                if (pend) issue_pv(pJ, pnx, pc, pfirst, pu);
             }
-            if (pend) issue_pv(pJ, pnx, pc, pfirst, pu);
         }
     } else {
-        const int x = (warp - 2) >> 2;         // Q tile of this warp group
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(ATC_REGS_HIGH));
+        const int x = (warp - 4) >> 2;         // Q tile of this warp group
         const int r = (warp & 3) * 32 + lane;  // query row inside the tile = TMEM lane
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float sl2 = 0.125f * 1.4426950408889634f;
@@ -506,6 +515,12 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
 }
 
 cudaError_t attn_tc_init_attributes() {
+    // The register split above assumes the compiled count: refuse to run on any other, since a
+    // softmax warp group asking for more registers than the launch holds would wait forever.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, k_attn_tc);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != ATC_REGS) return cudaErrorInvalidKernelImage;
     return cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, ATC_SMEM);
 }
 
